@@ -1,0 +1,455 @@
+"""Routing throughput of the B200 sigmoid router + Exact Quantile Balancing.
+
+One step = the whole hot path over one batch: router logits (tcgen05 GEMM),
+bias add + top-K + sigmoid gates + token bias, expert counts + stable
+permutation, and one exact EQB bias update.  Default workload: the
+million-token Kolibri-shaped batch (N = 1,048,576, d = 2560, E = 384, K = 6,
+Zipf(1.1) expert offsets), inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): the path has no exchange step on one
+node, so each rank runs an independent replica of the batch ("replicas
+only", weak scaling); the reported value is all ranks' tokens over the
+slowest rank's device time.
+
+``--impl reference`` times the CPU oracle on the host cores (bounded sample
+of the same workload per step); it is the slow baseline, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from expert_load_balancing_b200 import binding as B  # noqa: E402
+from expert_load_balancing_b200 import workloads  # noqa: E402
+
+METRIC = "routed tokens/sec (GEMM+top-K+permute+EQB) at N=1M, E=384, K=6; % of roofline"
+UNIT = "routed tokens/s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def algorithmic_work(N, d, E, K):
+    """FLOPs and bytes a perfect implementation must spend per step.
+
+    GEMM 2 N d E FLOP.  Bytes: x read (2Nd), Z written once and read once
+    (8NE), ids+gates written (8NK), perm+inv written (8NK), alpha (4N), W
+    once (2Ed); counts/offsets/beta are negligible."""
+    flops = 2.0 * N * d * E
+    bytes_ = 2.0 * N * d + 8.0 * N * E + 16.0 * N * K + 4.0 * N + 2.0 * E * d
+    return flops, bytes_
+
+
+def gemm_bytes(N, d, E):
+    """Algorithmic bytes of the logits GEMM alone: x in, Z out, W once."""
+    return 2.0 * N * d + 4.0 * N * E + 2.0 * E * d
+
+
+def launches_per_step(N, E, K):
+    """Kernels of ours per step: logits 1, top-K 1, permute 1 or 3, EQB 3 or 6."""
+    permute = 1 if N * K <= 4096 else 3
+    eqb = 3 if N <= 16384 else 6
+    return 1 + 1 + permute + eqb
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling during the timed region (SM clock, reasons)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- our path
+
+class RouterStep:
+    """Buffers and the four calls of one step, all on one stream."""
+
+    def __init__(self, wl, device, seed=0):
+        self.wl = wl
+        N, d, E, K = wl.N, wl.d, wl.E, wl.K
+        g = torch.Generator(device=device)
+        g.manual_seed(1234 + seed)
+        self.x = torch.empty((N, d), dtype=torch.bfloat16, device=device)
+        rows = 65536
+        for r0 in range(0, N, rows):
+            r1 = min(N, r0 + rows)
+            self.x[r0:r1] = torch.randn((r1 - r0, d), generator=g, device=device).to(torch.bfloat16)
+        if wl.offsets != "none":
+            self.x[:, 0] = 1.0
+        self.w = workloads.make_w(wl).to(device)
+        self.beta0 = workloads.make_beta(wl).to(device)
+        self.beta = self.beta0.clone()
+        self.z = torch.empty((N, E), dtype=torch.float32, device=device)
+        self.ids = torch.empty((N, K), dtype=torch.int32, device=device)
+        self.gates = torch.empty((N, K), dtype=torch.float32, device=device)
+        self.alpha = torch.empty((N,), dtype=torch.float32, device=device)
+        self.counts = torch.empty((E,), dtype=torch.int32, device=device)
+        self.offsets = torch.empty((E + 1,), dtype=torch.int64, device=device)
+        self.perm = torch.empty((N * K,), dtype=torch.int32, device=device)
+        self.inv = torch.empty((N * K,), dtype=torch.int32, device=device)
+        self.q = torch.empty((E,), dtype=torch.float32, device=device)
+        self.ws_perm = B.workspace(B.KOLIBRI_OP_PERMUTE, N, E, K, device)
+        self.ws_eqb = B.workspace(B.KOLIBRI_OP_EQB, N, E, K, device)
+
+    def run(self, stream, events=None):
+        wl = self.wl
+        if events:
+            events[0].record(stream)
+        B.kolibri_router_logits(self.x, self.w, self.z, stream=stream)
+        if events:
+            events[1].record(stream)
+        B.kolibri_router_topk(self.z, self.beta, wl.K, self.ids, self.gates, self.alpha,
+                              stream=stream)
+        if events:
+            events[2].record(stream)
+        B.kolibri_expert_permute(self.ids, wl.E, self.ws_perm, self.counts, self.offsets,
+                                 self.perm, self.inv, stream=stream)
+        if events:
+            events[3].record(stream)
+        B.kolibri_eqb_update(self.z, self.alpha, self.beta, wl.K, self.ws_eqb, self.q,
+                             stream=stream)
+        if events:
+            events[4].record(stream)
+
+
+def run_ours(args, rank, world, local_rank):
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    B.load()
+    wl = workloads.WORKLOADS[args.workload]
+    N, d, E, K = wl.N, wl.d, wl.E, wl.K
+    step = RouterStep(wl, device, seed=rank)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step.run(stream)
+    stream.synchronize()
+    st = B.kolibri_device_status(stream)
+    if st != B.KOLIBRI_OK:
+        raise RuntimeError(f"device status after warm-up: {B.status_string(st)}")
+
+    # ---- timed region: device time, CUDA events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    gpu_id = visible.split(",")[local_rank] if visible else str(local_rank)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    for i in range(args.steps):
+        step.run(stream, ev[i])
+    t1.record(stream)
+    t1.synchronize()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t0.elapsed_time(t1)
+    stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)]
+                         for i in range(args.steps)]).mean(axis=0)
+    st = B.kolibri_device_status(stream)
+    if st != B.KOLIBRI_OK:
+        raise RuntimeError(f"device status after timing: {B.status_string(st)}")
+
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, step, stream, device, world)
+
+    if rank != 0:
+        return None
+    peaks = _peaks()
+    flops, bytes_ = algorithmic_work(N, d, E, K)
+    roof_ms = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    gemm_ms = float(stage_ms[0])
+    gemm_tflops = 2.0 * N * d * E / (gemm_ms * 1e-3) / 1e12
+    peak_t = peaks["bf16_tflops_sustained"]
+    traffic = _traffic_from_profile()
+    line = {
+        "metric": METRIC,
+        "value": world * N / (ms_per_step * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16/fp32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "N": N, "d": d, "E": E, "K": K, "offsets": wl.offsets,
+                   "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (x %.2f GB, Z %.2f GB)" % (2 * N * d / 1e9, 4 * N * E / 1e9)},
+        "roofline": {"bound": "tensor", "kernel": "router_gemm_kernel",
+                     "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / peak_t, "traffic": traffic,
+                     "peak_kind": f"bf16 sustained, of {peaks['source']}"},
+        "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ms_per_step,
+                          "flops": flops, "bytes": bytes_,
+                          "peaks": f"bf16 burst {peaks['bf16_tflops']} TF/s, HBM {peaks['hbm_gbs']} GB/s, of {peaks['source']}"},
+        "stages_ms": {"logits": gemm_ms, "topk": float(stage_ms[1]),
+                      "permute": float(stage_ms[2]), "eqb": float(stage_ms[3])},
+        "gpu_launches": launches_per_step(N, E, K) * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    return line
+
+
+def _traffic_from_profile():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if current."""
+    path = os.path.join(ROOT, "profiles", "router_gemm_traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p.get("dram_bytes_per_launch_full")
+    except (OSError, ValueError):
+        return None
+
+
+def run_e2e(args, step, stream, device, world):
+    """Same step through the public API with the step's inputs copied in
+    from pinned host memory and its routing result read back, every step."""
+    wl = step.wl
+    N, d, E, K = wl.N, wl.d, wl.E, wl.K
+    x_h = torch.empty((N, d), dtype=torch.bfloat16, pin_memory=True)
+    x_h.copy_(step.x, non_blocking=False)
+    w_h = step.w.cpu().pin_memory()
+    b_h = step.beta0.cpu().pin_memory()
+    ids_h = torch.empty((N, K), dtype=torch.int32, pin_memory=True)
+    gates_h = torch.empty((N, K), dtype=torch.float32, pin_memory=True)
+    counts_h = torch.empty((E,), dtype=torch.int32, pin_memory=True)
+    beta_h = torch.empty((E,), dtype=torch.float32, pin_memory=True)
+    h2d = x_h.numel() * 2 + w_h.numel() * 2 + b_h.numel() * 4
+    d2h = ids_h.numel() * 4 + gates_h.numel() * 4 + counts_h.numel() * 4 + beta_h.numel() * 4
+
+    def one():
+        with torch.cuda.stream(stream):
+            step.x.copy_(x_h, non_blocking=True)
+            step.w.copy_(w_h, non_blocking=True)
+            step.beta.copy_(b_h, non_blocking=True)
+            step.run(stream)
+            ids_h.copy_(step.ids, non_blocking=True)
+            gates_h.copy_(step.gates, non_blocking=True)
+            counts_h.copy_(step.counts, non_blocking=True)
+            beta_h.copy_(step.beta, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        one()
+    stream.synchronize()
+    n = args.e2e_steps
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        one()
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b) / n
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    return {"value": world * N / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "steps": n,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------- the oracle
+
+def _oracle_step(oracle, wl, n_rows, beta):
+    """One oracle pass of the whole path over the first n_rows tokens."""
+    x = workloads.bf16_bits(workloads.x_rows(wl, np.arange(n_rows)))
+    w = workloads.bf16_bits(workloads.make_w(wl))
+    t = time.perf_counter()
+    z = oracle.router_logits(x, w)
+    ids, gates, alpha = oracle.select(z, beta, wl.K)
+    oracle.permute(ids, wl.E)
+    v = oracle.column_quantiles(z, alpha, oracle.eqb_target_rank(n_rows, wl.K, wl.E))
+    oracle.eqb_bias(v)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(wl, seconds):
+    import oracle
+    oracle.build()
+    beta = workloads.make_beta(wl).numpy()
+    t_cal = _oracle_step(oracle, wl, 256, beta)
+    n_rows = int(max(256, min(wl.N, 256 * seconds / max(t_cal, 1e-3))))
+    n_rows = (n_rows // 256) * 256
+    t = _oracle_step(oracle, wl, n_rows, beta)
+    return {"value": n_rows / t, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"first {n_rows} tokens of {wl.name} (full d, E, K), one pass of logits, "
+                      f"top-K, permutation and the EQB update over that sample; {t:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    wl = workloads.WORKLOADS[args.workload]
+    beta = workloads.make_beta(wl).numpy()
+    t_cal = _oracle_step(oracle, wl, 256, beta)
+    # size each step so the whole run takes a few minutes at most
+    total_steps = args.warmup + args.steps
+    per_step = min(20.0, 150.0 / max(total_steps, 1))
+    n_rows = int(max(256, min(wl.N, 256 * per_step / max(t_cal, 1e-3))))
+    n_rows = (n_rows // 256) * 256
+    for _ in range(args.warmup):
+        _oracle_step(oracle, wl, 256, beta)
+    times = [_oracle_step(oracle, wl, n_rows, beta) for _ in range(args.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    value = n_rows / (ms * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64/fp32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "N": wl.N, "d": wl.d, "E": wl.E, "K": wl.K,
+                   "parallelism": "host cores", "sample_tokens_per_step": n_rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"first {n_rows} tokens of {wl.name} per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="kolibri_n1m", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

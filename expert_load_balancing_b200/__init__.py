@@ -1,1 +1,17 @@
-"""B200-native sigmoid MoE router with Exact Quantile Balancing."""
+"""B200-native sigmoid MoE router with Exact Quantile Balancing (EQB).
+
+The routing path runs in ``libkolibri_router.so`` (hand-written sm_100a CUDA
+behind the C ABI in ``include/kolibri_router.h``).  ``binding`` is the thin
+ctypes layer with the same call names; ``workloads`` draws seeded synthetic
+inputs; ``build`` compiles the library in-tree.
+"""
+from . import binding  # noqa: F401  (loads the library lazily, on first call)
+from .binding import (  # noqa: F401
+    KolibriError,
+    kolibri_device_status,
+    kolibri_eqb_update,
+    kolibri_expert_permute,
+    kolibri_router_logits,
+    kolibri_router_topk,
+    kolibri_workspace_bytes,
+)

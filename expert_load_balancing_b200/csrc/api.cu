@@ -1,0 +1,123 @@
+// api.cu -- the extern "C" boundary declared in include/kolibri_router.h:
+// argument validation, workspace sizing and the device status word.
+#include <cstdint>
+
+#include "launch.h"
+#include "common.cuh"
+
+namespace kolibri {
+
+__device__ unsigned int g_status = 0u;
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0u; }
+
+kolibri_status check_ek(int64_t N, int32_t E, int32_t K) {
+  if (N < 1 || E < 1 || K < 1) return KOLIBRI_ERR_INVALID_ARG;
+  if (K >= E) return KOLIBRI_ERR_INVALID_ARG;
+  if (E > KOLIBRI_MAX_EXPERTS || K > KOLIBRI_MAX_TOPK || (E % 4) != 0)
+    return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (N * static_cast<int64_t>(K) >= (static_cast<int64_t>(1) << 31))
+    return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  return KOLIBRI_OK;
+}
+
+kolibri_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KOLIBRI_OK : KOLIBRI_ERR_CUDA; }
+
+}  // namespace
+}  // namespace kolibri
+
+using namespace kolibri;
+
+extern "C" {
+
+const char* kolibri_status_string(kolibri_status s) {
+  switch (s) {
+    case KOLIBRI_OK: return "KOLIBRI_OK";
+    case KOLIBRI_ERR_INVALID_ARG: return "KOLIBRI_ERR_INVALID_ARG";
+    case KOLIBRI_ERR_UNSUPPORTED_SHAPE: return "KOLIBRI_ERR_UNSUPPORTED_SHAPE";
+    case KOLIBRI_ERR_WORKSPACE_TOO_SMALL: return "KOLIBRI_ERR_WORKSPACE_TOO_SMALL";
+    case KOLIBRI_ERR_CUDA: return "KOLIBRI_ERR_CUDA";
+    case KOLIBRI_ERR_TIMEOUT: return "KOLIBRI_ERR_TIMEOUT";
+    case KOLIBRI_ERR_DEVICE: return "KOLIBRI_ERR_DEVICE";
+  }
+  return "KOLIBRI_ERR_UNKNOWN";
+}
+
+size_t kolibri_workspace_bytes(int op, int64_t N, int32_t E, int32_t K) {
+  if (check_ek(N, E, K) != KOLIBRI_OK) return 0;
+  if (op == KOLIBRI_OP_PERMUTE) return permute_layout(N, E, K).total;
+  if (op == KOLIBRI_OP_EQB) return eqb_layout(N, E, K).total;
+  return 0;
+}
+
+kolibri_status kolibri_router_logits(const void* x, const void* w, float* z, int64_t N, int32_t d,
+                                     int32_t E, void* stream) {
+  if (!x || !w || !z) return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(z)) return KOLIBRI_ERR_INVALID_ARG;
+  if (N < 1 || d < 1 || E < 1) return KOLIBRI_ERR_INVALID_ARG;
+  if (d % 64 != 0 || E % 16 != 0 || E > KOLIBRI_MAX_EXPERTS) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (N >= (static_cast<int64_t>(1) << 31)) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(launch_router_logits(x, w, z, N, d, E, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_router_topk(const float* z, const float* bias, int64_t N, int32_t E,
+                                   int32_t K, int32_t* ids, float* gates, float* alpha,
+                                   void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!z || !ids || !gates) return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(z) || (bias && !aligned16(bias))) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(
+      launch_topk(z, bias, N, E, K, ids, gates, alpha, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_expert_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K,
+                                      int32_t* counts, int64_t* offsets, int32_t* perm,
+                                      int32_t* inv, void* ws, size_t ws_bytes, void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!ids || !counts || !offsets || !perm) return KOLIBRI_ERR_INVALID_ARG;
+  const PermuteLayout L = permute_layout(N, E, K);
+  if (!L.single_cta) {
+    if (!ws) return KOLIBRI_ERR_INVALID_ARG;
+    if (ws_bytes < L.total) return KOLIBRI_ERR_WORKSPACE_TOO_SMALL;
+  }
+  return from_cuda(launch_permute(ids, N, E, K, counts, offsets, perm, inv, ws,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_update(const float* z, const float* alpha, float* bias, int64_t N,
+                                  int32_t E, int32_t K, float* quantiles, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!z || !bias || !ws) return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(z) || !aligned16(bias) || !aligned16(ws)) return KOLIBRI_ERR_INVALID_ARG;
+  if (ws_bytes < eqb_layout(N, E, K).total) return KOLIBRI_ERR_WORKSPACE_TOO_SMALL;
+  return from_cuda(
+      launch_eqb(z, alpha, bias, N, E, K, quantiles, ws, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KOLIBRI_ERR_CUDA;
+  unsigned int v = 0u, zero = 0u;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return KOLIBRI_ERR_CUDA;
+  if (v != 0u && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
+    return KOLIBRI_ERR_CUDA;
+  if (v & kStatusTimeout) return KOLIBRI_ERR_TIMEOUT;
+  if (v & kStatusBadInput) return KOLIBRI_ERR_DEVICE;
+  return KOLIBRI_OK;
+}
+
+}  // extern "C"

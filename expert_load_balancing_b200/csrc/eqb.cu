@@ -1,0 +1,298 @@
+// eqb.cu -- Exact Quantile Balancing update on one GPU.
+//
+// Method ("Kolibri Pre-Training from Scratch", 7.1 update rule, 7.2 order
+// of operations, 7.3 exact quantile by radix selection):
+//   v_e    = Q_m(Z_:,e + alpha)        (m+1)-th largest, m = floor(N K / E)
+//   beta_e = -v_e - mean_e'(-v_e')      (centred)
+//
+// The pages select the exact order statistic with radix passes whose digit
+// histograms are summed over ranks.  On one B200 the column lives in one HBM,
+// so the design reads Z once instead of once per digit:
+//   1. keys of Z + alpha at S strided sample rows (S = N for N <= 16384:
+//      then the sample IS the column and step 3 selects v directly);
+//   2. per expert, two sample order statistics bracket the target rank with
+//      a margin of six binomial standard deviations;
+//   3. one full pass counts the keys above the bracket and gathers the keys
+//      inside it;
+//   4. per expert, the target is inside the bracket iff
+//      above <= m < above + inside; then v is the (m - above)-th largest
+//      gathered key, found by radix selection (11-bit digits, shared-memory
+//      histograms, scanned from the top bin as on the pages);
+//   5. any expert whose bracket missed (or overflowed the gather buffer)
+//      falls back to radix selection over its whole column.
+// Every path returns the exact order statistic; the bracket only decides
+// how much of the column the radix passes must look at.
+#include <cmath>
+
+#include "launch.h"
+#include "common.cuh"
+
+namespace kolibri {
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+constexpr int kSelThreads = 512;
+constexpr int kDigitBits = 11;
+constexpr int kBins = 1 << kDigitBits;
+
+struct SelectSmem {
+  uint32_t hist[kBins];
+  uint32_t red_min[kSelThreads / kWarp];
+  uint32_t red_max[kSelThreads / kWarp];
+  uint32_t bcast[4];
+};
+
+// Exact (rank+1)-th largest key of {key_at(i) : i < n}, rank < n.
+// Skips the bits common to the minimum and maximum key, then resolves the
+// remaining bits most significant first, kDigitBits per pass.  Every thread
+// of the block must call it; the result is returned to all of them.
+template <class KeyAt>
+__device__ uint32_t block_select_desc(KeyAt key_at, int64_t n, int64_t rank, SelectSmem& sm) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
+  uint32_t mn = 0xffffffffu, mx = 0u;
+  for (int64_t i = tid; i < n; i += blockDim.x) {
+    uint32_t k = key_at(i);
+    mn = k < mn ? k : mn;
+    mx = k > mx ? k : mx;
+  }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0) {
+    sm.red_min[warp] = mn;
+    sm.red_max[warp] = mx;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t a = lane < nwarps ? sm.red_min[lane] : 0xffffffffu;
+    uint32_t b = lane < nwarps ? sm.red_max[lane] : 0u;
+    a = __reduce_min_sync(0xffffffffu, a);
+    b = __reduce_max_sync(0xffffffffu, b);
+    if (lane == 0) {
+      sm.bcast[0] = a;
+      sm.bcast[1] = b;
+    }
+  }
+  __syncthreads();
+  mn = sm.bcast[0];
+  mx = sm.bcast[1];
+  __syncthreads();
+  if (mn == mx) return mn;
+  int bits_left = 32 - __clz(static_cast<int>(mn ^ mx));  // lowest bits that still differ
+  uint32_t prefix = (bits_left == 32) ? 0u : (mx & ~((1u << bits_left) - 1u));
+  int64_t r = rank;
+  while (bits_left > 0) {
+    const int nb = bits_left < kDigitBits ? bits_left : kDigitBits;
+    const int shift = bits_left - nb;
+    const int nbins = 1 << nb;
+    const uint32_t hi_mask = (shift + nb >= 32) ? 0u : (0xffffffffu << (shift + nb));
+    for (int b = tid; b < nbins; b += blockDim.x) sm.hist[b] = 0u;
+    __syncthreads();
+    for (int64_t i = tid; i < n; i += blockDim.x) {
+      uint32_t k = key_at(i);
+      if ((k & hi_mask) == (prefix & hi_mask)) atomicAdd(&sm.hist[(k >> shift) & (nbins - 1)], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // bins are scanned from the top (largest keys first)
+      const int per = (nbins + 31) / 32;
+      // lane 0 owns the top `per` bins, lane 1 the next, ...
+      const int top = nbins - 1 - lane * per;
+      uint32_t part = 0;
+      for (int q = 0; q < per; ++q) {
+        int b = top - q;
+        if (b >= 0) part += sm.hist[b];
+      }
+      // exclusive prefix over lanes (in scan order)
+      uint32_t incl = part;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      uint32_t excl = incl - part;
+      bool mine = static_cast<int64_t>(excl) <= r && r < static_cast<int64_t>(incl);
+      if (mine) {
+        int64_t rr = r - excl;
+        int b = top;
+        for (int q = 0; q < per; ++q, --b) {
+          uint32_t c = sm.hist[b];
+          if (rr < static_cast<int64_t>(c)) break;
+          rr -= c;
+        }
+        sm.bcast[2] = static_cast<uint32_t>(b);
+        sm.bcast[3] = static_cast<uint32_t>(rr);
+      }
+    }
+    __syncthreads();
+    prefix |= sm.bcast[2] << shift;
+    r = sm.bcast[3];
+    bits_left = shift;
+    __syncthreads();
+  }
+  return prefix;
+}
+
+// Step 2 (or the whole selection when the sample is the column).
+__global__ void __launch_bounds__(kSelThreads) sample_select_kernel(
+    const uint32_t* __restrict__ sample, int64_t S, int64_t m_exact, int64_t r_hi, int64_t r_lo,
+    bool exact, float* __restrict__ v, uint32_t* __restrict__ lo, uint32_t* __restrict__ hi) {
+  __shared__ SelectSmem sm;
+  const int e = blockIdx.x;
+  const uint32_t* keys = sample + static_cast<int64_t>(e) * S;
+  auto at = [keys](int64_t i) { return __ldg(keys + i); };
+  if (exact) {
+    uint32_t k = block_select_desc(at, S, m_exact, sm);
+    if (threadIdx.x == 0) v[e] = key_to_float(k);
+  } else {
+    uint32_t kh = block_select_desc(at, S, r_hi, sm);
+    uint32_t kl = block_select_desc(at, S, r_lo, sm);
+    if (threadIdx.x == 0) {
+      hi[e] = kh;
+      lo[e] = kl;
+    }
+  }
+}
+
+// Step 4.
+__global__ void __launch_bounds__(kSelThreads) bracket_select_kernel(
+    const uint32_t* __restrict__ cand, const uint32_t* __restrict__ cnt,
+    const uint32_t* __restrict__ above, int64_t cap, int64_t m, float* __restrict__ v,
+    uint32_t* __restrict__ flag) {
+  __shared__ SelectSmem sm;
+  const int e = blockIdx.x;
+  const int64_t c = cnt[e], ab = above[e];
+  const bool ok = c <= cap && ab <= m && m < ab + c;
+  if (!ok) {
+    if (threadIdx.x == 0) flag[e] = 1u;
+    return;
+  }
+  const uint32_t* keys = cand + static_cast<int64_t>(e) * cap;
+  auto at = [keys](int64_t i) { return __ldg(keys + i); };
+  uint32_t k = block_select_desc(at, c, m - ab, sm);
+  if (threadIdx.x == 0) {
+    v[e] = key_to_float(k);
+    flag[e] = 0u;
+  }
+}
+
+// Step 5: radix selection over the whole column of the flagged experts.
+__global__ void __launch_bounds__(kSelThreads) column_fallback_kernel(
+    const float* __restrict__ z, const float* __restrict__ alpha, int64_t N, int E, int64_t m,
+    const uint32_t* __restrict__ flag, float* __restrict__ v) {
+  __shared__ SelectSmem sm;
+  const int e = blockIdx.x;
+  if (flag[e] == 0u) return;
+  auto at = [z, alpha, E, e](int64_t t) {
+    return order_key(__fadd_rn(__ldg(z + t * E + e), __ldg(alpha + t)));
+  };
+  uint32_t k = block_select_desc(at, N, m, sm);
+  if (threadIdx.x == 0) v[e] = key_to_float(k);
+}
+
+// a5: beta = -v, centred.  fp64 sum in ascending expert order (one thread),
+// mean rounded once to fp32, subtraction in fp32.
+__global__ void bias_update_kernel(const float* __restrict__ v, int E, float* __restrict__ bias,
+                                   float* __restrict__ quantiles) {
+  __shared__ float mean_s;
+  if (threadIdx.x == 0) {
+    double sum = 0.0;
+    for (int e = 0; e < E; ++e) sum = __dadd_rn(sum, static_cast<double>(-v[e]));
+    mean_s = __double2float_rn(__ddiv_rn(sum, static_cast<double>(E)));
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float ve = v[e];
+    bias[e] = __fsub_rn(-ve, mean_s);
+    if (quantiles) quantiles[e] = ve;
+  }
+}
+
+}  // namespace
+
+EqbLayout eqb_layout(int64_t N, int32_t E, int32_t K) {
+  (void)K;
+  EqbLayout L;
+  L.exact_small = N <= kSampleMax;
+  L.S = L.exact_small ? N : kSampleMax;
+  L.stride = L.exact_small ? 1 : N / L.S;
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.off_sample = take(sizeof(uint32_t) * static_cast<size_t>(E) * static_cast<size_t>(L.S));
+  L.off_lo = take(sizeof(uint32_t) * E);
+  L.off_hi = take(sizeof(uint32_t) * E);
+  L.off_above = take(sizeof(uint32_t) * E);
+  L.off_cnt = take(sizeof(uint32_t) * E);
+  L.off_flag = take(sizeof(uint32_t) * E);
+  L.off_v = take(sizeof(float) * E);
+  if (!L.exact_small) {
+    L.off_cand = take(sizeof(uint32_t) * static_cast<size_t>(E) * static_cast<size_t>(kCandCap));
+    L.off_alpha = take(sizeof(float) * static_cast<size_t>(N));
+  }
+  L.total = off;
+  return L;
+}
+
+cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
+                       int32_t K, float* quantiles, void* ws, cudaStream_t s) {
+  const EqbLayout L = eqb_layout(N, E, K);
+  char* base = static_cast<char*>(ws);
+  auto u32 = [base](size_t off) { return reinterpret_cast<uint32_t*>(base + off); };
+  uint32_t* sample = u32(L.off_sample);
+  uint32_t* lo = u32(L.off_lo);
+  uint32_t* hi = u32(L.off_hi);
+  uint32_t* above = u32(L.off_above);
+  uint32_t* cnt = u32(L.off_cnt);
+  uint32_t* flag = u32(L.off_flag);
+  float* v = reinterpret_cast<float*>(base + L.off_v);
+  const int64_t m = (N * static_cast<int64_t>(K)) / E;
+
+  // alpha is computed from bias_in before bias is overwritten (stream order)
+  cudaError_t err = launch_eqb_sample(z, alpha, alpha ? nullptr : bias, N, E, K, L.S, L.stride,
+                                      sample, s);
+  if (err != cudaSuccess) return err;
+
+  if (L.exact_small) {
+    sample_select_kernel<<<E, kSelThreads, 0, s>>>(sample, L.S, m, 0, 0, true, v, lo, hi);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  } else {
+    // bracket ranks in the sample, descending order: the target sits at
+    // about q*S with q = (m+1)/N; margin 6 binomial standard deviations
+    const double q = static_cast<double>(m + 1) / static_cast<double>(N);
+    const double center = q * static_cast<double>(L.S);
+    const double sd = std::sqrt(center * (1.0 - q));
+    const int64_t margin = static_cast<int64_t>(std::ceil(6.0 * sd)) + 8;
+    int64_t r_hi = static_cast<int64_t>(std::floor(center)) - margin;
+    int64_t r_lo = static_cast<int64_t>(std::ceil(center)) + margin;
+    if (r_hi < 0) r_hi = 0;
+    if (r_lo > L.S - 1) r_lo = L.S - 1;
+    err = cudaMemsetAsync(base + L.off_above, 0, L.off_v - L.off_above, s);  // above, cnt, flag
+    if (err != cudaSuccess) return err;
+    sample_select_kernel<<<E, kSelThreads, 0, s>>>(sample, L.S, 0, r_hi, r_lo, false, v, lo, hi);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    float* alpha_ws = reinterpret_cast<float*>(base + L.off_alpha);
+    uint32_t* cand = u32(L.off_cand);
+    err = launch_eqb_window_pass(z, alpha, alpha ? nullptr : bias, alpha ? nullptr : alpha_ws, N,
+                                 E, K, lo, hi, above, cnt, cand, kCandCap, s);
+    if (err != cudaSuccess) return err;
+    bracket_select_kernel<<<E, kSelThreads, 0, s>>>(cand, cnt, above, kCandCap, m, v, flag);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    column_fallback_kernel<<<E, kSelThreads, 0, s>>>(z, alpha ? alpha : alpha_ws, N, E, m, flag,
+                                                     v);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  bias_update_kernel<<<1, 512, 0, s>>>(v, E, bias, quantiles);
+  return cudaGetLastError();
+}
+
+}  // namespace kolibri

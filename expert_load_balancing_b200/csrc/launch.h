@@ -1,0 +1,66 @@
+// launch.h -- host launchers of the router kernels (internal to the library).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace kolibri {
+
+// Row sample used by the EQB bracket: S rows t = s * stride, s < S.
+constexpr int64_t kSampleMax = 16384;
+// Candidate capacity per expert in the bracketed full pass.
+constexpr int64_t kCandCap = 65536;
+
+struct EqbLayout {
+  int64_t S = 0, stride = 1;
+  bool exact_small = false;   // S == N: the sample is the whole column
+  size_t off_sample = 0;      // u32 [E][S]   keys of Z + alpha at sampled rows
+  size_t off_lo = 0;          // u32 [E]      lower bracket key
+  size_t off_hi = 0;          // u32 [E]      upper bracket key
+  size_t off_above = 0;       // u32 [E]      keys above the bracket
+  size_t off_cnt = 0;         // u32 [E]      keys inside the bracket
+  size_t off_flag = 0;        // u32 [E]      1 = bracket missed, radix fallback
+  size_t off_v = 0;           // f32 [E]      the quantiles v_e
+  size_t off_cand = 0;        // u32 [E][cap] keys inside the bracket
+  size_t off_alpha = 0;       // f32 [N]      token bias when none is given
+  size_t total = 0;
+};
+EqbLayout eqb_layout(int64_t N, int32_t E, int32_t K);
+
+struct PermuteLayout {
+  int64_t chunk = 0;          // slots per chunk
+  int64_t nchunks = 0;
+  bool single_cta = false;
+  size_t off_chunk_counts = 0;  // u32 [E][nchunks]
+  size_t off_counts = 0;        // u32 [E]
+  size_t off_ticket = 0;        // u32 [1]
+  size_t total = 0;
+};
+PermuteLayout permute_layout(int64_t N, int32_t E, int32_t K);
+
+cudaError_t launch_router_logits(const void* x, const void* w, float* z, int64_t N, int32_t d,
+                                 int32_t E, cudaStream_t s);
+
+cudaError_t launch_topk(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
+                        int32_t* ids, float* gates, float* alpha, cudaStream_t s);
+
+cudaError_t launch_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K, int32_t* counts,
+                           int64_t* offsets, int32_t* perm, int32_t* inv, void* ws,
+                           cudaStream_t s);
+
+cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
+                       int32_t K, float* quantiles, void* ws, cudaStream_t s);
+
+// pieces of the EQB update living in route.cu (they walk rows of Z)
+cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* bias, int64_t N,
+                              int32_t E, int32_t K, int64_t S, int64_t stride, uint32_t* sample,
+                              cudaStream_t s);
+cudaError_t launch_eqb_window_pass(const float* z, const float* alpha_in, const float* bias,
+                                   float* alpha_out, int64_t N, int32_t E, int32_t K,
+                                   const uint32_t* lo, const uint32_t* hi, uint32_t* above,
+                                   uint32_t* cnt, uint32_t* cand, int64_t cap, cudaStream_t s);
+
+int device_sm_count();
+
+}  // namespace kolibri

@@ -1,0 +1,164 @@
+/*
+ * kolibri_router.h -- C ABI of the B200 (sm_100a) sigmoid MoE router with
+ * Exact Quantile Balancing (EQB).
+ *
+ * The method (page "Kolibri Pre-Training from Scratch: UniBPE, Hybrid
+ * Attention and Exact Quantile Balancing", sections 6.1 and 7; page
+ * "Kolibri 1 im Detail: hybride RNoPE-Attention, Sparse MoE und FP8-Serving",
+ * section "Routing: Auswahl-Bias und Mischgewichte sind getrennt"):
+ *
+ *   Z = x W^T                         router logits, bf16 in, fp32 out
+ *   B = Z + 1 beta^T                  selection bias, used for selection only
+ *   I_t = Top-K(B_t,:)                the K experts of token t
+ *   S_t,e = sigma(Z_t,e), e in I_t    mixing weights from the RAW logits,
+ *                                     not renormalised
+ *   alpha_t = -Q_K(B_t,:)             token bias
+ *   beta_e  = -Q_r(Z_:,e + alpha),    expert bias, r = N K / E, then centred
+ *
+ * Q_m(list) is the (m+1)-th largest entry (section 1).  EQB computes the
+ * column quantile exactly, not by a histogram approximation (section 7.3).
+ *
+ * Conventions shared by every call
+ *   - All data pointers are DEVICE pointers owned by the caller.  No call
+ *     allocates or frees device memory, and none synchronises the host,
+ *     except kolibri_device_status().  Work is enqueued on `stream`, a
+ *     cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - Arrays are dense and row-major with the shapes given below.  Pointers
+ *     must be 16-byte aligned.
+ *   - Order of fp32 scores: the total order of the order-preserving key of
+ *     the bit pattern (so -0.0 ranks below +0.0).  Equal scores rank the
+ *     lower expert id first.  Inputs must be finite (not checked).
+ *   - Arguments are validated on the host before anything is enqueued; on
+ *     an argument error nothing is written.
+ *   - Each call returns KOLIBRI_OK once its work is enqueued.  A launch
+ *     failure returns KOLIBRI_ERR_CUDA.  Errors found later on the device
+ *     (a bounded wait that expired, an expert id out of range) are recorded
+ *     in a per-device status word read by kolibri_device_status().
+ *   - Calls on different streams may run concurrently if they use separate
+ *     workspaces; one workspace must not be shared by calls that can
+ *     overlap on the GPU.
+ */
+#ifndef KOLIBRI_ROUTER_H
+#define KOLIBRI_ROUTER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KOLIBRI_API __attribute__((visibility("default")))
+#else
+#define KOLIBRI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kolibri_status {
+    KOLIBRI_OK = 0,
+    KOLIBRI_ERR_INVALID_ARG = 1,        /* null pointer, misalignment, K >= E ... */
+    KOLIBRI_ERR_UNSUPPORTED_SHAPE = 2,  /* shape outside the supported range      */
+    KOLIBRI_ERR_WORKSPACE_TOO_SMALL = 3,/* ws_bytes < kolibri_workspace_bytes()   */
+    KOLIBRI_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed   */
+    KOLIBRI_ERR_TIMEOUT = 5,            /* a bounded device-side wait expired     */
+    KOLIBRI_ERR_DEVICE = 6              /* a device-side check failed (bad id)    */
+} kolibri_status;
+
+/* Operation selector for kolibri_workspace_bytes(). */
+enum {
+    KOLIBRI_OP_PERMUTE = 1,
+    KOLIBRI_OP_EQB = 2
+};
+
+/* Limits.  E (experts) and K (top-K) must satisfy 1 <= K < E <= 512,
+ * K <= 16, E % 4 == 0.  N (tokens) must satisfy 1 <= N and N*K < 2^31.
+ * d (width) must satisfy 64 <= d, d % 64 == 0. */
+#define KOLIBRI_MAX_EXPERTS 512
+#define KOLIBRI_MAX_TOPK 16
+
+/* Human-readable name of a status code (static string, never NULL). */
+KOLIBRI_API const char *kolibri_status_string(kolibri_status status);
+
+/* Bytes of caller-provided device workspace that `op` needs for these sizes
+ * (0 if the sizes are invalid).  The workspace need not be initialised. */
+KOLIBRI_API size_t kolibri_workspace_bytes(int op, int64_t N, int32_t E, int32_t K);
+
+/*
+ * Router logits Z = x W^T ("Kolibri Pre-Training from Scratch" 6.1; "Kolibri
+ * 1 im Detail", routing: bf16 router, tokens [N, d] -> fp32 logits [N, E]).
+ *   x  [N, d] bf16 (raw 16-bit patterns), row-major
+ *   w  [E, d] bf16, row-major (one row per expert)
+ *   z  [N, E] fp32, row-major, written
+ * Products are exact, accumulation is fp32 on the tensor cores (tcgen05).
+ * Shapes: d % 64 == 0, E % 16 == 0, 16 <= E <= 512.
+ */
+KOLIBRI_API kolibri_status kolibri_router_logits(const void *x, const void *w, float *z,
+                                     int64_t N, int32_t d, int32_t E, void *stream);
+
+/*
+ * Bias add, top-K selection and sigmoid gates ("Kolibri Pre-Training from
+ * Scratch" 6.1 and 7.1; "Kolibri 1 im Detail", routing steps 1 and 2).
+ *   z      [N, E] fp32 logits
+ *   bias   [E] fp32 selection bias beta, or NULL for no bias (B = Z exactly)
+ *   ids    [N, K] int32, written: the K experts of each token, biased score
+ *          descending, ties to the lower id
+ *   gates  [N, K] fp32, written: sigma(z[t, ids[t,k]]) from the raw logits,
+ *          computed in fp64 and rounded once; not renormalised
+ *   alpha  [N] fp32, written if not NULL: -(the (K+1)-th largest biased
+ *          score), the token bias of section 7.1
+ */
+KOLIBRI_API kolibri_status kolibri_router_topk(const float *z, const float *bias, int64_t N, int32_t E,
+                                   int32_t K, int32_t *ids, float *gates, float *alpha,
+                                   void *stream);
+
+/*
+ * Expert loads and the grouping of routed slots by expert (loads c_e of
+ * "Kolibri Pre-Training from Scratch" 6.1/6.2).  Slot j = t*K + k.
+ *   ids      [N, K] int32 expert ids in [0, E)
+ *   counts   [E] int32, written: c_e
+ *   offsets  [E+1] int64, written: exclusive prefix sum of counts
+ *   perm     [N*K] int32, written: perm[p] = slot at grouped position p;
+ *            experts ascending, slots ascending inside an expert (stable)
+ *   inv      [N*K] int32, written if not NULL: inv[perm[p]] = p
+ *   ws       device workspace of kolibri_workspace_bytes(KOLIBRI_OP_PERMUTE)
+ * An id outside [0, E) sets KOLIBRI_ERR_DEVICE in the device status word;
+ * the outputs are then unspecified.
+ */
+KOLIBRI_API kolibri_status kolibri_expert_permute(const int32_t *ids, int64_t N, int32_t E, int32_t K,
+                                      int32_t *counts, int64_t *offsets, int32_t *perm,
+                                      int32_t *inv, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Exact Quantile Balancing update ("Kolibri Pre-Training from Scratch" 7.1
+ * update rule, 7.2 order of operations, 7.3 exactness):
+ *   v_e  = Q_m(Z_:,e + alpha), the (m+1)-th largest entry of the fp32 sums,
+ *          m = floor(N*K/E), computed exactly (radix selection on keys)
+ *   beta = -v, then centred: mean = fp32(fp64 sum over e ascending / E),
+ *          beta_e = -v_e - mean in fp32
+ *   z          [N, E] fp32 logits
+ *   alpha      [N] fp32 token bias (from kolibri_router_topk), or NULL: then
+ *              alpha_t = -Q_K(Z_t,: + bias_in) is computed here
+ *   bias       [E] fp32: read as beta_in when alpha is NULL; always
+ *              overwritten with the new centred beta
+ *   quantiles  [E] fp32, written if not NULL: v_e
+ *   ws         device workspace of kolibri_workspace_bytes(KOLIBRI_OP_EQB)
+ * The result is exact for every input; large batches are first bracketed
+ * from a strided row sample and fall back to full radix passes for any
+ * expert whose bracket misses.
+ */
+KOLIBRI_API kolibri_status kolibri_eqb_update(const float *z, const float *alpha, float *bias,
+                                  int64_t N, int32_t E, int32_t K, float *quantiles,
+                                  void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current device: KOLIBRI_OK, KOLIBRI_ERR_TIMEOUT or KOLIBRI_ERR_DEVICE
+ * (the first recorded), or KOLIBRI_ERR_CUDA if the synchronisation failed.
+ */
+KOLIBRI_API kolibri_status kolibri_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KOLIBRI_ROUTER_H */

@@ -25,3 +25,11 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def kolibri_lib():
+    """The router library, built in-tree if missing or stale."""
+    from expert_load_balancing_b200 import binding, build
+    build.build()
+    return binding.load()
