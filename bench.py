@@ -198,6 +198,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     B.load()
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens:
+        import dataclasses
+        wl = dataclasses.replace(wl, N=args.tokens)
     N, d, E, K = wl.N, wl.d, wl.E, wl.K
     step = RouterStep(wl, device, seed=rank)
     stream = torch.cuda.Stream(device)
@@ -421,6 +424,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="kolibri_n1m", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override N (smaller captures for the profiler only)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
