@@ -72,10 +72,12 @@ def gemm_bytes(N, d, E):
 
 
 def launches_per_step(N, E, K):
-    """Kernels of ours per step: logits 1, top-K 1, permute 1 or 3, EQB 3 or 6."""
+    """Kernels of ours per step: logits 1; routing + EQB 4 (N <= 16384: route,
+    sample, select, bias) or 6 (sample, bracket, fused pass, select,
+    fallback check, bias); permutation 1 or 3."""
+    route_eqb = 4 if N <= 16384 else 6
     permute = 1 if N * K <= 4096 else 3
-    eqb = 3 if N <= 16384 else 6
-    return 1 + 1 + permute + eqb
+    return 1 + route_eqb + permute
 
 
 # ---------------------------------------------------------------- clocks
@@ -173,24 +175,21 @@ class RouterStep:
         self.ws_eqb = B.workspace(B.KOLIBRI_OP_EQB, N, E, K, device)
 
     def run(self, stream, events=None):
+        """logits -> routing + EQB update (one call, one read of Z) -> permutation."""
         wl = self.wl
         if events:
             events[0].record(stream)
         B.kolibri_router_logits(self.x, self.w, self.z, stream=stream)
         if events:
             events[1].record(stream)
-        B.kolibri_router_topk(self.z, self.beta, wl.K, self.ids, self.gates, self.alpha,
-                              stream=stream)
+        B.kolibri_route_and_balance(self.z, self.beta, wl.K, self.ws_eqb, self.ids, self.gates,
+                                    self.alpha, self.q, stream=stream)
         if events:
             events[2].record(stream)
         B.kolibri_expert_permute(self.ids, wl.E, self.ws_perm, self.counts, self.offsets,
                                  self.perm, self.inv, stream=stream)
         if events:
             events[3].record(stream)
-        B.kolibri_eqb_update(self.z, self.alpha, self.beta, wl.K, self.ws_eqb, self.q,
-                             stream=stream)
-        if events:
-            events[4].record(stream)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -213,7 +212,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status after warm-up: {B.status_string(st)}")
 
     # ---- timed region: device time, CUDA events on the launching stream
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
@@ -233,7 +232,7 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     total_ms = t0.elapsed_time(t1)
-    stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(4)]
+    stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(3)]
                          for i in range(args.steps)]).mean(axis=0)
     st = B.kolibri_device_status(stream)
     if st != B.KOLIBRI_OK:
@@ -282,8 +281,8 @@ def run_ours(args, rank, world, local_rank):
         "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ms_per_step,
                           "flops": flops, "bytes": bytes_,
                           "peaks": f"bf16 burst {peaks['bf16_tflops']} TF/s, HBM {peaks['hbm_gbs']} GB/s, of {peaks['source']}"},
-        "stages_ms": {"logits": gemm_ms, "topk": float(stage_ms[1]),
-                      "permute": float(stage_ms[2]), "eqb": float(stage_ms[3])},
+        "stages_ms": {"logits": gemm_ms, "route_and_eqb": float(stage_ms[1]),
+                      "permute": float(stage_ms[2])},
         "gpu_launches": launches_per_step(N, E, K) * args.steps,
         "clocks": clocks,
         "e2e": e2e,

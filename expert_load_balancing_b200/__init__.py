@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     kolibri_device_status,
     kolibri_eqb_update,
     kolibri_expert_permute,
+    kolibri_route_and_balance,
     kolibri_router_logits,
     kolibri_router_topk,
     kolibri_workspace_bytes,

@@ -35,6 +35,8 @@ SIGNATURES = {
     "kolibri_router_topk": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P]),
     "kolibri_expert_permute": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "kolibri_eqb_update": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _SZ, _P]),
+    "kolibri_route_and_balance": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P, _P,
+                                                 _SZ, _P]),
     "kolibri_device_status": (ctypes.c_int, [_P]),
 }
 
@@ -186,6 +188,36 @@ def kolibri_eqb_update(z: torch.Tensor, alpha: torch.Tensor | None, bias: torch.
            load().kolibri_eqb_update(_ptr(z), _ptr(alpha), _ptr(bias), N, E, K, _ptr(quantiles),
                                      _ptr(ws), ws.numel(), _stream(stream)))
     return bias, quantiles
+
+
+def kolibri_route_and_balance(z: torch.Tensor, bias: torch.Tensor, K: int,
+                              ws: torch.Tensor | None = None, ids=None, gates=None, alpha=None,
+                              quantiles=None, want_alpha: bool = True,
+                              want_quantiles: bool = True, stream=None):
+    """Routing with ``bias`` then the EQB update of ``bias`` in place.
+
+    Returns (ids [N,K] int32, gates [N,K] fp32, alpha [N] or None, quantiles [E] or None)."""
+    N, E = z.shape
+    _need(z, torch.float32, (N, E), "z")
+    _need(bias, torch.float32, (E,), "bias")
+    dev = z.device
+    if ws is None:
+        ws = workspace(KOLIBRI_OP_EQB, N, E, K, dev)
+    if ids is None:
+        ids = torch.empty((N, K), dtype=torch.int32, device=dev)
+    if gates is None:
+        gates = torch.empty((N, K), dtype=torch.float32, device=dev)
+    if alpha is None and want_alpha:
+        alpha = torch.empty((N,), dtype=torch.float32, device=dev)
+    if quantiles is None and want_quantiles:
+        quantiles = torch.empty((E,), dtype=torch.float32, device=dev)
+    _need(ids, torch.int32, (N, K), "ids")
+    _need(gates, torch.float32, (N, K), "gates")
+    _check("kolibri_route_and_balance",
+           load().kolibri_route_and_balance(_ptr(z), _ptr(bias), N, E, K, _ptr(ids), _ptr(gates),
+                                            _ptr(alpha), _ptr(quantiles), _ptr(ws), ws.numel(),
+                                            _stream(stream)))
+    return ids, gates, alpha, quantiles
 
 
 def kolibri_device_status(stream=None) -> int:

@@ -108,6 +108,19 @@ kolibri_status kolibri_eqb_update(const float* z, const float* alpha, float* bia
       launch_eqb(z, alpha, bias, N, E, K, quantiles, ws, static_cast<cudaStream_t>(stream)));
 }
 
+kolibri_status kolibri_route_and_balance(const float* z, float* bias, int64_t N, int32_t E,
+                                         int32_t K, int32_t* ids, float* gates, float* alpha,
+                                         float* quantiles, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!z || !bias || !ids || !gates || !ws) return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(z) || !aligned16(bias) || !aligned16(ws)) return KOLIBRI_ERR_INVALID_ARG;
+  if (ws_bytes < eqb_layout(N, E, K).total) return KOLIBRI_ERR_WORKSPACE_TOO_SMALL;
+  return from_cuda(launch_route_balance(z, bias, N, E, K, ids, gates, alpha, quantiles, ws,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 kolibri_status kolibri_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KOLIBRI_ERR_CUDA;

@@ -231,68 +231,126 @@ EqbLayout eqb_layout(int64_t N, int32_t E, int32_t K) {
   L.off_cnt = take(sizeof(uint32_t) * E);
   L.off_flag = take(sizeof(uint32_t) * E);
   L.off_v = take(sizeof(float) * E);
-  if (!L.exact_small) {
+  L.off_alpha = take(sizeof(float) * static_cast<size_t>(N));
+  if (!L.exact_small)
     L.off_cand = take(sizeof(uint32_t) * static_cast<size_t>(E) * static_cast<size_t>(kCandCap));
-    L.off_alpha = take(sizeof(float) * static_cast<size_t>(N));
-  }
   L.total = off;
   return L;
 }
 
+namespace {
+
+struct EqbBuffers {
+  EqbLayout L;
+  uint32_t *sample, *lo, *hi, *above, *cnt, *flag, *cand;
+  float *v, *alpha_ws;
+  char* base;
+};
+
+EqbBuffers eqb_buffers(int64_t N, int32_t E, int32_t K, void* ws) {
+  EqbBuffers b;
+  b.L = eqb_layout(N, E, K);
+  b.base = static_cast<char*>(ws);
+  auto u32 = [&b](size_t off) { return reinterpret_cast<uint32_t*>(b.base + off); };
+  b.sample = u32(b.L.off_sample);
+  b.lo = u32(b.L.off_lo);
+  b.hi = u32(b.L.off_hi);
+  b.above = u32(b.L.off_above);
+  b.cnt = u32(b.L.off_cnt);
+  b.flag = u32(b.L.off_flag);
+  b.cand = b.L.exact_small ? nullptr : u32(b.L.off_cand);
+  b.v = reinterpret_cast<float*>(b.base + b.L.off_v);
+  b.alpha_ws = reinterpret_cast<float*>(b.base + b.L.off_alpha);
+  return b;
+}
+
+// Steps 1-2: sample keys (token bias given, or computed from bias_in), then
+// either the exact quantile (small N) or the per-expert bracket.
+cudaError_t eqb_begin(const float* z, const float* alpha, const float* bias, int64_t N, int32_t E,
+                      int32_t K, const EqbBuffers& b, cudaStream_t s) {
+  const EqbLayout& L = b.L;
+  const int64_t m = (N * static_cast<int64_t>(K)) / E;
+  cudaError_t err = launch_eqb_sample(z, alpha, alpha ? nullptr : bias, N, E, K, L.S, L.stride,
+                                      b.sample, s);
+  if (err != cudaSuccess) return err;
+  if (L.exact_small) {
+    sample_select_kernel<<<E, kSelThreads, 0, s>>>(b.sample, L.S, m, 0, 0, true, b.v, b.lo, b.hi);
+    return cudaGetLastError();
+  }
+  // bracket ranks in the sample, descending order: the target sits at
+  // about q*S with q = (m+1)/N; margin 6 binomial standard deviations
+  const double q = static_cast<double>(m + 1) / static_cast<double>(N);
+  const double center = q * static_cast<double>(L.S);
+  const double sd = std::sqrt(center * (1.0 - q));
+  const int64_t margin = static_cast<int64_t>(std::ceil(6.0 * sd)) + 8;
+  int64_t r_hi = static_cast<int64_t>(std::floor(center)) - margin;
+  int64_t r_lo = static_cast<int64_t>(std::ceil(center)) + margin;
+  if (r_hi < 0) r_hi = 0;
+  if (r_lo > L.S - 1) r_lo = L.S - 1;
+  err = cudaMemsetAsync(b.base + L.off_above, 0, L.off_v - L.off_above, s);  // above, cnt, flag
+  if (err != cudaSuccess) return err;
+  sample_select_kernel<<<E, kSelThreads, 0, s>>>(b.sample, L.S, 0, r_hi, r_lo, false, b.v, b.lo,
+                                                 b.hi);
+  return cudaGetLastError();
+}
+
+// Steps 4-5 and the bias update.
+cudaError_t eqb_end(const float* z, const float* alpha_used, float* bias, int64_t N, int32_t E,
+                    int32_t K, float* quantiles, const EqbBuffers& b, cudaStream_t s) {
+  const int64_t m = (N * static_cast<int64_t>(K)) / E;
+  cudaError_t err;
+  if (!b.L.exact_small) {
+    bracket_select_kernel<<<E, kSelThreads, 0, s>>>(b.cand, b.cnt, b.above, kCandCap, m, b.v,
+                                                    b.flag);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    column_fallback_kernel<<<E, kSelThreads, 0, s>>>(z, alpha_used, N, E, m, b.flag, b.v);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  bias_update_kernel<<<1, 512, 0, s>>>(b.v, E, bias, quantiles);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
                        int32_t K, float* quantiles, void* ws, cudaStream_t s) {
-  const EqbLayout L = eqb_layout(N, E, K);
-  char* base = static_cast<char*>(ws);
-  auto u32 = [base](size_t off) { return reinterpret_cast<uint32_t*>(base + off); };
-  uint32_t* sample = u32(L.off_sample);
-  uint32_t* lo = u32(L.off_lo);
-  uint32_t* hi = u32(L.off_hi);
-  uint32_t* above = u32(L.off_above);
-  uint32_t* cnt = u32(L.off_cnt);
-  uint32_t* flag = u32(L.off_flag);
-  float* v = reinterpret_cast<float*>(base + L.off_v);
-  const int64_t m = (N * static_cast<int64_t>(K)) / E;
-
-  // alpha is computed from bias_in before bias is overwritten (stream order)
-  cudaError_t err = launch_eqb_sample(z, alpha, alpha ? nullptr : bias, N, E, K, L.S, L.stride,
-                                      sample, s);
+  const EqbBuffers b = eqb_buffers(N, E, K, ws);
+  cudaError_t err = eqb_begin(z, alpha, bias, N, E, K, b, s);
   if (err != cudaSuccess) return err;
+  const float* alpha_used = alpha;
+  if (!b.L.exact_small) {
+    // the full pass; it also derives alpha from bias_in when none is given
+    err = launch_route_window_pass(z, bias, alpha, N, E, K, nullptr, nullptr,
+                                   alpha ? nullptr : b.alpha_ws, b.lo, b.hi, b.above, b.cnt,
+                                   b.cand, kCandCap, s);
+    if (err != cudaSuccess) return err;
+    if (!alpha) alpha_used = b.alpha_ws;
+  }
+  return eqb_end(z, alpha_used, bias, N, E, K, quantiles, b, s);
+}
 
-  if (L.exact_small) {
-    sample_select_kernel<<<E, kSelThreads, 0, s>>>(sample, L.S, m, 0, 0, true, v, lo, hi);
-    err = cudaGetLastError();
+cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t E, int32_t K,
+                                 int32_t* ids, float* gates, float* alpha, float* quantiles,
+                                 void* ws, cudaStream_t s) {
+  const EqbBuffers b = eqb_buffers(N, E, K, ws);
+  float* alpha_out = alpha ? alpha : b.alpha_ws;
+  cudaError_t err;
+  if (b.L.exact_small) {
+    // the sample is the whole column: route first, then select from its alpha
+    err = launch_topk(z, bias, N, E, K, ids, gates, alpha_out, s);
+    if (err != cudaSuccess) return err;
+    err = eqb_begin(z, alpha_out, bias, N, E, K, b, s);
     if (err != cudaSuccess) return err;
   } else {
-    // bracket ranks in the sample, descending order: the target sits at
-    // about q*S with q = (m+1)/N; margin 6 binomial standard deviations
-    const double q = static_cast<double>(m + 1) / static_cast<double>(N);
-    const double center = q * static_cast<double>(L.S);
-    const double sd = std::sqrt(center * (1.0 - q));
-    const int64_t margin = static_cast<int64_t>(std::ceil(6.0 * sd)) + 8;
-    int64_t r_hi = static_cast<int64_t>(std::floor(center)) - margin;
-    int64_t r_lo = static_cast<int64_t>(std::ceil(center)) + margin;
-    if (r_hi < 0) r_hi = 0;
-    if (r_lo > L.S - 1) r_lo = L.S - 1;
-    err = cudaMemsetAsync(base + L.off_above, 0, L.off_v - L.off_above, s);  // above, cnt, flag
+    // the bracket comes from sampled rows routed with the same bias; one
+    // pass then routes every row and feeds the bracket
+    err = eqb_begin(z, nullptr, bias, N, E, K, b, s);
     if (err != cudaSuccess) return err;
-    sample_select_kernel<<<E, kSelThreads, 0, s>>>(sample, L.S, 0, r_hi, r_lo, false, v, lo, hi);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    float* alpha_ws = reinterpret_cast<float*>(base + L.off_alpha);
-    uint32_t* cand = u32(L.off_cand);
-    err = launch_eqb_window_pass(z, alpha, alpha ? nullptr : bias, alpha ? nullptr : alpha_ws, N,
-                                 E, K, lo, hi, above, cnt, cand, kCandCap, s);
-    if (err != cudaSuccess) return err;
-    bracket_select_kernel<<<E, kSelThreads, 0, s>>>(cand, cnt, above, kCandCap, m, v, flag);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    column_fallback_kernel<<<E, kSelThreads, 0, s>>>(z, alpha ? alpha : alpha_ws, N, E, m, flag,
-                                                     v);
-    err = cudaGetLastError();
+    err = launch_route_window_pass(z, bias, nullptr, N, E, K, ids, gates, alpha_out, b.lo, b.hi,
+                                   b.above, b.cnt, b.cand, kCandCap, s);
     if (err != cudaSuccess) return err;
   }
-  bias_update_kernel<<<1, 512, 0, s>>>(v, E, bias, quantiles);
-  return cudaGetLastError();
+  return eqb_end(z, alpha_out, bias, N, E, K, quantiles, b, s);
 }
 
 }  // namespace kolibri

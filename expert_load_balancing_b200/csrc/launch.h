@@ -52,14 +52,22 @@ cudaError_t launch_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K, 
 cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
                        int32_t K, float* quantiles, void* ws, cudaStream_t s);
 
+cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t E, int32_t K,
+                                 int32_t* ids, float* gates, float* alpha, float* quantiles,
+                                 void* ws, cudaStream_t s);
+
 // pieces of the EQB update living in route.cu (they walk rows of Z)
 cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* bias, int64_t N,
                               int32_t E, int32_t K, int64_t S, int64_t stride, uint32_t* sample,
                               cudaStream_t s);
-cudaError_t launch_eqb_window_pass(const float* z, const float* alpha_in, const float* bias,
-                                   float* alpha_out, int64_t N, int32_t E, int32_t K,
-                                   const uint32_t* lo, const uint32_t* hi, uint32_t* above,
-                                   uint32_t* cnt, uint32_t* cand, int64_t cap, cudaStream_t s);
+// Bracketed full pass.  alpha_in given: use it.  Otherwise alpha is derived
+// from bias (and written to alpha_out); with ids/gates non-null the same
+// pass also writes the routing.
+cudaError_t launch_route_window_pass(const float* z, const float* bias, const float* alpha_in,
+                                     int64_t N, int32_t E, int32_t K, int32_t* ids, float* gates,
+                                     float* alpha_out, const uint32_t* lo, const uint32_t* hi,
+                                     uint32_t* above, uint32_t* cnt, uint32_t* cand, int64_t cap,
+                                     cudaStream_t s);
 
 int device_sm_count();
 

@@ -4,9 +4,14 @@
 //     Detail", routing steps 1-2);
 //   * the two row passes of the exact EQB quantile (7.1, 7.3): the keys of
 //     Z + alpha at sampled rows, and the full pass that counts keys above a
-//     per-expert bracket and gathers the keys inside it.
+//     per-expert bracket and gathers the keys inside it.  The full pass can
+//     run inside the selection kernel, so Z is streamed from HBM once for
+//     routing and balancing together.
 //
-// One warp per row; rows are HBM-streamed once with 512-byte warp loads.
+// One warp per row (see route.cuh for the selection); each block runs its
+// warps over consecutive rows and stages bracketed keys in shared memory,
+// flushing them to the per-expert gather buffer once per batch of rows with
+// one global atomic per expert.
 #include "launch.h"
 #include "route.cuh"
 
@@ -14,14 +19,17 @@ namespace kolibri {
 
 namespace {
 
-constexpr int kRouteThreads = 256;
-constexpr int kRouteWarps = kRouteThreads / kWarp;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / kWarp;
+constexpr int kRowsPerWarp = 32;     // rows per warp between gather flushes
+constexpr int kStageSlots = 16;      // staged bracket keys per expert per block
 
-struct RouteArgs {
+struct RouteParams {
   const float* z;
   const float* beta;  // may be null
   int64_t N;
   int E, K;
+  // selection outputs
   int32_t* ids;
   float* gates;
   float* alpha_out;
@@ -36,97 +44,274 @@ struct RouteArgs {
 };
 
 template <int Q>
-__device__ __forceinline__ void load_lane_vec(const float* __restrict__ p, int E, int lane,
-                                              float (&v)[4 * Q]) {
-  load_row<Q>(p, E, lane, v);
+struct WarpScratch {
+  float row[128 * Q];   // this row's raw logits, lane-major
+  float gz[32];         // gate inputs waiting for a batched evaluation
+  uint32_t gidx[32];    // their output positions
+  uint32_t ckey[32];    // compacted candidates: key and expert id
+  uint32_t cid[32];
+};
+
+// Shared-memory layout (dynamic): beta[E] | lo[E] | hi[E] | above[E] |
+// stage_n[E] | stage[E][kStageSlots] | WarpScratch[kWarps]
+struct SmemLayout {
+  int off_beta, off_lo, off_hi, off_above, off_stage_n, off_stage, off_warp, total;
+};
+
+template <int Q, bool kWindow>
+__host__ __device__ SmemLayout smem_layout(int E) {
+  SmemLayout L;
+  int o = 0;
+  L.off_beta = o;
+  o += 4 * E;
+  const int w = kWindow ? 1 : 0;
+  L.off_lo = o;
+  o += 4 * E * w;
+  L.off_hi = o;
+  o += 4 * E * w;
+  L.off_above = o;
+  o += 4 * E * w;
+  L.off_stage_n = o;
+  o += 4 * E * w;
+  L.off_stage = o;
+  o += 4 * E * kStageSlots * w;
+  o = (o + 15) & ~15;
+  L.off_warp = o;
+  o += static_cast<int>(sizeof(WarpScratch<Q>)) * kWarps;
+  L.total = o;
+  return L;
 }
 
-template <int Q>
-__device__ __forceinline__ void load_lane_u32(const uint32_t* __restrict__ p, int E, int lane,
-                                              uint32_t (&v)[4 * Q]) {
-#pragma unroll
-  for (int q = 0; q < Q; ++q) {
-    int e0 = 128 * q + 4 * lane;
-    uint4 t = make_uint4(0u, 0u, 0u, 0u);
-    if (e0 < E) t = __ldg(reinterpret_cast<const uint4*>(p + e0));
-    v[4 * q + 0] = t.x;
-    v[4 * q + 1] = t.y;
-    v[4 * q + 2] = t.z;
-    v[4 * q + 3] = t.w;
-  }
+__device__ __forceinline__ float z_of(const float* row, int lane, int j, int V) {
+  return row[lane * V + j];
 }
 
-// kRoute: write ids/gates.  kAlphaOut: write alpha.  kAlphaIn: read alpha
-// instead of selecting (only without kRoute).  kWindow: bracketed pass.
-template <int Q, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
-__global__ void __launch_bounds__(kRouteThreads) route_rows_kernel(const RouteArgs a) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warp0 = static_cast<int64_t>(blockIdx.x) * kRouteWarps + (threadIdx.x >> 5);
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kRouteWarps;
-  const int E = a.E, K = a.K;
+// Evaluate the staged gates (lanes < n) and store them.
+__device__ __forceinline__ void flush_gates(float* __restrict__ gates, const float* gz,
+                                            const uint32_t* gidx, int n, int lane) {
+  if (lane < n) gates[gidx[lane]] = gate_sigmoid(gz[lane]);
+}
 
-  float beta_l[4 * Q];
-  const bool has_bias = a.beta != nullptr;
-  if (has_bias) load_lane_vec<Q>(a.beta, E, lane, beta_l);
-  else {
-#pragma unroll
-    for (int j = 0; j < 4 * Q; ++j) beta_l[j] = 0.f;
-  }
-  uint32_t lo_l[4 * Q], hi_l[4 * Q], above_l[4 * Q];
-  if constexpr (kWindow) {
-    load_lane_u32<Q>(a.lo, E, lane, lo_l);
-    load_lane_u32<Q>(a.hi, E, lane, hi_l);
-#pragma unroll
-    for (int j = 0; j < 4 * Q; ++j) above_l[j] = 0u;
-  }
+template <int Q, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
+__global__ void __launch_bounds__(kThreads, 3) route_rows_kernel(const RouteParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int V = 4 * Q;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int E = p.E, K = p.K;
+  const SmemLayout L = smem_layout<Q, kWindow>(E);
+  float* beta_s = reinterpret_cast<float*>(smem + L.off_beta);
+  uint32_t* lo_s = reinterpret_cast<uint32_t*>(smem + L.off_lo);
+  uint32_t* hi_s = reinterpret_cast<uint32_t*>(smem + L.off_hi);
+  uint32_t* above_s = reinterpret_cast<uint32_t*>(smem + L.off_above);
+  uint32_t* stage_n = reinterpret_cast<uint32_t*>(smem + L.off_stage_n);
+  uint32_t* stage = reinterpret_cast<uint32_t*>(smem + L.off_stage);
+  WarpScratch<Q>& ws = reinterpret_cast<WarpScratch<Q>*>(smem + L.off_warp)[warp];
 
-  for (int64_t row = warp0; row < a.N; row += nwarps) {
-    const float* zrow = a.z + row * E;
-    float z[4 * Q];
-    load_row<Q>(zrow, E, lane, z);
-    float alpha = 0.f;
-    if constexpr (!kAlphaIn) {
-      uint32_t key[4 * Q];
-      row_keys<Q>(z, beta_l, has_bias, E, lane, key);
-      uint32_t out_key, out_id;
-      warp_topk<Q>(key, K, lane, out_key, out_id);
-      if constexpr (kRoute) {
-        if (lane < K) {
-          float zs = __ldg(zrow + out_id);
-          a.ids[row * K + lane] = static_cast<int32_t>(out_id);
-          a.gates[row * K + lane] = gate_sigmoid(zs);
-        }
-      }
-      uint32_t kk = __shfl_sync(0xffffffffu, out_key, K);
-      alpha = -key_to_float(kk);
-      if constexpr (kAlphaOut) {
-        if (lane == 0) a.alpha_out[row] = alpha;
-      }
-    } else {
-      alpha = __ldg(a.alpha_in + row);
-    }
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    if constexpr (kBias) beta_s[e] = p.beta[e];
     if constexpr (kWindow) {
+      lo_s[e] = p.lo[e];
+      hi_s[e] = p.hi[e];
+      above_s[e] = 0u;
+      stage_n[e] = 0u;
+    }
+  }
+  __syncthreads();
+
+  // valid-slot mask of this lane (fixed for the kernel)
+  uint32_t valid = 0u;
 #pragma unroll
-      for (int j = 0; j < 4 * Q; ++j) {
-        int e = static_cast<int>(slot_expert(lane, j));
-        if (e < E) {
-          uint32_t k = order_key(__fadd_rn(z[j], alpha));
-          if (k > hi_l[j]) {
-            above_l[j] += 1u;
-          } else if (k >= lo_l[j]) {
-            uint32_t pos = atomicAdd(a.cand_cnt + e, 1u);
-            if (pos < a.cap) a.cand[static_cast<int64_t>(e) * a.cap + pos] = k;
+  for (int j = 0; j < V; ++j) valid |= (static_cast<int>(slot_expert(lane, j)) < E) ? (1u << j) : 0u;
+  int gate_n = 0;
+
+  const int64_t rows_per_block = static_cast<int64_t>(kWarps) * kRowsPerWarp;
+  for (int64_t base = static_cast<int64_t>(blockIdx.x) * rows_per_block; base < p.N;
+       base += static_cast<int64_t>(gridDim.x) * rows_per_block) {
+    const int64_t r0 = base + static_cast<int64_t>(warp) * kRowsPerWarp;
+    const int64_t r1 = (r0 + kRowsPerWarp < p.N) ? r0 + kRowsPerWarp : p.N;
+    float znext[V];
+    if (r0 < r1) load_row<Q>(p.z + r0 * E, E, lane, znext);
+    for (int64_t row = r0; row < r1; ++row) {
+      float z[V];
+#pragma unroll
+      for (int j = 0; j < V; ++j) z[j] = znext[j];
+      if (row + 1 < r1) load_row<Q>(p.z + (row + 1) * E, E, lane, znext);
+
+      float alpha;
+      if constexpr (!kAlphaIn) {
+        // ---- scores, lane maximum, threshold, candidate mask
+        float b[V];
+        float lane_max = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+          float4 bq = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (kBias && (valid & (1u << (4 * q))))
+            bq = *reinterpret_cast<const float4*>(&beta_s[128 * q + 4 * lane]);
+          const float bv[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int j = 4 * q + i;
+            b[j] = kBias ? __fadd_rn(z[j], bv[i]) : z[j];
+            if (valid & (1u << j)) lane_max = fmaxf(lane_max, b[j]);
+          }
+        }
+        const float T = threshold_from_groups(lane_max, K);
+        uint32_t cand = 0u;
+#pragma unroll
+        for (int j = 0; j < V; ++j) cand |= (b[j] >= T) ? (1u << j) : 0u;
+        cand &= valid;
+        // raw logits to the row buffer for indexed access
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < Q; ++q)
+          *reinterpret_cast<float4*>(&ws.row[lane * V + 4 * q]) =
+              make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
+        // ---- compact the candidates to at most one per lane
+        const int c = __popc(cand);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        uint32_t out_key = 0u, out_id = kNoId;
+        if (total <= 32) {
+          int pos = incl - c;
+          uint32_t m = cand;
+          while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1u;
+            const uint32_t e = slot_expert(lane, j);
+            const float bb = kBias ? __fadd_rn(z_of(ws.row, lane, j, V), beta_s[e]) : z_of(ws.row, lane, j, V);
+            ws.ckey[pos] = order_key(bb);
+            ws.cid[pos] = e;
+            ++pos;
+          }
+          __syncwarp();
+          uint32_t k = lane < total ? ws.ckey[lane] : 0u;
+          uint32_t id = lane < total ? ws.cid[lane] : kNoId;
+          for (int r = 0; r <= K; ++r) {
+            const uint32_t M = __reduce_max_sync(0xffffffffu, k);
+            const uint32_t mine = (k == M) ? id : kNoId;
+            const uint32_t I = __reduce_min_sync(0xffffffffu, mine);
+            if (lane == r) {
+              out_key = M;
+              out_id = I;
+            }
+            if (id == I) {  // the owner (ids are distinct); I == kNoId only for bad input
+              k = 0u;
+              id = kNoId;
+            }
+          }
+        } else {
+          // many candidates (heavy ties): K+1 rounds, each owner rescans its own
+          __syncwarp();
+          auto lane_best = [&](uint32_t mm, uint32_t& bk, uint32_t& bid) {
+            bk = 0u;
+            bid = kNoId;
+            while (mm) {
+              const int j = __ffs(mm) - 1;
+              mm &= mm - 1u;
+              const uint32_t e = slot_expert(lane, j);
+              const float zz = z_of(ws.row, lane, j, V);
+              const uint32_t k = order_key(kBias ? __fadd_rn(zz, beta_s[e]) : zz);
+              if (k > bk) {  // slots ascend in id: strict '>' keeps the lower id
+                bk = k;
+                bid = e;
+              }
+            }
+          };
+          uint32_t bk, bid;
+          lane_best(cand, bk, bid);
+          for (int r = 0; r <= K; ++r) {
+            const uint32_t M = __reduce_max_sync(0xffffffffu, bk);
+            const uint32_t mine = (bk == M) ? bid : kNoId;
+            const uint32_t I = __reduce_min_sync(0xffffffffu, mine);
+            if (lane == r) {
+              out_key = M;
+              out_id = I;
+            }
+            if (bid == I && I != kNoId) {
+              cand &= ~(1u << (4 * static_cast<int>(I >> 7) + static_cast<int>(I & 3)));
+              lane_best(cand, bk, bid);
+            }
+          }
+        }
+        alpha = -key_to_float(__shfl_sync(0xffffffffu, out_key, K));
+        if constexpr (kRoute) {
+          if (lane < K) {
+            // out_id < E for finite inputs; clamp so no input can index outside
+            const uint32_t e = out_id < static_cast<uint32_t>(E) ? out_id : 0u;
+            p.ids[row * K + lane] = static_cast<int32_t>(out_id);
+            ws.gz[gate_n + lane] = ws.row[buffer_pos<Q>(e)];
+            ws.gidx[gate_n + lane] = static_cast<uint32_t>(row * K + lane);
+          }
+          gate_n += K;
+          if (gate_n + K > 32) {
+            __syncwarp();
+            flush_gates(p.gates, ws.gz, ws.gidx, gate_n, lane);
+            gate_n = 0;
+          }
+        }
+        if constexpr (kAlphaOut) {
+          if (lane == 0) p.alpha_out[row] = alpha;
+        }
+        __syncwarp();
+      } else {
+        alpha = __ldg(p.alpha_in + row);
+      }
+
+      if constexpr (kWindow) {
+#pragma unroll
+        for (int q = 0; q < Q; ++q) {
+          if (!(valid & (1u << (4 * q)))) continue;
+          const int e0 = 128 * q + 4 * lane;
+          const uint4 hq = *reinterpret_cast<const uint4*>(&hi_s[e0]);
+          const uint4 lq = *reinterpret_cast<const uint4*>(&lo_s[e0]);
+          const uint32_t hv[4] = {hq.x, hq.y, hq.z, hq.w};
+          const uint32_t lv[4] = {lq.x, lq.y, lq.z, lq.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t k = order_key(__fadd_rn(z[4 * q + i], alpha));
+            if (k > hv[i]) {
+              atomicAdd(&above_s[e0 + i], 1u);
+            } else if (k >= lv[i]) {
+              const uint32_t pos = atomicAdd(&stage_n[e0 + i], 1u);
+              if (pos < kStageSlots) {
+                stage[(e0 + i) * kStageSlots + pos] = k;
+              } else {  // block buffer full: append directly
+                const uint32_t g = atomicAdd(p.cand_cnt + e0 + i, 1u);
+                if (g < p.cap) p.cand[static_cast<int64_t>(e0 + i) * p.cap + g] = k;
+              }
+            }
           }
         }
       }
     }
+    if constexpr (kWindow) {
+      __syncthreads();
+      for (int e = threadIdx.x; e < E; e += kThreads) {
+        uint32_t n = stage_n[e];
+        if (n > kStageSlots) n = kStageSlots;
+        if (n) {
+          const uint32_t g = atomicAdd(p.cand_cnt + e, n);
+          for (uint32_t i = 0; i < n; ++i)
+            if (g + i < p.cap) p.cand[static_cast<int64_t>(e) * p.cap + g + i] = stage[e * kStageSlots + i];
+        }
+        stage_n[e] = 0u;
+      }
+      __syncthreads();
+    }
+  }
+  if constexpr (kRoute) {
+    __syncwarp();
+    flush_gates(p.gates, ws.gz, ws.gidx, gate_n, lane);
   }
   if constexpr (kWindow) {
-#pragma unroll
-    for (int j = 0; j < 4 * Q; ++j) {
-      int e = static_cast<int>(slot_expert(lane, j));
-      if (e < E && above_l[j] != 0u) atomicAdd(a.above + e, above_l[j]);
-    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kThreads)
+      if (above_s[e] != 0u) atomicAdd(p.above + e, above_s[e]);
   }
 }
 
@@ -136,87 +321,129 @@ __global__ void __launch_bounds__(kRouteThreads) route_rows_kernel(const RouteAr
 constexpr int kSampleRows = 32;
 
 template <int Q, bool kAlphaIn>
-__global__ void __launch_bounds__(kRouteThreads) sample_keys_kernel(
+__global__ void __launch_bounds__(kThreads) sample_keys_kernel(
     const float* __restrict__ z, const float* __restrict__ alpha_in, const float* __restrict__ beta,
     int64_t N, int E, int K, int64_t S, int64_t stride, uint32_t* __restrict__ sample) {
-  extern __shared__ uint32_t tile[];  // [kSampleRows][E + 1]
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int V = 4 * Q;
+  uint32_t* tile = reinterpret_cast<uint32_t*>(smem);  // [kSampleRows][E + 1]
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t s0 = static_cast<int64_t>(blockIdx.x) * kSampleRows;
   const int ld = E + 1;
 
-  float beta_l[4 * Q];
-  const bool has_bias = beta != nullptr;
-  if (has_bias) load_row<Q>(beta, E, lane, beta_l);
-  else {
+  float beta_l[V];
+  uint32_t valid = 0u;
 #pragma unroll
-    for (int j = 0; j < 4 * Q; ++j) beta_l[j] = 0.f;
+  for (int j = 0; j < V; ++j) {
+    const uint32_t e = slot_expert(lane, j);
+    const bool ok = static_cast<int>(e) < E;
+    valid |= ok ? (1u << j) : 0u;
+    beta_l[j] = (ok && beta) ? beta[e] : 0.f;
   }
-
-  for (int r = warp; r < kSampleRows; r += kRouteWarps) {
-    int64_t s = s0 + r;
+  for (int r = warp; r < kSampleRows; r += kWarps) {
+    const int64_t s = s0 + r;
     if (s >= S) break;
-    int64_t row = s * stride;
-    const float* zrow = z + row * E;
-    float zv[4 * Q];
-    load_row<Q>(zrow, E, lane, zv);
+    const int64_t row = s * stride;
+    float zv[V];
+    load_row<Q>(z + row * E, E, lane, zv);
     float alpha;
     if constexpr (kAlphaIn) {
       alpha = __ldg(alpha_in + row);
     } else {
-      uint32_t key[4 * Q];
-      row_keys<Q>(zv, beta_l, has_bias, E, lane, key);
-      uint32_t out_key, out_id;
-      warp_topk<Q>(key, K, lane, out_key, out_id);
-      alpha = -key_to_float(__shfl_sync(0xffffffffu, out_key, K));
+      // exact (K+1)-th largest biased score by K+1 warp-maximum rounds over
+      // packed (key, id) pairs; only a few thousand rows take this path
+      uint64_t pk[V];
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const float bb = beta ? __fadd_rn(zv[j], beta_l[j]) : zv[j];
+        pk[j] = (valid & (1u << j))
+                    ? ((static_cast<uint64_t>(order_key(bb)) << 32) | (0xffffffffu - slot_expert(lane, j)))
+                    : 0ull;
+      }
+      uint64_t win = 0ull;
+      for (int r2 = 0; r2 <= K; ++r2) {
+        uint64_t mx = 0ull;
+#pragma unroll
+        for (int j = 0; j < V; ++j) mx = pk[j] > mx ? pk[j] : mx;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const uint64_t t = __shfl_xor_sync(0xffffffffu, mx, o);
+          mx = t > mx ? t : mx;
+        }
+        win = mx;
+#pragma unroll
+        for (int j = 0; j < V; ++j)
+          if (pk[j] == mx) pk[j] = 0ull;
+      }
+      alpha = -key_to_float(static_cast<uint32_t>(win >> 32));
     }
 #pragma unroll
-    for (int j = 0; j < 4 * Q; ++j) {
-      int e = static_cast<int>(slot_expert(lane, j));
+    for (int j = 0; j < V; ++j) {
+      const int e = static_cast<int>(slot_expert(lane, j));
       if (e < E) tile[r * ld + e] = order_key(__fadd_rn(zv[j], alpha));
     }
   }
   __syncthreads();
   const int64_t rows_here = (S - s0) < kSampleRows ? (S - s0) : kSampleRows;
-  for (int i = threadIdx.x; i < E * kSampleRows; i += blockDim.x) {
-    int e = i / kSampleRows, r = i % kSampleRows;
+  for (int i = threadIdx.x; i < E * kSampleRows; i += kThreads) {
+    const int e = i / kSampleRows, r = i % kSampleRows;
     if (r < rows_here) sample[static_cast<int64_t>(e) * S + s0 + r] = tile[r * ld + e];
   }
 }
 
-template <int Q>
-cudaError_t launch_route_q(const RouteArgs& a, bool route, bool alpha_out, bool alpha_in,
-                           bool window, cudaStream_t s) {
-  int64_t warps_needed = a.N;
-  int sms = device_sm_count();
-  int64_t blocks = (warps_needed + kRouteWarps - 1) / kRouteWarps;
-  int64_t cap_blocks = static_cast<int64_t>(sms) * 8;
-  if (blocks > cap_blocks) blocks = cap_blocks;
-  if (blocks < 1) blocks = 1;
-  dim3 grid(static_cast<unsigned>(blocks)), block(kRouteThreads);
-  if (route && alpha_out && !window)
-    route_rows_kernel<Q, true, true, false, false><<<grid, block, 0, s>>>(a);
-  else if (route && !alpha_out && !window)
-    route_rows_kernel<Q, true, false, false, false><<<grid, block, 0, s>>>(a);
-  else if (route && alpha_out && window)
-    route_rows_kernel<Q, true, true, false, true><<<grid, block, 0, s>>>(a);
-  else if (!route && alpha_in && window)
-    route_rows_kernel<Q, false, false, true, true><<<grid, block, 0, s>>>(a);
-  else if (!route && !alpha_in && window && alpha_out)
-    route_rows_kernel<Q, false, true, false, true><<<grid, block, 0, s>>>(a);
-  else
-    return cudaErrorInvalidValue;
+template <int Q, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
+cudaError_t launch_rows(const RouteParams& p, cudaStream_t s) {
+  auto kern = route_rows_kernel<Q, kBias, kRoute, kAlphaOut, kAlphaIn, kWindow>;
+  const SmemLayout L = smem_layout<Q, kWindow>(p.E);
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  if (err != cudaSuccess) return err;
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, L.total);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t rows_per_block = static_cast<int64_t>(kWarps) * kRowsPerWarp;
+  int64_t blocks = (p.N + rows_per_block - 1) / rows_per_block;
+  const int64_t resident = static_cast<int64_t>(device_sm_count()) * per_sm;
+  if (blocks > resident) blocks = resident;
+  kern<<<static_cast<unsigned>(blocks), kThreads, L.total, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_route(const RouteArgs& a, bool route, bool alpha_out, bool alpha_in,
-                         bool window, cudaStream_t s) {
-  int Q = (a.E + 127) / 128;
-  switch (Q) {
-    case 1: return launch_route_q<1>(a, route, alpha_out, alpha_in, window, s);
-    case 2: return launch_route_q<2>(a, route, alpha_out, alpha_in, window, s);
-    case 3: return launch_route_q<3>(a, route, alpha_out, alpha_in, window, s);
-    case 4: return launch_route_q<4>(a, route, alpha_out, alpha_in, window, s);
+// route: write ids/gates; alpha_out: write alpha; alpha_in: read alpha
+// instead of selecting; window: bracketed full pass.
+template <int Q>
+cudaError_t dispatch_q(const RouteParams& p, bool route, bool alpha_out, bool alpha_in, bool window,
+                       cudaStream_t s) {
+  const bool bias = p.beta != nullptr;
+#define KOLIBRI_ROWS(B, R, AO, AI, W)                                        \
+  if (bias == B && route == R && alpha_out == AO && alpha_in == AI && window == W) \
+    return launch_rows<Q, B, R, AO, AI, W>(p, s);
+  KOLIBRI_ROWS(true, true, true, false, false)
+  KOLIBRI_ROWS(true, true, false, false, false)
+  KOLIBRI_ROWS(false, true, true, false, false)
+  KOLIBRI_ROWS(false, true, false, false, false)
+  KOLIBRI_ROWS(true, true, true, false, true)
+  KOLIBRI_ROWS(false, true, true, false, true)
+  KOLIBRI_ROWS(true, false, true, false, true)
+  KOLIBRI_ROWS(false, false, true, false, true)
+  KOLIBRI_ROWS(false, false, false, true, true)
+  KOLIBRI_ROWS(true, false, false, true, true)
+#undef KOLIBRI_ROWS
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t dispatch(const RouteParams& p, bool route, bool alpha_out, bool alpha_in, bool window,
+                     cudaStream_t s) {
+  switch ((p.E + 127) / 128) {
+    case 1: return dispatch_q<1>(p, route, alpha_out, alpha_in, window, s);
+    case 2: return dispatch_q<2>(p, route, alpha_out, alpha_in, window, s);
+    case 3: return dispatch_q<3>(p, route, alpha_out, alpha_in, window, s);
+    case 4: return dispatch_q<4>(p, route, alpha_out, alpha_in, window, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -225,17 +452,13 @@ template <int Q>
 cudaError_t launch_sample_q(const float* z, const float* alpha, const float* bias, int64_t N,
                             int E, int K, int64_t S, int64_t stride, uint32_t* sample,
                             cudaStream_t s) {
-  size_t smem = sizeof(uint32_t) * kSampleRows * (E + 1);
-  dim3 grid(static_cast<unsigned>((S + kSampleRows - 1) / kSampleRows)), block(kRouteThreads);
-  if (alpha) {
-    auto k = sample_keys_kernel<Q, true>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    k<<<grid, block, smem, s>>>(z, alpha, bias, N, E, K, S, stride, sample);
-  } else {
-    auto k = sample_keys_kernel<Q, false>;
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    k<<<grid, block, smem, s>>>(z, alpha, bias, N, E, K, S, stride, sample);
-  }
+  const size_t smem = sizeof(uint32_t) * kSampleRows * (E + 1);
+  dim3 grid(static_cast<unsigned>((S + kSampleRows - 1) / kSampleRows)), block(kThreads);
+  auto k = alpha ? sample_keys_kernel<Q, true> : sample_keys_kernel<Q, false>;
+  cudaError_t err =
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  k<<<grid, block, smem, s>>>(z, alpha, bias, N, E, K, S, stride, sample);
   return cudaGetLastError();
 }
 
@@ -243,23 +466,22 @@ cudaError_t launch_sample_q(const float* z, const float* alpha, const float* bia
 
 cudaError_t launch_topk(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
                         int32_t* ids, float* gates, float* alpha, cudaStream_t s) {
-  RouteArgs a{};
-  a.z = z;
-  a.beta = bias;
-  a.N = N;
-  a.E = E;
-  a.K = K;
-  a.ids = ids;
-  a.gates = gates;
-  a.alpha_out = alpha;
-  return launch_route(a, true, alpha != nullptr, false, false, s);
+  RouteParams p{};
+  p.z = z;
+  p.beta = bias;
+  p.N = N;
+  p.E = E;
+  p.K = K;
+  p.ids = ids;
+  p.gates = gates;
+  p.alpha_out = alpha;
+  return dispatch(p, true, alpha != nullptr, false, false, s);
 }
 
 cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* bias, int64_t N,
                               int32_t E, int32_t K, int64_t S, int64_t stride, uint32_t* sample,
                               cudaStream_t s) {
-  int Q = (E + 127) / 128;
-  switch (Q) {
+  switch ((E + 127) / 128) {
     case 1: return launch_sample_q<1>(z, alpha, bias, N, E, K, S, stride, sample, s);
     case 2: return launch_sample_q<2>(z, alpha, bias, N, E, K, S, stride, sample, s);
     case 3: return launch_sample_q<3>(z, alpha, bias, N, E, K, S, stride, sample, s);
@@ -268,26 +490,29 @@ cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* b
   }
 }
 
-cudaError_t launch_eqb_window_pass(const float* z, const float* alpha_in, const float* bias,
-                                   float* alpha_out, int64_t N, int32_t E, int32_t K,
-                                   const uint32_t* lo, const uint32_t* hi, uint32_t* above,
-                                   uint32_t* cnt, uint32_t* cand, int64_t cap, cudaStream_t s) {
-  RouteArgs a{};
-  a.z = z;
-  a.beta = bias;
-  a.N = N;
-  a.E = E;
-  a.K = K;
-  a.alpha_in = alpha_in;
-  a.alpha_out = alpha_out;
-  a.lo = lo;
-  a.hi = hi;
-  a.above = above;
-  a.cand_cnt = cnt;
-  a.cand = cand;
-  a.cap = cap;
-  if (alpha_in) return launch_route(a, false, false, true, true, s);
-  return launch_route(a, false, true, false, true, s);
+cudaError_t launch_route_window_pass(const float* z, const float* bias, const float* alpha_in,
+                                     int64_t N, int32_t E, int32_t K, int32_t* ids, float* gates,
+                                     float* alpha_out, const uint32_t* lo, const uint32_t* hi,
+                                     uint32_t* above, uint32_t* cnt, uint32_t* cand, int64_t cap,
+                                     cudaStream_t s) {
+  RouteParams p{};
+  p.z = z;
+  p.beta = alpha_in ? nullptr : bias;
+  p.N = N;
+  p.E = E;
+  p.K = K;
+  p.ids = ids;
+  p.gates = gates;
+  p.alpha_out = alpha_out;
+  p.alpha_in = alpha_in;
+  p.lo = lo;
+  p.hi = hi;
+  p.above = above;
+  p.cand_cnt = cnt;
+  p.cand = cand;
+  p.cap = cap;
+  const bool route = ids != nullptr;
+  return dispatch(p, route, alpha_out != nullptr, alpha_in != nullptr, true, s);
 }
 
 }  // namespace kolibri

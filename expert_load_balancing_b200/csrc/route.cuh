@@ -7,15 +7,20 @@
 //   alpha_t = -(the (K+1)-th largest B_t,e)  (= -Q_K(Z_t,: + beta))
 //
 // Layout: one warp owns one row.  Lane l holds experts
-//   e = 128*q + 4*l + i,  q = 0..Q-1, i = 0..3
+//   e = 128*q + 4*l + i,  q = 0..Q-1, i = 0..3   (slot j = 4q + i)
 // loaded as Q float4 vectors (each warp-wide load is 512 contiguous bytes).
 //
-// Selection: each lane keeps the two best (key, slot) of its own values.
-// Round r (r = 0..K) takes the warp maximum key with one redux.sync, breaks
-// ties with a redux.sync minimum over expert ids, and the owning lane pops
-// its head.  A lane popped a second time rescans its values below the last
-// popped (key, id) to refill its two best, so every round is exact.  After
-// K+1 rounds lane r holds the r-th (key, id) of the row.
+// Selection in three steps, exact for every input:
+//  1. threshold: the lanes are cut into G groups (G >= K+1); each group's
+//     maximum is a distinct element, so the (K+1)-th largest group maximum T
+//     (or the smallest one when G = 8) is a lower bound of the (K+1)-th
+//     largest score: any element below T is beaten by at least K+1 others;
+//  2. candidates: the elements with score >= T (usually ~3% of the row);
+//  3. K+1 rounds over candidates only: the warp maximum key (redux.sync),
+//     ties to the lowest id (a second redux.sync); the owning lane drops that
+//     candidate and rescans its own few candidates.
+// Scores are compared as order-preserving keys in step 3; steps 1-2 use
+// plain float compares, which only ever admit extra candidates.
 #pragma once
 
 #include "common.cuh"
@@ -24,14 +29,16 @@ namespace kolibri {
 
 constexpr uint32_t kNoId = 0xffffffffu;
 
-template <int Q>
-struct RowSlots {
-  float z[4 * Q];       // raw logits (0 for slots past E)
-  uint32_t key[4 * Q];  // order key of z + beta (0 = absent; finite scores never map to 0)
-};
-
 __device__ __forceinline__ uint32_t slot_expert(int lane, int j) {
   return static_cast<uint32_t>(128 * (j >> 2) + 4 * lane + (j & 3));
+}
+
+// Lane-major position of expert e's value in a row buffer laid out as
+// buf[lane * 4Q + j].
+template <int Q>
+__device__ __forceinline__ int buffer_pos(uint32_t e) {
+  const int q = static_cast<int>(e >> 7), r = static_cast<int>(e & 127);
+  return (r >> 2) * (4 * Q) + 4 * q + (r & 3);
 }
 
 template <int Q>
@@ -49,78 +56,39 @@ __device__ __forceinline__ void load_row(const float* __restrict__ zrow, int E, 
   }
 }
 
-// Biased keys of one row.  beta_lane holds beta for this lane's slots (or
-// nothing when has_bias is false: then B = Z exactly).
-template <int Q>
-__device__ __forceinline__ void row_keys(const float (&z)[4 * Q], const float (&beta_lane)[4 * Q],
-                                         bool has_bias, int E, int lane, uint32_t (&key)[4 * Q]) {
-#pragma unroll
-  for (int j = 0; j < 4 * Q; ++j) {
-    float b = has_bias ? __fadd_rn(z[j], beta_lane[j]) : z[j];
-    key[j] = (static_cast<int>(slot_expert(lane, j)) < E) ? order_key(b) : 0u;
+// Float lower bound T of the (K+1)-th largest of the lanes' values.
+// lane_max is this lane's maximum (-inf if it holds no expert).
+__device__ __forceinline__ float threshold_from_groups(float lane_max, int K) {
+  const unsigned full = 0xffffffffu;
+  if (K + 1 <= 8) {
+    // 8 groups of 4 lanes; T = smallest group maximum
+    float g = fmaxf(lane_max, __shfl_xor_sync(full, lane_max, 1));
+    g = fmaxf(g, __shfl_xor_sync(full, g, 2));
+    float t = fminf(g, __shfl_xor_sync(full, g, 4));
+    t = fminf(t, __shfl_xor_sync(full, t, 8));
+    t = fminf(t, __shfl_xor_sync(full, t, 16));
+    return t;
   }
-}
-
-// Two best (key desc, id asc) among this lane's slots that rank strictly
-// below (below_key, below_id) in that order.  Pass below_key = ~0u and
-// below_id = kNoId... for "no bound" use has_bound = false.
-template <int Q>
-__device__ __forceinline__ void lane_top2(const uint32_t (&key)[4 * Q], int lane, bool has_bound,
-                                          uint32_t below_key, uint32_t below_id, uint32_t& k1,
-                                          int& j1, uint32_t& k2, int& j2) {
-  k1 = 0u;
-  j1 = -1;
-  k2 = 0u;
-  j2 = -1;
-#pragma unroll
-  for (int j = 0; j < 4 * Q; ++j) {
-    uint32_t k = key[j];
-    bool ok = k != 0u;
-    if (has_bound) {
-      uint32_t e = slot_expert(lane, j);
-      ok = ok && (k < below_key || (k == below_key && e > below_id));
-    }
-    // slots ascend in expert id inside a lane, so strict '>' keeps the
-    // lower id ahead on equal keys
-    bool gt1 = ok && k > k1;
-    bool gt2 = ok && k > k2;
-    k2 = gt1 ? k1 : (gt2 ? k : k2);
-    j2 = gt1 ? j1 : (gt2 ? j : j2);
-    k1 = gt1 ? k : k1;
-    j1 = gt1 ? j : j1;
+  // 16 groups of 2 lanes (K+1 <= 16) or 32 groups of 1 lane: bitonic sort of
+  // the group maxima across lanes (descending), then take the (K+1)-th.
+  const int lane = threadIdx.x & 31;
+  float v = lane_max;
+  int stride_lo = 1;
+  if (K + 1 <= 16) {
+    v = fmaxf(v, __shfl_xor_sync(full, v, 1));
+    stride_lo = 2;  // lanes 2g, 2g+1 hold group g
   }
-}
-
-// Exact top-(K+1) of the row.  On return lane r (r <= K) holds the r-th
-// best key in out_key and its expert id in out_id; other lanes hold junk.
-template <int Q>
-__device__ __forceinline__ void warp_topk(const uint32_t (&key)[4 * Q], int K, int lane,
-                                          uint32_t& out_key, uint32_t& out_id) {
-  uint32_t k1, k2;
-  int j1, j2;
-  lane_top2<Q>(key, lane, false, 0u, 0u, k1, j1, k2, j2);
-  bool second_known = true;  // k2/j2 valid
-  out_key = 0u;
-  out_id = kNoId;
-  for (int r = 0; r <= K; ++r) {
-    uint32_t M = __reduce_max_sync(0xffffffffu, k1);
-    uint32_t my_id = (k1 == M && j1 >= 0) ? slot_expert(lane, j1) : kNoId;
-    uint32_t I = __reduce_min_sync(0xffffffffu, my_id);
-    if (lane == r) {
-      out_key = M;
-      out_id = I;
-    }
-    if (my_id == I) {  // exactly one owner: ids are distinct
-      if (second_known) {
-        k1 = k2;
-        j1 = j2;
-        second_known = false;
-      } else {
-        lane_top2<Q>(key, lane, true, M, I, k1, j1, k2, j2);
-        second_known = true;
-      }
+  // sort over the lane bits >= stride_lo, descending in the group index
+  for (int size = 2 * stride_lo; size <= 32; size <<= 1) {
+    for (int stride = size >> 1; stride >= stride_lo; stride >>= 1) {
+      float o = __shfl_xor_sync(full, v, stride);
+      bool up = ((lane & size) == 0);          // descending blocks
+      bool lower = ((lane & stride) == 0);
+      bool take_max = (lower == up);
+      v = take_max ? fmaxf(v, o) : fminf(v, o);
     }
   }
+  return __shfl_sync(full, v, K * stride_lo);
 }
 
 }  // namespace kolibri

@@ -151,6 +151,28 @@ KOLIBRI_API kolibri_status kolibri_eqb_update(const float *z, const float *alpha
                                   void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Routing and the EQB update in one call: the outputs of
+ * kolibri_router_topk(z, bias, ...) followed by kolibri_eqb_update(z, alpha,
+ * bias, ...) on the token biases that routing produced ("Kolibri
+ * Pre-Training from Scratch" 7.1: each step performs one token update, then
+ * one expert update; routing uses the current beta).  Large batches stream Z
+ * from HBM once for both: the bracket of step 2 of the update comes from
+ * sampled rows routed with the same bias, and the routing pass gathers the
+ * bracketed keys.
+ *   z          [N, E] fp32 logits
+ *   bias       [E] fp32: beta used for routing, then overwritten with the
+ *              new centred beta
+ *   ids, gates [N, K], written as by kolibri_router_topk
+ *   alpha      [N] fp32, written if not NULL
+ *   quantiles  [E] fp32, written if not NULL
+ *   ws         device workspace of kolibri_workspace_bytes(KOLIBRI_OP_EQB)
+ */
+KOLIBRI_API kolibri_status kolibri_route_and_balance(const float *z, float *bias, int64_t N,
+                                                     int32_t E, int32_t K, int32_t *ids,
+                                                     float *gates, float *alpha, float *quantiles,
+                                                     void *ws, size_t ws_bytes, void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device: KOLIBRI_OK, KOLIBRI_ERR_TIMEOUT or KOLIBRI_ERR_DEVICE
  * (the first recorded), or KOLIBRI_ERR_CUDA if the synchronisation failed.

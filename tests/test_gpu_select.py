@@ -230,3 +230,39 @@ def test_outputs_fully_written_and_deterministic(oracle_mod):
     ids, gates, alpha = runs[0][:3]
     assert (ids >= 0).all() and np.isfinite(gates).all() and np.isfinite(alpha).all()
     check_status()
+
+
+# ------------------------------------------------ fused routing + EQB
+
+@pytest.mark.parametrize("N,E,K", [(4, 4, 2), (300, 384, 6), (16384, 384, 6), (16385, 384, 6),
+                                   (70001, 384, 6), (65536, 128, 8), (40000, 132, 3)])
+def test_route_and_balance(oracle_mod, N, E, K):
+    z = workloads.random_logits(N, E, seed=N + 3)
+    z[:, : max(1, E // 48)] += np.float32(3.0)
+    beta = workloads.random_logits(1, E, seed=2)[0] * np.float32(0.3)
+    bt = dev(beta.copy())
+    ids, gates, alpha, q = B.kolibri_route_and_balance(dev(z), bt, K)
+    ids_o, gates_o, alpha_o = oracle_mod.select(z, beta, K)
+    assert_bit_equal(host(ids), ids_o, "ids")
+    assert_bit_equal(host(gates), gates_o, "gates")
+    assert_bit_equal(host(alpha), alpha_o, "alpha")
+    v_o = oracle_mod.column_quantiles(z, alpha_o, oracle_mod.eqb_target_rank(N, K, E))
+    assert_bit_equal(host(q), v_o, "quantiles")
+    assert_bit_equal(host(bt), oracle_mod.eqb_bias(v_o), "beta")
+    check_status()
+
+
+def test_route_and_balance_fallback_and_ties(oracle_mod):
+    N, E, K = 131072, 64, 4
+    z = workloads.random_logits(N, E, seed=19)
+    z[:: N // 16384] += np.float32(25.0)      # the sample misleads the bracket
+    z[:1000] = workloads.tied_logits(1000, E, seed=20)
+    bt = dev(np.zeros(E, np.float32))
+    ids, gates, alpha, q = B.kolibri_route_and_balance(dev(z), bt, K, want_alpha=False)
+    ids_o, gates_o, alpha_o = oracle_mod.select(z, np.zeros(E, np.float32), K)
+    assert_bit_equal(host(ids), ids_o, "ids")
+    assert_bit_equal(host(gates), gates_o, "gates")
+    v_o = oracle_mod.column_quantiles(z, alpha_o, oracle_mod.eqb_target_rank(N, K, E))
+    assert_bit_equal(host(q), v_o, "quantiles")
+    assert_bit_equal(host(bt), oracle_mod.eqb_bias(v_o), "beta")
+    check_status()
