@@ -4,18 +4,20 @@
 // "Kolibri 1 im Detail", routing and FP8 sections: the router stays bf16 and
 // its logits are fp32, tokens [N, 2560] -> logits [N, 384].
 //
-// Design (one CTA per SM, persistent over 128-token tiles):
-//   warp 0      TMA producer: x tile [128 x 64] and W [E x 64] per k-block,
-//               128-byte swizzle, into a ring of shared-memory stages;
-//   warp 1      owns the TMEM allocation and issues tcgen05.mma (kind::f16,
-//               bf16 x bf16 -> fp32, M = 128, N = one or two expert chunks of
-//               at most 256) from a single thread, committing each stage
-//               back to the producer and each finished tile to the epilogue;
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (thread = token
-//               row, TMEM lane) and 16-byte stores of Z.
-// The whole E-wide row tile lives in TMEM (E <= 512 columns), so each x tile
-// is read from HBM exactly once and W (<= 0.5 MB per k-block pass) stays in
-// L2.  No cluster multicast is used.
+// Design: persistent kernel, clusters of two CTAs on an SM pair.  A pair
+// owns a 256-token tile; the leader issues tcgen05.mma.cta_group::2 (M = 256,
+// bf16 x bf16 -> fp32, N = one or two expert chunks of at most 256), so each
+// CTA stages its own 128 token rows but only HALF of the router weights: per
+// 64-wide k-block a CTA loads 16 KB of x and E x 64 B of W instead of
+// E x 128 B, which halves the L2 -> SM traffic per FLOP of a one-CTA tile.
+//   warp 0      TMA producer (both CTAs; completions land on the leader's
+//               full barrier)
+//   warp 1      TMEM owner; in the leader, the single MMA-issuing thread
+//   warps 2..5  epilogue: tcgen05.ld (thread = token row = TMEM lane),
+//               registers -> 128B-swizzled shared staging -> TMA tensor store
+// The E-wide accumulator of a tile lives in TMEM (E <= 512 columns), so every
+// x tile is read from HBM once and W stays L2-resident.  No load uses cluster
+// multicast; only tcgen05.commit multicasts its arrival to both CTAs.
 #include <cuda.h>
 
 #include "launch.h"
@@ -25,31 +27,83 @@ namespace kolibri {
 
 namespace {
 
-constexpr int kBM = 128;
+constexpr int kBM = 128;                 // token rows per CTA (256 per pair)
 constexpr int kBK = 64;                  // one 128-byte swizzle atom of bf16
 constexpr int kThreads = 192;
 constexpr int kMaxStages = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kStoreCols = 32;           // fp32 columns per TMA store box
+constexpr int kStageBuf = kStoreCols * 32 * 4;  // 4 KB: 32 rows x 128 B
 constexpr int kSmemLimit = 227 * 1024;
 
 struct GemmShape {
   int64_t N;
   int d, E;
-  int nchunks, chunk_n;   // expert chunks per MMA step and their width
+  int nchunks, chunk_n;   // expert chunks per MMA step (pair-wide width)
   int stages;
   uint32_t tmem_cols;
-  int64_t num_tiles;
+  int64_t num_pairs;      // 256-token tiles
 };
 
 // ---- PTX wrappers -------------------------------------------------------
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
-                                            uint32_t bar, uint64_t policy) {
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t num_clusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// shared::cluster address of the same shared variable in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+// TMA 2D load into this CTA's shared memory; completion bytes are counted on
+// the mbarrier at `bar_cluster` (the pair leader's barrier).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int c0,
+                                                 int c1, uint32_t bar_cluster, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster), "l"(policy)
       : "memory");
 }
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int c0, int c1, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
@@ -70,16 +124,22 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+// Arrive once on the barrier at the same offset in both CTAs of the pair
+// when all previously issued MMAs of this thread have completed.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -124,17 +184,18 @@ __device__ __forceinline__ void tmem_wait_ld() {
 // ---- kernel ---------------------------------------------------------------
 
 __global__ void __launch_bounds__(kThreads, 1)
-    router_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
-                       const __grid_constant__ CUtensorMap tm_w, float* __restrict__ z,
-                       const GemmShape sh) {
+    router_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_x,
+                            const __grid_constant__ CUtensorMap tm_w,
+                            const __grid_constant__ CUtensorMap tm_z, const GemmShape sh) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
+  const int half_n = sh.chunk_n / 2;                       // W rows per CTA per chunk
   const uint32_t a_bytes = kBM * kBK * 2;
-  const uint32_t b_bytes = static_cast<uint32_t>(sh.nchunks * sh.chunk_n) * kBK * 2;
+  const uint32_t b_bytes = static_cast<uint32_t>(sh.nchunks * half_n) * kBK * 2;
   const uint32_t stage_bytes = a_bytes + b_bytes;
-  const uint32_t bars = base + stage_bytes * sh.stages;
-  // barrier block: full[kMaxStages], empty[kMaxStages], tmem_full, tmem_empty, holder
+  const uint32_t staging = base + stage_bytes * sh.stages;  // epilogue buffers (1 KB aligned)
+  const uint32_t bars = staging + kEpiWarps * 2 * kStageBuf;
   auto full_bar = [bars](int s) { return bars + 8u * s; };
   auto empty_bar = [bars](int s) { return bars + 8u * (kMaxStages + s); };
   const uint32_t tmem_full = bars + 8u * (2 * kMaxStages);
@@ -143,7 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* const holder_ptr = smem_raw + (holder - raw);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
   const int k_blocks = sh.d / kBK;
+  const uint32_t cid = cluster_id_x(), ncl = num_clusters_x();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < sh.stages; ++s) {
@@ -151,20 +215,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(empty_bar(s), 1);
     }
     mbar_init(tmem_full, 1);
-    mbar_init(tmem_empty, 128);
+    mbar_init(tmem_empty, 2 * kEpiWarps);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_z)) : "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder),
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder),
                  "r"(sh.tmem_cols)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();          // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(holder_ptr);
 
@@ -175,19 +239,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < sh.num_tiles && ok; tile += gridDim.x) {
+      for (int64_t pt = cid; pt < sh.num_pairs && ok; pt += ncl) {
+        const int row0 = static_cast<int>(pt * 2 * kBM + rank * kBM);
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(stage), stage_bytes);
+          const uint32_t fb = map_to_rank(full_bar(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * stage_bytes);
           const uint32_t a_dst = base + stage_bytes * stage;
           const uint32_t b_dst = a_dst + a_bytes;
-          tma_load_2d(a_dst, &tm_x, kb * kBK, static_cast<int>(tile * kBM), full_bar(stage), pol_x);
+          tma_load_2d_pair(a_dst, &tm_x, kb * kBK, row0, fb, pol_x);
           for (int c = 0; c < sh.nchunks; ++c)
-            tma_load_2d(b_dst + static_cast<uint32_t>(c * sh.chunk_n) * (kBK * 2), &tm_w, kb * kBK,
-                        c * sh.chunk_n, full_bar(stage), pol_w);
+            tma_load_2d_pair(b_dst + static_cast<uint32_t>(c * half_n) * (kBK * 2), &tm_w, kb * kBK,
+                             c * sh.chunk_n + static_cast<int>(rank) * half_n, fb, pol_w);
           if (++stage == sh.stages) {
             stage = 0;
             phase ^= 1u;
@@ -196,12 +262,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = make_idesc(kBM, sh.chunk_n);
+    if (leader && lane == 0) {
+      const uint32_t idesc = make_idesc(2 * kBM, sh.chunk_n);
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < sh.num_tiles && ok; tile += gridDim.x) {
+      for (int64_t pt = cid; pt < sh.num_pairs && ok; pt += ncl) {
         if (!mbar_wait(tmem_empty, acc_phase ^ 1u)) break;
         tc_fence_after();
         for (int kb = 0; kb < k_blocks; ++kb) {
@@ -217,60 +283,72 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < kBK / 16; ++ks) {
             for (int c = 0; c < sh.nchunks; ++c) {
               const uint64_t b_desc =
-                  sw128_desc(b_addr + static_cast<uint32_t>(c * sh.chunk_n) * (kBK * 2));
-              // advancing 16 bf16 along K moves 32 bytes inside the swizzle atom
-              tc_mma(tmem_base + static_cast<uint32_t>(c * sh.chunk_n), a_desc + 2u * ks,
-                     b_desc + 2u * ks, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+                  sw128_desc(b_addr + static_cast<uint32_t>(c * half_n) * (kBK * 2));
+              // 16 bf16 along K = 32 bytes inside the swizzle atom
+              tc_mma_pair(tmem_base + static_cast<uint32_t>(c * sh.chunk_n), a_desc + 2u * ks,
+                          b_desc + 2u * ks, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
             }
           }
-          tc_commit(empty_bar(stage));
+          tc_commit_pair(empty_bar(stage));
           if (++stage == sh.stages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(tmem_full);
+        tc_commit_pair(tmem_full);
         acc_phase ^= 1u;
       }
     }
   } else {
     // epilogue warps 2..5; TMEM lane quarter is fixed by warp % 4
     const int quarter = warp & 3;
+    const int ew = warp - 2;
+    const uint32_t buf0 = staging + static_cast<uint32_t>(ew * 2 * kStageBuf);
+    const uint32_t empty_leader = map_to_rank(tmem_empty, 0);
     uint32_t acc_phase = 0;
-    for (int64_t tile = blockIdx.x; tile < sh.num_tiles; tile += gridDim.x) {
+    int nbuf = 0;
+    for (int64_t pt = cid; pt < sh.num_pairs; pt += ncl) {
       if (!mbar_wait(tmem_full, acc_phase)) break;
       tc_fence_after();
-      const int64_t row = tile * kBM + quarter * 32 + lane;
-      float* zrow = z + row * sh.E;
+      const int row_base = static_cast<int>(pt * 2 * kBM + rank * kBM + quarter * 32);
       const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-      for (int c0 = 0; c0 < sh.E; c0 += 32) {
+      for (int c0 = 0; c0 < sh.E; c0 += kStoreCols) {
         uint32_t r[32];
         tmem_ld32(lane_addr + static_cast<uint32_t>(c0), r);
         tmem_wait_ld();
-        if (row < sh.N) {
-          const int ncols = (sh.E - c0) < 32 ? (sh.E - c0) : 32;
+        // staging buffer: 32 rows x 128 bytes, 16-byte chunks swizzled by row
+        const uint32_t buf = buf0 + static_cast<uint32_t>(nbuf * kStageBuf);
+        if (lane == 0) bulk_wait_read_1();  // the store that last used this buffer has read it
+        __syncwarp();
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (4 * q < ncols) {
-              float4 v = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
-                                     __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
-              *reinterpret_cast<float4*>(zrow + c0 + 4 * q) = v;
-            }
-          }
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t dst = buf + static_cast<uint32_t>(lane * 128 + ((q ^ (lane & 7)) * 16));
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(r[4 * q]),
+                       "r"(r[4 * q + 1]), "r"(r[4 * q + 2]), "r"(r[4 * q + 3])
+                       : "memory");
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_z, c0, row_base, buf);
+          bulk_commit();
+        }
+        nbuf ^= 1;
       }
       tc_fence_before();
-      mbar_arrive(tmem_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(empty_leader);
       acc_phase ^= 1u;
     }
+    if (lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(sh.tmem_cols)
                  : "memory");
   }
@@ -296,16 +374,16 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool encode_bf16_2d(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer,
-                    uint32_t box_inner, uint32_t box_outer) {
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, size_t elem, const void* ptr,
+               uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {inner * elem};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  CUresult r = fn(map, type, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -319,35 +397,63 @@ cudaError_t launch_router_logits(const void* x, const void* w, float* z, int64_t
   sh.d = d;
   sh.E = E;
   sh.nchunks = (E + 255) / 256;
-  int cn = (E + sh.nchunks - 1) / sh.nchunks;
+  const int cn = (E + sh.nchunks - 1) / sh.nchunks;
   sh.chunk_n = (cn + 15) / 16 * 16;
+  if (sh.chunk_n < 32) sh.chunk_n = 32;  // M = 256 needs N >= 32 so each half is >= 16 rows
   const int cols = sh.nchunks * sh.chunk_n;
   uint32_t tc = 32;
   while (tc < static_cast<uint32_t>(cols)) tc <<= 1;
   sh.tmem_cols = tc;
-  const size_t stage_bytes = static_cast<size_t>(kBM) * kBK * 2 + static_cast<size_t>(cols) * kBK * 2;
-  const size_t fixed = 1024 /*alignment slack*/ + 8 * (2 * kMaxStages + 3);
+  const size_t stage_bytes =
+      static_cast<size_t>(kBM) * kBK * 2 + static_cast<size_t>(cols / 2) * kBK * 2;
+  const size_t fixed = 1024 /*alignment slack*/ + kEpiWarps * 2 * kStageBuf + 8 * (2 * kMaxStages + 3);
   int stages = static_cast<int>((kSmemLimit - fixed) / stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return cudaErrorInvalidValue;
   sh.stages = stages;
-  sh.num_tiles = (N + kBM - 1) / kBM;
+  sh.num_pairs = (N + 2 * kBM - 1) / (2 * kBM);
 
-  CUtensorMap tm_x, tm_w;
-  if (!encode_bf16_2d(&tm_x, x, static_cast<uint64_t>(d), static_cast<uint64_t>(N), kBK, kBM))
+  CUtensorMap tm_x, tm_w, tm_z;
+  if (!encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, static_cast<uint64_t>(d),
+                 static_cast<uint64_t>(N), kBK, kBM))
     return cudaErrorInvalidValue;
-  if (!encode_bf16_2d(&tm_w, w, static_cast<uint64_t>(d), static_cast<uint64_t>(E), kBK,
-                      static_cast<uint32_t>(sh.chunk_n)))
+  if (!encode_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, static_cast<uint64_t>(d),
+                 static_cast<uint64_t>(E), kBK, static_cast<uint32_t>(sh.chunk_n / 2)))
+    return cudaErrorInvalidValue;
+  if (!encode_2d(&tm_z, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, z, static_cast<uint64_t>(E),
+                 static_cast<uint64_t>(N), kStoreCols, 32))
     return cudaErrorInvalidValue;
 
   const size_t smem = fixed + stage_bytes * stages;
-  cudaError_t err = cudaFuncSetAttribute(router_gemm_kernel,
+  cudaError_t err = cudaFuncSetAttribute(router_gemm_pair_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  int sms = device_sm_count();
-  int64_t grid = sh.num_tiles < sms ? sh.num_tiles : sms;
-  router_gemm_kernel<<<static_cast<unsigned>(grid), kThreads, smem, s>>>(tm_x, tm_w, z, sh);
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // as many pairs as can be resident at once, at most one per tile
+  static int max_clusters = 0;
+  if (max_clusters == 0) {
+    cfg.gridDim = dim3(2 * static_cast<unsigned>(device_sm_count() / 2), 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, router_gemm_pair_kernel, &cfg) != cudaSuccess || n < 1)
+      n = device_sm_count() / 2;
+    max_clusters = n;
+  }
+  int64_t clusters = sh.num_pairs < max_clusters ? sh.num_pairs : max_clusters;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  err = cudaLaunchKernelEx(&cfg, router_gemm_pair_kernel, tm_x, tm_w, tm_z, sh);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
