@@ -75,7 +75,7 @@ def launches_per_step(N, E, K):
     """Kernels of ours per step: logits 1; routing + EQB 4 (N <= 16384: route,
     sample, select, bias) or 6 (sample, bracket, fused pass, select,
     fallback check, bias); permutation 1 or 3."""
-    route_eqb = 4 if N <= 16384 else 6
+    route_eqb = 4 if N <= 16384 else 7
     permute = 1 if N * K <= 4096 else 3
     return 1 + route_eqb + permute
 

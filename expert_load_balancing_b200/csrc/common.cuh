@@ -9,7 +9,7 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
-#include "../../include/kolibri_router.h"
+#include "kolibri_router.h"
 
 namespace kolibri {
 

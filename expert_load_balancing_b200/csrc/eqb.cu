@@ -135,14 +135,38 @@ __device__ uint32_t block_select_desc(KeyAt key_at, int64_t n, int64_t rank, Sel
   return prefix;
 }
 
+// Keys of one expert staged in shared memory when they fit (kSmemKeys),
+// otherwise read from global memory (L2) on every pass.
+constexpr int kSmemKeys = 16384;
+
+__device__ __forceinline__ int64_t stage_keys(const uint32_t* __restrict__ keys, int64_t n,
+                                              uint32_t* keys_s) {
+  if (n > kSmemKeys) return n;
+  // 16-byte vector loads only from a 16-byte aligned source
+  const bool vec = (reinterpret_cast<uintptr_t>(keys) & 15u) == 0u;
+  const int64_t n4 = vec ? (n & ~static_cast<int64_t>(3)) : 0;
+  for (int64_t i = 4 * threadIdx.x; i < n4; i += 4 * blockDim.x)
+    *reinterpret_cast<uint4*>(keys_s + i) = __ldg(reinterpret_cast<const uint4*>(keys + i));
+  for (int64_t i = n4 + threadIdx.x; i < n; i += blockDim.x) keys_s[i] = __ldg(keys + i);
+  __syncthreads();
+  return n;
+}
+
 // Step 2 (or the whole selection when the sample is the column).
 __global__ void __launch_bounds__(kSelThreads) sample_select_kernel(
     const uint32_t* __restrict__ sample, int64_t S, int64_t m_exact, int64_t r_hi, int64_t r_lo,
-    bool exact, float* __restrict__ v, uint32_t* __restrict__ lo, uint32_t* __restrict__ hi) {
+    int64_t S_ld, bool exact, float* __restrict__ v, uint32_t* __restrict__ lo,
+    uint32_t* __restrict__ hi) {
   __shared__ SelectSmem sm;
+  extern __shared__ __align__(16) uint32_t keys_s[];
   const int e = blockIdx.x;
-  const uint32_t* keys = sample + static_cast<int64_t>(e) * S;
-  auto at = [keys](int64_t i) { return __ldg(keys + i); };
+  const uint32_t* keys = sample + static_cast<int64_t>(e) * S_ld;
+  stage_keys(keys, S, keys_s);
+  const bool in_smem = S <= kSmemKeys;
+  auto at = [keys, in_smem](int64_t i) {
+    extern __shared__ __align__(16) uint32_t ks[];
+    return in_smem ? ks[i] : __ldg(keys + i);
+  };
   if (exact) {
     uint32_t k = block_select_desc(at, S, m_exact, sm);
     if (threadIdx.x == 0) v[e] = key_to_float(k);
@@ -162,6 +186,7 @@ __global__ void __launch_bounds__(kSelThreads) bracket_select_kernel(
     const uint32_t* __restrict__ above, int64_t cap, int64_t m, float* __restrict__ v,
     uint32_t* __restrict__ flag) {
   __shared__ SelectSmem sm;
+  extern __shared__ __align__(16) uint32_t keys_s[];
   const int e = blockIdx.x;
   const int64_t c = cnt[e], ab = above[e];
   const bool ok = c <= cap && ab <= m && m < ab + c;
@@ -170,7 +195,12 @@ __global__ void __launch_bounds__(kSelThreads) bracket_select_kernel(
     return;
   }
   const uint32_t* keys = cand + static_cast<int64_t>(e) * cap;
-  auto at = [keys](int64_t i) { return __ldg(keys + i); };
+  stage_keys(keys, c, keys_s);
+  const bool in_smem = c <= kSmemKeys;
+  auto at = [keys, in_smem](int64_t i) {
+    extern __shared__ __align__(16) uint32_t ks[];
+    return in_smem ? ks[i] : __ldg(keys + i);
+  };
   uint32_t k = block_select_desc(at, c, m - ab, sm);
   if (threadIdx.x == 0) {
     v[e] = key_to_float(k);
@@ -197,9 +227,12 @@ __global__ void __launch_bounds__(kSelThreads) column_fallback_kernel(
 __global__ void bias_update_kernel(const float* __restrict__ v, int E, float* __restrict__ bias,
                                    float* __restrict__ quantiles) {
   __shared__ float mean_s;
+  __shared__ float v_s[KOLIBRI_MAX_EXPERTS];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) v_s[e] = v[e];
+  __syncthreads();
   if (threadIdx.x == 0) {
     double sum = 0.0;
-    for (int e = 0; e < E; ++e) sum = __dadd_rn(sum, static_cast<double>(-v[e]));
+    for (int e = 0; e < E; ++e) sum = __dadd_rn(sum, static_cast<double>(-v_s[e]));
     mean_s = __double2float_rn(__ddiv_rn(sum, static_cast<double>(E)));
   }
   __syncthreads();
@@ -224,7 +257,8 @@ EqbLayout eqb_layout(int64_t N, int32_t E, int32_t K) {
     off += align256(bytes);
     return o;
   };
-  L.off_sample = take(sizeof(uint32_t) * static_cast<size_t>(E) * static_cast<size_t>(L.S));
+  L.S_ld = (L.S + 3) & ~static_cast<int64_t>(3);  // 16-byte aligned expert rows
+  L.off_sample = take(sizeof(uint32_t) * static_cast<size_t>(E) * static_cast<size_t>(L.S_ld));
   L.off_lo = take(sizeof(uint32_t) * E);
   L.off_hi = take(sizeof(uint32_t) * E);
   L.off_above = take(sizeof(uint32_t) * E);
@@ -239,6 +273,19 @@ EqbLayout eqb_layout(int64_t N, int32_t E, int32_t K) {
 }
 
 namespace {
+
+size_t select_smem(int64_t n) {
+  return sizeof(uint32_t) * static_cast<size_t>(n < kSmemKeys ? n : kSmemKeys);
+}
+
+cudaError_t set_select_smem() {
+  const int bytes = static_cast<int>(sizeof(uint32_t) * kSmemKeys);
+  cudaError_t err = cudaFuncSetAttribute(sample_select_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err != cudaSuccess) return err;
+  return cudaFuncSetAttribute(bracket_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              bytes);
+}
 
 struct EqbBuffers {
   EqbLayout L;
@@ -271,10 +318,13 @@ cudaError_t eqb_begin(const float* z, const float* alpha, const float* bias, int
   const EqbLayout& L = b.L;
   const int64_t m = (N * static_cast<int64_t>(K)) / E;
   cudaError_t err = launch_eqb_sample(z, alpha, alpha ? nullptr : bias, N, E, K, L.S, L.stride,
-                                      b.sample, s);
+                                      L.S_ld, b.sample, s);
   if (err != cudaSuccess) return err;
   if (L.exact_small) {
-    sample_select_kernel<<<E, kSelThreads, 0, s>>>(b.sample, L.S, m, 0, 0, true, b.v, b.lo, b.hi);
+    err = set_select_smem();
+    if (err != cudaSuccess) return err;
+    sample_select_kernel<<<E, kSelThreads, select_smem(L.S), s>>>(b.sample, L.S, m, 0, 0, L.S_ld,
+                                                                   true, b.v, b.lo, b.hi);
     return cudaGetLastError();
   }
   // bracket ranks in the sample, descending order: the target sits at
@@ -289,8 +339,10 @@ cudaError_t eqb_begin(const float* z, const float* alpha, const float* bias, int
   if (r_lo > L.S - 1) r_lo = L.S - 1;
   err = cudaMemsetAsync(b.base + L.off_above, 0, L.off_v - L.off_above, s);  // above, cnt, flag
   if (err != cudaSuccess) return err;
-  sample_select_kernel<<<E, kSelThreads, 0, s>>>(b.sample, L.S, 0, r_hi, r_lo, false, b.v, b.lo,
-                                                 b.hi);
+  err = set_select_smem();
+  if (err != cudaSuccess) return err;
+  sample_select_kernel<<<E, kSelThreads, select_smem(L.S), s>>>(b.sample, L.S, 0, r_hi, r_lo,
+                                                                 L.S_ld, false, b.v, b.lo, b.hi);
   return cudaGetLastError();
 }
 
@@ -300,8 +352,10 @@ cudaError_t eqb_end(const float* z, const float* alpha_used, float* bias, int64_
   const int64_t m = (N * static_cast<int64_t>(K)) / E;
   cudaError_t err;
   if (!b.L.exact_small) {
-    bracket_select_kernel<<<E, kSelThreads, 0, s>>>(b.cand, b.cnt, b.above, kCandCap, m, b.v,
-                                                    b.flag);
+    err = set_select_smem();
+    if (err != cudaSuccess) return err;
+    bracket_select_kernel<<<E, kSelThreads, select_smem(kSmemKeys), s>>>(b.cand, b.cnt, b.above,
+                                                                          kCandCap, m, b.v, b.flag);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     column_fallback_kernel<<<E, kSelThreads, 0, s>>>(z, alpha_used, N, E, m, b.flag, b.v);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
@@ -342,12 +396,15 @@ cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t
     err = eqb_begin(z, alpha_out, bias, N, E, K, b, s);
     if (err != cudaSuccess) return err;
   } else {
-    // the bracket comes from sampled rows routed with the same bias; one
-    // pass then routes every row and feeds the bracket
-    err = eqb_begin(z, nullptr, bias, N, E, K, b, s);
+    // Routing first (writes alpha), then the bracketed pass with alpha given.
+    // Two streams over Z; a single fused pass measured slower on B200 (its
+    // per-row dependency chain is longer than 24 warps per SM can hide).
+    err = launch_topk(z, bias, N, E, K, ids, gates, alpha_out, s);
     if (err != cudaSuccess) return err;
-    err = launch_route_window_pass(z, bias, nullptr, N, E, K, ids, gates, alpha_out, b.lo, b.hi,
-                                   b.above, b.cnt, b.cand, kCandCap, s);
+    err = eqb_begin(z, alpha_out, bias, N, E, K, b, s);
+    if (err != cudaSuccess) return err;
+    err = launch_route_window_pass(z, bias, alpha_out, N, E, K, nullptr, nullptr, nullptr, b.lo,
+                                   b.hi, b.above, b.cnt, b.cand, kCandCap, s);
     if (err != cudaSuccess) return err;
   }
   return eqb_end(z, alpha_out, bias, N, E, K, quantiles, b, s);

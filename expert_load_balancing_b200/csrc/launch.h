@@ -14,6 +14,7 @@ constexpr int64_t kCandCap = 65536;
 
 struct EqbLayout {
   int64_t S = 0, stride = 1;
+  int64_t S_ld = 0;           // row stride of the sample buffer (multiple of 4)
   bool exact_small = false;   // S == N: the sample is the whole column
   size_t off_sample = 0;      // u32 [E][S]   keys of Z + alpha at sampled rows
   size_t off_lo = 0;          // u32 [E]      lower bracket key
@@ -58,8 +59,8 @@ cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t
 
 // pieces of the EQB update living in route.cu (they walk rows of Z)
 cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* bias, int64_t N,
-                              int32_t E, int32_t K, int64_t S, int64_t stride, uint32_t* sample,
-                              cudaStream_t s);
+                              int32_t E, int32_t K, int64_t S, int64_t stride, int64_t S_ld,
+                              uint32_t* sample, cudaStream_t s);
 // Bracketed full pass.  alpha_in given: use it.  Otherwise alpha is derived
 // from bias (and written to alpha_out); with ids/gates non-null the same
 // pass also writes the routing.

@@ -24,7 +24,7 @@ namespace {
 
 constexpr int kPermThreads = 256;
 constexpr int kPermWarps = kPermThreads / kWarp;
-constexpr int64_t kChunk = 4096;        // slots per warp chunk
+constexpr int64_t kChunk = 1024;        // slots per warp chunk
 constexpr int64_t kSingleMax = 4096;    // N*K handled by one block
 constexpr int kUnroll = 8;
 
@@ -108,17 +108,35 @@ __global__ void __launch_bounds__(kPermThreads) chunk_scan_kernel(
   __syncthreads();
   if (!last_s) return;
   __threadfence();
-  if (threadIdx.x == 0) {
-    int64_t run = 0;
-    for (int x = 0; x < E; ++x) {
-      uint32_t cx = *reinterpret_cast<volatile uint32_t*>(totals + x);
-      offsets[x] = run;
-      counts[x] = static_cast<int32_t>(cx);
-      run += cx;
-    }
-    offsets[E] = run;
-    *ticket = 0u;  // ready for the next call
+  // exclusive scan of the E totals by the whole block (E <= 512: two per thread)
+  __shared__ uint32_t tot_s[KOLIBRI_MAX_EXPERTS];
+  for (int x = threadIdx.x; x < E; x += kPermThreads)
+    tot_s[x] = *reinterpret_cast<volatile uint32_t*>(totals + x);
+  __syncthreads();
+  const int x0 = 2 * threadIdx.x;
+  const uint32_t a0 = x0 < E ? tot_s[x0] : 0u, a1 = x0 + 1 < E ? tot_s[x0 + 1] : 0u;
+  const uint32_t pair = a0 + a1;
+  uint32_t incl = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
   }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  uint32_t wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += warp_sums[w];
+  const uint32_t excl = wbase + incl - pair;
+  if (x0 < E) {
+    offsets[x0] = excl;
+    counts[x0] = static_cast<int32_t>(a0);
+  }
+  if (x0 + 1 < E) {
+    offsets[x0 + 1] = excl + a0;
+    counts[x0 + 1] = static_cast<int32_t>(a1);
+  }
+  if (x0 + 1 == E || x0 + 2 == E) offsets[E] = excl + pair;  // the thread holding the last expert
+  if (threadIdx.x == 0) *ticket = 0u;  // ready for the next call
 }
 
 __device__ __forceinline__ void scatter_round(int32_t e, int64_t j, int lane, uint32_t* cursor,

@@ -45,11 +45,9 @@ struct RouteParams {
 
 template <int Q>
 struct WarpScratch {
-  float row[128 * Q];   // this row's raw logits, lane-major
+  RowScratch<Q> sel;    // selection scratch (row buffer, compacted candidates)
   float gz[32];         // gate inputs waiting for a batched evaluation
   uint32_t gidx[32];    // their output positions
-  uint32_t ckey[32];    // compacted candidates: key and expert id
-  uint32_t cid[32];
 };
 
 // Shared-memory layout (dynamic): beta[E] | lo[E] | hi[E] | above[E] |
@@ -82,18 +80,28 @@ __host__ __device__ SmemLayout smem_layout(int E) {
   return L;
 }
 
-__device__ __forceinline__ float z_of(const float* row, int lane, int j, int V) {
-  return row[lane * V + j];
-}
-
 // Evaluate the staged gates (lanes < n) and store them.
 __device__ __forceinline__ void flush_gates(float* __restrict__ gates, const float* gz,
                                             const uint32_t* gidx, int n, int lane) {
   if (lane < n) gates[gidx[lane]] = gate_sigmoid(gz[lane]);
 }
 
-template <int Q, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
-__global__ void __launch_bounds__(kThreads, 3) route_rows_kernel(const RouteParams p) {
+// Append one bracketed key of expert e: block staging, or the global gather
+// buffer directly when the block's slots for e are full.
+__device__ __forceinline__ void stage_bracket_key(uint32_t e, uint32_t k, uint32_t* stage_n,
+                                                  uint32_t* stage, uint32_t* __restrict__ cand_cnt,
+                                                  uint32_t* __restrict__ cand, int64_t cap) {
+  const uint32_t pos = atomicAdd(&stage_n[e], 1u);
+  if (pos < kStageSlots) {
+    stage[e * kStageSlots + pos] = k;
+  } else {
+    const uint32_t g = atomicAdd(cand_cnt + e, 1u);
+    if (g < cap) cand[static_cast<int64_t>(e) * cap + g] = k;
+  }
+}
+
+template <int Q, bool kFull, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
+__global__ void __launch_bounds__(kThreads, kAlphaIn ? 4 : 3) route_rows_kernel(const RouteParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int V = 4 * Q;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -118,8 +126,7 @@ __global__ void __launch_bounds__(kThreads, 3) route_rows_kernel(const RoutePara
   }
   __syncthreads();
 
-  // valid-slot mask of this lane (fixed for the kernel)
-  uint32_t valid = 0u;
+  uint32_t valid = 0u;  // this lane's slots that hold an expert
 #pragma unroll
   for (int j = 0; j < V; ++j) valid |= (static_cast<int>(slot_expert(lane, j)) < E) ? (1u << j) : 0u;
   int gate_n = 0;
@@ -129,123 +136,42 @@ __global__ void __launch_bounds__(kThreads, 3) route_rows_kernel(const RoutePara
        base += static_cast<int64_t>(gridDim.x) * rows_per_block) {
     const int64_t r0 = base + static_cast<int64_t>(warp) * kRowsPerWarp;
     const int64_t r1 = (r0 + kRowsPerWarp < p.N) ? r0 + kRowsPerWarp : p.N;
+    // per-lane counts of keys above the bracket, one byte per slot (<= 32 rows per batch)
+    uint32_t above_b[kWindow ? Q : 1];
+    if constexpr (kWindow) {
+#pragma unroll
+      for (int q = 0; q < Q; ++q) above_b[q] = 0u;
+    }
     float znext[V];
-    if (r0 < r1) load_row<Q>(p.z + r0 * E, E, lane, znext);
+    float anext = 0.f;
+    if (r0 < r1) {
+      load_row<Q, kFull>(p.z + r0 * E, E, lane, znext);
+      if constexpr (kAlphaIn) anext = __ldg(p.alpha_in + r0);
+    }
     for (int64_t row = r0; row < r1; ++row) {
       float z[V];
 #pragma unroll
       for (int j = 0; j < V; ++j) z[j] = znext[j];
-      if (row + 1 < r1) load_row<Q>(p.z + (row + 1) * E, E, lane, znext);
+      const float acur = anext;
+      if (row + 1 < r1) {
+        load_row<Q, kFull>(p.z + (row + 1) * E, E, lane, znext);
+        if constexpr (kAlphaIn) anext = __ldg(p.alpha_in + row + 1);
+      }
 
       float alpha;
       if constexpr (!kAlphaIn) {
-        // ---- scores, lane maximum, threshold, candidate mask
-        float b[V];
-        float lane_max = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < Q; ++q) {
-          float4 bq = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (kBias && (valid & (1u << (4 * q))))
-            bq = *reinterpret_cast<const float4*>(&beta_s[128 * q + 4 * lane]);
-          const float bv[4] = {bq.x, bq.y, bq.z, bq.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int j = 4 * q + i;
-            b[j] = kBias ? __fadd_rn(z[j], bv[i]) : z[j];
-            if (valid & (1u << j)) lane_max = fmaxf(lane_max, b[j]);
-          }
-        }
-        const float T = threshold_from_groups(lane_max, K);
-        uint32_t cand = 0u;
-#pragma unroll
-        for (int j = 0; j < V; ++j) cand |= (b[j] >= T) ? (1u << j) : 0u;
-        cand &= valid;
-        // raw logits to the row buffer for indexed access
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < Q; ++q)
-          *reinterpret_cast<float4*>(&ws.row[lane * V + 4 * q]) =
-              make_float4(z[4 * q], z[4 * q + 1], z[4 * q + 2], z[4 * q + 3]);
-        // ---- compact the candidates to at most one per lane
-        const int c = __popc(cand);
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        const int total = __shfl_sync(0xffffffffu, incl, 31);
-        uint32_t out_key = 0u, out_id = kNoId;
-        if (total <= 32) {
-          int pos = incl - c;
-          uint32_t m = cand;
-          while (m) {
-            const int j = __ffs(m) - 1;
-            m &= m - 1u;
-            const uint32_t e = slot_expert(lane, j);
-            const float bb = kBias ? __fadd_rn(z_of(ws.row, lane, j, V), beta_s[e]) : z_of(ws.row, lane, j, V);
-            ws.ckey[pos] = order_key(bb);
-            ws.cid[pos] = e;
-            ++pos;
-          }
-          __syncwarp();
-          uint32_t k = lane < total ? ws.ckey[lane] : 0u;
-          uint32_t id = lane < total ? ws.cid[lane] : kNoId;
-          for (int r = 0; r <= K; ++r) {
-            const uint32_t M = __reduce_max_sync(0xffffffffu, k);
-            const uint32_t mine = (k == M) ? id : kNoId;
-            const uint32_t I = __reduce_min_sync(0xffffffffu, mine);
-            if (lane == r) {
-              out_key = M;
-              out_id = I;
-            }
-            if (id == I) {  // the owner (ids are distinct); I == kNoId only for bad input
-              k = 0u;
-              id = kNoId;
-            }
-          }
-        } else {
-          // many candidates (heavy ties): K+1 rounds, each owner rescans its own
-          __syncwarp();
-          auto lane_best = [&](uint32_t mm, uint32_t& bk, uint32_t& bid) {
-            bk = 0u;
-            bid = kNoId;
-            while (mm) {
-              const int j = __ffs(mm) - 1;
-              mm &= mm - 1u;
-              const uint32_t e = slot_expert(lane, j);
-              const float zz = z_of(ws.row, lane, j, V);
-              const uint32_t k = order_key(kBias ? __fadd_rn(zz, beta_s[e]) : zz);
-              if (k > bk) {  // slots ascend in id: strict '>' keeps the lower id
-                bk = k;
-                bid = e;
-              }
-            }
-          };
-          uint32_t bk, bid;
-          lane_best(cand, bk, bid);
-          for (int r = 0; r <= K; ++r) {
-            const uint32_t M = __reduce_max_sync(0xffffffffu, bk);
-            const uint32_t mine = (bk == M) ? bid : kNoId;
-            const uint32_t I = __reduce_min_sync(0xffffffffu, mine);
-            if (lane == r) {
-              out_key = M;
-              out_id = I;
-            }
-            if (bid == I && I != kNoId) {
-              cand &= ~(1u << (4 * static_cast<int>(I >> 7) + static_cast<int>(I & 3)));
-              lane_best(cand, bk, bid);
-            }
-          }
-        }
-        alpha = -key_to_float(__shfl_sync(0xffffffffu, out_key, K));
+        int rank;
+        uint32_t key, id;
+        warp_select_row<Q, kFull, kBias>(z, beta_s, valid, K, lane, ws.sel, rank, key, id);
+        const uint32_t kth = __ballot_sync(0xffffffffu, rank == K);
+        alpha = -key_to_float(__shfl_sync(0xffffffffu, key, __ffs(kth) - 1));
         if constexpr (kRoute) {
-          if (lane < K) {
-            // out_id < E for finite inputs; clamp so no input can index outside
-            const uint32_t e = out_id < static_cast<uint32_t>(E) ? out_id : 0u;
-            p.ids[row * K + lane] = static_cast<int32_t>(out_id);
-            ws.gz[gate_n + lane] = ws.row[buffer_pos<Q>(e)];
-            ws.gidx[gate_n + lane] = static_cast<uint32_t>(row * K + lane);
+          if (rank >= 0 && rank < K) {
+            // id < E for finite inputs; clamp so no input can index outside
+            const uint32_t e = id < static_cast<uint32_t>(E) ? id : 0u;
+            p.ids[row * K + rank] = static_cast<int32_t>(id);
+            ws.gz[gate_n + rank] = ws.sel.row[buffer_pos<Q>(e)];
+            ws.gidx[gate_n + rank] = static_cast<uint32_t>(row * K + rank);
           }
           gate_n += K;
           if (gate_n + K > 32) {
@@ -259,13 +185,14 @@ __global__ void __launch_bounds__(kThreads, 3) route_rows_kernel(const RoutePara
         }
         __syncwarp();
       } else {
-        alpha = __ldg(p.alpha_in + row);
+        alpha = acur;
       }
 
       if constexpr (kWindow) {
+        uint32_t wmask = 0u;
 #pragma unroll
         for (int q = 0; q < Q; ++q) {
-          if (!(valid & (1u << (4 * q)))) continue;
+          if (!kFull && !(valid & (1u << (4 * q)))) continue;
           const int e0 = 128 * q + 4 * lane;
           const uint4 hq = *reinterpret_cast<const uint4*>(&hi_s[e0]);
           const uint4 lq = *reinterpret_cast<const uint4*>(&lo_s[e0]);
@@ -274,22 +201,30 @@ __global__ void __launch_bounds__(kThreads, 3) route_rows_kernel(const RoutePara
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const uint32_t k = order_key(__fadd_rn(z[4 * q + i], alpha));
-            if (k > hv[i]) {
-              atomicAdd(&above_s[e0 + i], 1u);
-            } else if (k >= lv[i]) {
-              const uint32_t pos = atomicAdd(&stage_n[e0 + i], 1u);
-              if (pos < kStageSlots) {
-                stage[(e0 + i) * kStageSlots + pos] = k;
-              } else {  // block buffer full: append directly
-                const uint32_t g = atomicAdd(p.cand_cnt + e0 + i, 1u);
-                if (g < p.cap) p.cand[static_cast<int64_t>(e0 + i) * p.cap + g] = k;
-              }
-            }
+            const bool ab = k > hv[i];
+            above_b[q] += ab ? (1u << (8 * i)) : 0u;
+            wmask |= (!ab && k >= lv[i]) ? (1u << (4 * q + i)) : 0u;
           }
+        }
+        while (wmask) {  // rare: keys inside the bracket
+          const int j = __ffs(wmask) - 1;
+          wmask &= wmask - 1u;
+          const uint32_t e = slot_expert(lane, j);
+          const uint32_t k = order_key(__fadd_rn(__ldg(p.z + row * E + e), alpha));
+          stage_bracket_key(e, k, stage_n, stage, p.cand_cnt, p.cand, p.cap);
         }
       }
     }
     if constexpr (kWindow) {
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        if (above_b[q] == 0u) continue;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t n = (above_b[q] >> (8 * i)) & 0xffu;
+          if (n) atomicAdd(&above_s[128 * q + 4 * lane + i], n);
+        }
+      }
       __syncthreads();
       for (int e = threadIdx.x; e < E; e += kThreads) {
         uint32_t n = stage_n[e];
@@ -320,63 +255,45 @@ __global__ void __launch_bounds__(kThreads, 3) route_rows_kernel(const RoutePara
 // them through shared memory so every expert row is written in 128-byte runs.
 constexpr int kSampleRows = 32;
 
-template <int Q, bool kAlphaIn>
+template <int Q, bool kAlphaIn, bool kBias>
 __global__ void __launch_bounds__(kThreads) sample_keys_kernel(
     const float* __restrict__ z, const float* __restrict__ alpha_in, const float* __restrict__ beta,
-    int64_t N, int E, int K, int64_t S, int64_t stride, uint32_t* __restrict__ sample) {
+    int64_t N, int E, int K, int64_t S, int64_t stride, int64_t S_ld,
+    uint32_t* __restrict__ sample) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int V = 4 * Q;
+  const int ld = E + 1;
   uint32_t* tile = reinterpret_cast<uint32_t*>(smem);  // [kSampleRows][E + 1]
+  float* beta_s = reinterpret_cast<float*>(smem + ((4 * kSampleRows * ld + 15) & ~15));
+  RowScratch<Q>* scr = reinterpret_cast<RowScratch<Q>*>(
+      smem + ((4 * kSampleRows * ld + 15) & ~15) + ((4 * E + 15) & ~15));
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t s0 = static_cast<int64_t>(blockIdx.x) * kSampleRows;
-  const int ld = E + 1;
-
-  float beta_l[V];
+  if constexpr (kBias) {
+    for (int e = threadIdx.x; e < E; e += kThreads) beta_s[e] = beta[e];
+  }
+  __syncthreads();
   uint32_t valid = 0u;
 #pragma unroll
-  for (int j = 0; j < V; ++j) {
-    const uint32_t e = slot_expert(lane, j);
-    const bool ok = static_cast<int>(e) < E;
-    valid |= ok ? (1u << j) : 0u;
-    beta_l[j] = (ok && beta) ? beta[e] : 0.f;
-  }
+  for (int j = 0; j < V; ++j) valid |= (static_cast<int>(slot_expert(lane, j)) < E) ? (1u << j) : 0u;
+
   for (int r = warp; r < kSampleRows; r += kWarps) {
     const int64_t s = s0 + r;
     if (s >= S) break;
     const int64_t row = s * stride;
     float zv[V];
-    load_row<Q>(z + row * E, E, lane, zv);
+    load_row<Q, false>(z + row * E, E, lane, zv);
     float alpha;
     if constexpr (kAlphaIn) {
       alpha = __ldg(alpha_in + row);
     } else {
-      // exact (K+1)-th largest biased score by K+1 warp-maximum rounds over
-      // packed (key, id) pairs; only a few thousand rows take this path
-      uint64_t pk[V];
-#pragma unroll
-      for (int j = 0; j < V; ++j) {
-        const float bb = beta ? __fadd_rn(zv[j], beta_l[j]) : zv[j];
-        pk[j] = (valid & (1u << j))
-                    ? ((static_cast<uint64_t>(order_key(bb)) << 32) | (0xffffffffu - slot_expert(lane, j)))
-                    : 0ull;
-      }
-      uint64_t win = 0ull;
-      for (int r2 = 0; r2 <= K; ++r2) {
-        uint64_t mx = 0ull;
-#pragma unroll
-        for (int j = 0; j < V; ++j) mx = pk[j] > mx ? pk[j] : mx;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const uint64_t t = __shfl_xor_sync(0xffffffffu, mx, o);
-          mx = t > mx ? t : mx;
-        }
-        win = mx;
-#pragma unroll
-        for (int j = 0; j < V; ++j)
-          if (pk[j] == mx) pk[j] = 0ull;
-      }
-      alpha = -key_to_float(static_cast<uint32_t>(win >> 32));
+      int rank;
+      uint32_t key, id;
+      warp_select_row<Q, false, kBias>(zv, beta_s, valid, K, lane, scr[warp], rank, key, id);
+      const uint32_t kth = __ballot_sync(0xffffffffu, rank == K);
+      alpha = -key_to_float(__shfl_sync(0xffffffffu, key, __ffs(kth) - 1));
+      __syncwarp();
     }
 #pragma unroll
     for (int j = 0; j < V; ++j) {
@@ -388,13 +305,13 @@ __global__ void __launch_bounds__(kThreads) sample_keys_kernel(
   const int64_t rows_here = (S - s0) < kSampleRows ? (S - s0) : kSampleRows;
   for (int i = threadIdx.x; i < E * kSampleRows; i += kThreads) {
     const int e = i / kSampleRows, r = i % kSampleRows;
-    if (r < rows_here) sample[static_cast<int64_t>(e) * S + s0 + r] = tile[r * ld + e];
+    if (r < rows_here) sample[static_cast<int64_t>(e) * S_ld + s0 + r] = tile[r * ld + e];
   }
 }
 
-template <int Q, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
+template <int Q, bool kFull, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
 cudaError_t launch_rows(const RouteParams& p, cudaStream_t s) {
-  auto kern = route_rows_kernel<Q, kBias, kRoute, kAlphaOut, kAlphaIn, kWindow>;
+  auto kern = route_rows_kernel<Q, kFull, kBias, kRoute, kAlphaOut, kAlphaIn, kWindow>;
   const SmemLayout L = smem_layout<Q, kWindow>(p.E);
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
@@ -416,13 +333,13 @@ cudaError_t launch_rows(const RouteParams& p, cudaStream_t s) {
 
 // route: write ids/gates; alpha_out: write alpha; alpha_in: read alpha
 // instead of selecting; window: bracketed full pass.
-template <int Q>
+template <int Q, bool kFull>
 cudaError_t dispatch_q(const RouteParams& p, bool route, bool alpha_out, bool alpha_in, bool window,
                        cudaStream_t s) {
   const bool bias = p.beta != nullptr;
-#define KOLIBRI_ROWS(B, R, AO, AI, W)                                        \
+#define KOLIBRI_ROWS(B, R, AO, AI, W)                                                   \
   if (bias == B && route == R && alpha_out == AO && alpha_in == AI && window == W) \
-    return launch_rows<Q, B, R, AO, AI, W>(p, s);
+    return launch_rows<Q, kFull, B, R, AO, AI, W>(p, s);
   KOLIBRI_ROWS(true, true, true, false, false)
   KOLIBRI_ROWS(true, true, false, false, false)
   KOLIBRI_ROWS(false, true, true, false, false)
@@ -432,33 +349,39 @@ cudaError_t dispatch_q(const RouteParams& p, bool route, bool alpha_out, bool al
   KOLIBRI_ROWS(true, false, true, false, true)
   KOLIBRI_ROWS(false, false, true, false, true)
   KOLIBRI_ROWS(false, false, false, true, true)
-  KOLIBRI_ROWS(true, false, false, true, true)
 #undef KOLIBRI_ROWS
   return cudaErrorInvalidValue;
 }
 
 cudaError_t dispatch(const RouteParams& p, bool route, bool alpha_out, bool alpha_in, bool window,
                      cudaStream_t s) {
+  const bool full = (p.E % 128) == 0;
   switch ((p.E + 127) / 128) {
-    case 1: return dispatch_q<1>(p, route, alpha_out, alpha_in, window, s);
-    case 2: return dispatch_q<2>(p, route, alpha_out, alpha_in, window, s);
-    case 3: return dispatch_q<3>(p, route, alpha_out, alpha_in, window, s);
-    case 4: return dispatch_q<4>(p, route, alpha_out, alpha_in, window, s);
+    case 1: return full ? dispatch_q<1, true>(p, route, alpha_out, alpha_in, window, s)
+                        : dispatch_q<1, false>(p, route, alpha_out, alpha_in, window, s);
+    case 2: return full ? dispatch_q<2, true>(p, route, alpha_out, alpha_in, window, s)
+                        : dispatch_q<2, false>(p, route, alpha_out, alpha_in, window, s);
+    case 3: return full ? dispatch_q<3, true>(p, route, alpha_out, alpha_in, window, s)
+                        : dispatch_q<3, false>(p, route, alpha_out, alpha_in, window, s);
+    case 4: return full ? dispatch_q<4, true>(p, route, alpha_out, alpha_in, window, s)
+                        : dispatch_q<4, false>(p, route, alpha_out, alpha_in, window, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 template <int Q>
 cudaError_t launch_sample_q(const float* z, const float* alpha, const float* bias, int64_t N,
-                            int E, int K, int64_t S, int64_t stride, uint32_t* sample,
-                            cudaStream_t s) {
-  const size_t smem = sizeof(uint32_t) * kSampleRows * (E + 1);
+                            int E, int K, int64_t S, int64_t stride, int64_t S_ld,
+                            uint32_t* sample, cudaStream_t s) {
+  const size_t smem = ((4 * kSampleRows * (E + 1) + 15) & ~15) + ((4 * E + 15) & ~15) +
+                      sizeof(RowScratch<Q>) * kWarps;
   dim3 grid(static_cast<unsigned>((S + kSampleRows - 1) / kSampleRows)), block(kThreads);
-  auto k = alpha ? sample_keys_kernel<Q, true> : sample_keys_kernel<Q, false>;
+  auto k = alpha ? sample_keys_kernel<Q, true, false>
+                 : (bias ? sample_keys_kernel<Q, false, true> : sample_keys_kernel<Q, false, false>);
   cudaError_t err =
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  k<<<grid, block, smem, s>>>(z, alpha, bias, N, E, K, S, stride, sample);
+  k<<<grid, block, smem, s>>>(z, alpha, bias, N, E, K, S, stride, S_ld, sample);
   return cudaGetLastError();
 }
 
@@ -479,13 +402,13 @@ cudaError_t launch_topk(const float* z, const float* bias, int64_t N, int32_t E,
 }
 
 cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* bias, int64_t N,
-                              int32_t E, int32_t K, int64_t S, int64_t stride, uint32_t* sample,
-                              cudaStream_t s) {
+                              int32_t E, int32_t K, int64_t S, int64_t stride, int64_t S_ld,
+                              uint32_t* sample, cudaStream_t s) {
   switch ((E + 127) / 128) {
-    case 1: return launch_sample_q<1>(z, alpha, bias, N, E, K, S, stride, sample, s);
-    case 2: return launch_sample_q<2>(z, alpha, bias, N, E, K, S, stride, sample, s);
-    case 3: return launch_sample_q<3>(z, alpha, bias, N, E, K, S, stride, sample, s);
-    case 4: return launch_sample_q<4>(z, alpha, bias, N, E, K, S, stride, sample, s);
+    case 1: return launch_sample_q<1>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s);
+    case 2: return launch_sample_q<2>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s);
+    case 3: return launch_sample_q<3>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s);
+    case 4: return launch_sample_q<4>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s);
     default: return cudaErrorInvalidValue;
   }
 }
