@@ -5,16 +5,17 @@
 // index j = t*K + k by expert: offsets = exclusive prefix sum of counts,
 // perm[p] = j in (expert, j) order, inv[j] = p.
 //
-// Large inputs, three launches:
-//   A  each warp counts its chunk of slots into a shared histogram and
-//      writes it to chunk_counts[chunk][E] (coalesced);
-//   B  one block per expert turns its column of chunk counts into an
+// Large inputs, three launches over tiles of 8192 slots:
+//   A  each block counts its tile into a shared histogram and writes it to
+//      tile_counts[tile][E] (coalesced);
+//   B  one block per expert turns its column of tile counts into an
 //      exclusive prefix; the last block to finish (ticket) scans the totals
 //      into offsets/counts;
-//   C  each warp replays its chunk 32 slots at a time; __match_any_sync
-//      groups lanes by expert, the rank inside the group is the popcount of
-//      lower lanes, and a per-warp running cursor keeps the order stable.
-// Small inputs (decode) run the same three steps inside one block.
+//   C  each block re-sorts its tile in shared memory with a stable counting
+//      sort (__match_any_sync groups a warp's lanes by expert, per-warp
+//      running counters keep slot order), writes inv in slot order and perm
+//      as one contiguous run per expert.
+// Small inputs (decode) run the same steps inside one block.
 #include "launch.h"
 #include "common.cuh"
 
@@ -24,44 +25,32 @@ namespace {
 
 constexpr int kPermThreads = 256;
 constexpr int kPermWarps = kPermThreads / kWarp;
-constexpr int64_t kChunk = 1024;        // slots per warp chunk
+constexpr int kSlotsPerThread = 32;
+constexpr int64_t kTile = static_cast<int64_t>(kPermThreads) * kSlotsPerThread;  // 8192 slots
 constexpr int64_t kSingleMax = 4096;    // N*K handled by one block
-constexpr int kUnroll = 8;
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-__global__ void __launch_bounds__(kPermThreads) chunk_count_kernel(
-    const int32_t* __restrict__ ids, int64_t NK, int E, int64_t nchunks,
-    uint32_t* __restrict__ chunk_counts) {
-  extern __shared__ uint32_t hist_all[];  // [kPermWarps][E]
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t* hist = hist_all + warp * E;
-  for (int e = lane; e < E; e += 32) hist[e] = 0u;
-  __syncwarp();
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * kPermWarps + warp;
-  if (c >= nchunks) return;
-  const int64_t j0 = c * kChunk;
-  const int64_t j1 = (j0 + kChunk < NK) ? j0 + kChunk : NK;
+__global__ void __launch_bounds__(kPermThreads) tile_count_kernel(
+    const int32_t* __restrict__ ids, int64_t NK, int E, uint32_t* __restrict__ tile_counts) {
+  __shared__ uint32_t hist[KOLIBRI_MAX_EXPERTS];
+  for (int e = threadIdx.x; e < E; e += kPermThreads) hist[e] = 0u;
+  __syncthreads();
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
   bool bad = false;
-  for (int64_t base = j0; base < j1; base += 32 * kUnroll) {
-    int32_t v[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      int64_t j = base + u * 32 + lane;
-      v[u] = j < j1 ? __ldg(ids + j) : -1;
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      int64_t j = base + u * 32 + lane;
-      if (j < j1) {
-        if (v[u] >= 0 && v[u] < E) atomicAdd(&hist[v[u]], 1u);
-        else bad = true;
-      }
+#pragma unroll 8
+  for (int u = 0; u < kSlotsPerThread; ++u) {
+    const int64_t j = t0 + u * kPermThreads + threadIdx.x;
+    if (j < NK) {
+      const int32_t x = __ldg(ids + j);
+      if (x >= 0 && x < E) atomicAdd(&hist[x], 1u);
+      else bad = true;
     }
   }
   if (bad) raise_status(kStatusBadInput);
-  __syncwarp();
-  for (int e = lane; e < E; e += 32) chunk_counts[c * E + e] = hist[e];
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kPermThreads)
+    tile_counts[static_cast<int64_t>(blockIdx.x) * E + e] = hist[e];
 }
 
 // One block per expert: exclusive prefix over chunks, then the last block
@@ -155,30 +144,113 @@ __device__ __forceinline__ void scatter_round(int32_t e, int64_t j, int lane, ui
   __syncwarp();
 }
 
-__global__ void __launch_bounds__(kPermThreads) chunk_scatter_kernel(
-    const int32_t* __restrict__ ids, int64_t NK, int E, int64_t nchunks,
-    const uint32_t* __restrict__ chunk_prefix, const int64_t* __restrict__ offsets,
-    int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
-  extern __shared__ uint32_t cur_all[];  // [kPermWarps][E]
+// Exclusive prefix of n <= 2 * kPermThreads values held two per thread
+// (thread t owns v0 = element 2t, v1 = element 2t+1); returns the prefix of
+// element 2t and writes the grand total to *total.
+__device__ __forceinline__ uint32_t block_scan_pairs(uint32_t v0, uint32_t v1, uint32_t* warp_sums,
+                                                     uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t* cursor = cur_all + warp * E;
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * kPermWarps + warp;
-  if (c >= nchunks) return;
-  for (int e = lane; e < E; e += 32)
-    cursor[e] = static_cast<uint32_t>(offsets[e]) + chunk_prefix[c * E + e];
+  const uint32_t pair = v0 + v1;
+  uint32_t incl = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  uint32_t wbase = 0, all = 0;
+  for (int w = 0; w < kPermWarps; ++w) {
+    const uint32_t x = warp_sums[w];
+    if (w < warp) wbase += x;
+    all += x;
+  }
+  *total = all;
+  return wbase + incl - pair;
+}
+
+// Stable counting sort of one tile in shared memory, then coalesced output.
+__global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
+    const int32_t* __restrict__ ids, int64_t NK, int E, const uint32_t* __restrict__ tile_prefix,
+    const int64_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  extern __shared__ __align__(16) uint32_t sm[];
+  uint32_t* cnt_w = sm;                                   // [kPermWarps][E]
+  uint32_t* lo_e = cnt_w + kPermWarps * E;                // [E] tile-local start of expert e
+  uint32_t* base_e = lo_e + E;                            // [E] global start of e's run
+  uint32_t* sorted = base_e + E;                          // [kTile] slot index by local position
+  uint32_t* sorted_e = sorted + kTile;                    // [kTile] its expert
+  __shared__ uint32_t warp_sums[kPermWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
+  uint32_t* my_cnt = cnt_w + warp * E;
+  for (int e = lane; e < E; e += 32) my_cnt[e] = 0u;
   __syncwarp();
-  const int64_t j0 = c * kChunk;
-  const int64_t j1 = (j0 + kChunk < NK) ? j0 + kChunk : NK;
-  for (int64_t base = j0; base < j1; base += 32 * kUnroll) {
-    int32_t v[kUnroll];
+  // ---- phase 1: per-warp stable ranks, 32 consecutive slots per round
+  int32_t ex[kSlotsPerThread];
+  uint32_t rk[kSlotsPerThread];
+  const int64_t w0 = t0 + static_cast<int64_t>(warp) * (kSlotsPerThread * 32);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      int64_t j = base + u * 32 + lane;
-      int32_t x = j < j1 ? __ldg(ids + j) : -1;
-      v[u] = (x >= 0 && x < E) ? x : -1;
+  for (int r = 0; r < kSlotsPerThread; ++r) {
+    const int64_t j = w0 + r * 32 + lane;
+    const int32_t x = j < NK ? __ldg(ids + j) : -1;
+    ex[r] = (x >= 0 && x < E) ? x : -1;
+  }
+#pragma unroll
+  for (int r = 0; r < kSlotsPerThread; ++r) {
+    const int32_t e = ex[r];
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const uint32_t below = __popc(peers & lt);
+    rk[r] = (e >= 0) ? my_cnt[e] + below : 0u;
+    __syncwarp();
+    if (e >= 0 && below == 0u) my_cnt[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // ---- phase 2: warp prefixes per expert, tile-local and global starts
+  const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
+  uint32_t tot0 = 0u, tot1 = 0u;
+  for (int w = 0; w < kPermWarps; ++w) {
+    if (e0 < E) {
+      const uint32_t c = cnt_w[w * E + e0];
+      cnt_w[w * E + e0] = tot0;
+      tot0 += c;
     }
+    if (e1 < E) {
+      const uint32_t c = cnt_w[w * E + e1];
+      cnt_w[w * E + e1] = tot1;
+      tot1 += c;
+    }
+  }
+  uint32_t tile_total;
+  const uint32_t start0 = block_scan_pairs(tot0, tot1, warp_sums, &tile_total);
+  if (e0 < E) {
+    lo_e[e0] = start0;
+    base_e[e0] = static_cast<uint32_t>(offsets[e0]) + tile_prefix[static_cast<int64_t>(blockIdx.x) * E + e0];
+  }
+  if (e1 < E) {
+    lo_e[e1] = start0 + tot0;
+    base_e[e1] = static_cast<uint32_t>(offsets[e1]) + tile_prefix[static_cast<int64_t>(blockIdx.x) * E + e1];
+  }
+  __syncthreads();
+  // ---- phase 3: local positions; inv in slot order
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) scatter_round(v[u], base + u * 32 + lane, lane, cursor, perm, inv);
+  for (int r = 0; r < kSlotsPerThread; ++r) {
+    const int32_t e = ex[r];
+    if (e >= 0) {
+      const uint32_t within = my_cnt[e] + rk[r];           // position inside e's tile run
+      const uint32_t lpos = lo_e[e] + within;
+      const int64_t j = w0 + r * 32 + lane;
+      sorted[lpos] = static_cast<uint32_t>(j);
+      sorted_e[lpos] = static_cast<uint32_t>(e);
+      if (inv) inv[j] = static_cast<int32_t>(base_e[e] + within);
+    }
+  }
+  __syncthreads();
+  // ---- phase 4: perm as one contiguous run per expert
+  for (uint32_t pidx = threadIdx.x; pidx < tile_total; pidx += kPermThreads) {
+    const uint32_t e = sorted_e[pidx];
+    perm[base_e[e] + (pidx - lo_e[e])] = static_cast<int32_t>(sorted[pidx]);
   }
 }
 
@@ -222,11 +294,16 @@ __global__ void __launch_bounds__(1024) permute_single_kernel(
 
 }  // namespace
 
+size_t tile_scatter_smem(int E) {
+  return sizeof(uint32_t) * (static_cast<size_t>(kPermWarps) * E + 2 * static_cast<size_t>(E) +
+                             2 * static_cast<size_t>(kTile));
+}
+
 PermuteLayout permute_layout(int64_t N, int32_t E, int32_t K) {
   PermuteLayout L;
   const int64_t NK = N * K;
-  L.chunk = kChunk;
-  L.nchunks = (NK + kChunk - 1) / kChunk;
+  L.chunk = kTile;
+  L.nchunks = (NK + kTile - 1) / kTile;
   L.single_cta = NK <= kSingleMax;
   size_t off = 0;
   L.off_chunk_counts = off;
@@ -249,20 +326,22 @@ cudaError_t launch_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K, 
     return cudaGetLastError();
   }
   char* base = static_cast<char*>(ws);
-  uint32_t* chunk_counts = reinterpret_cast<uint32_t*>(base + L.off_chunk_counts);
+  uint32_t* tile_counts = reinterpret_cast<uint32_t*>(base + L.off_chunk_counts);
   uint32_t* totals = reinterpret_cast<uint32_t*>(base + L.off_counts);
   uint32_t* ticket = reinterpret_cast<uint32_t*>(base + L.off_ticket);
   cudaError_t err = cudaMemsetAsync(ticket, 0, sizeof(uint32_t), s);
   if (err != cudaSuccess) return err;
-  const unsigned blocks = static_cast<unsigned>((L.nchunks + kPermWarps - 1) / kPermWarps);
-  const size_t smem = sizeof(uint32_t) * kPermWarps * static_cast<size_t>(E);
-  chunk_count_kernel<<<blocks, kPermThreads, smem, s>>>(ids, NK, E, L.nchunks, chunk_counts);
+  const unsigned tiles = static_cast<unsigned>(L.nchunks);
+  tile_count_kernel<<<tiles, kPermThreads, 0, s>>>(ids, NK, E, tile_counts);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  chunk_scan_kernel<<<E, kPermThreads, 0, s>>>(chunk_counts, L.nchunks, E, totals, ticket, counts,
+  chunk_scan_kernel<<<E, kPermThreads, 0, s>>>(tile_counts, L.nchunks, E, totals, ticket, counts,
                                                offsets);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  chunk_scatter_kernel<<<blocks, kPermThreads, smem, s>>>(ids, NK, E, L.nchunks, chunk_counts,
-                                                          offsets, perm, inv);
+  const size_t smem = tile_scatter_smem(E);
+  err = cudaFuncSetAttribute(tile_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  tile_scatter_kernel<<<tiles, kPermThreads, smem, s>>>(ids, NK, E, tile_counts, offsets, perm, inv);
   return cudaGetLastError();
 }
 

@@ -34,7 +34,9 @@ constexpr int kMaxStages = 8;
 constexpr int kEpiWarps = 4;
 constexpr int kStoreCols = 32;           // fp32 columns per TMA store box
 constexpr int kStageBuf = kStoreCols * 32 * 4;  // 4 KB: 32 rows x 128 B
+constexpr int kEpiBufs = 4;              // staging buffers per epilogue warp
 constexpr int kSmemLimit = 227 * 1024;
+constexpr int kPrefetch = 8;             // x k-blocks warmed in L2 ahead of their load
 
 struct GemmShape {
   int64_t N;
@@ -93,6 +95,14 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// Warm L2 with a tile that a later k-block will load (no shared memory).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int c0, int c1, uint32_t src) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
@@ -100,8 +110,9 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int c0, int
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read_1() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+// at most kEpiBufs - 1 stores may still be reading their staging buffer
+__device__ __forceinline__ void bulk_wait_read_ring() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kEpiBufs - 1) : "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -195,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t b_bytes = static_cast<uint32_t>(sh.nchunks * half_n) * kBK * 2;
   const uint32_t stage_bytes = a_bytes + b_bytes;
   const uint32_t staging = base + stage_bytes * sh.stages;  // epilogue buffers (1 KB aligned)
-  const uint32_t bars = staging + kEpiWarps * 2 * kStageBuf;
+  const uint32_t bars = staging + kEpiWarps * kEpiBufs * kStageBuf;
   auto full_bar = [bars](int s) { return bars + 8u * s; };
   auto empty_bar = [bars](int s) { return bars + 8u * (kMaxStages + s); };
   const uint32_t tmem_full = bars + 8u * (2 * kMaxStages);
@@ -239,6 +250,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      if (static_cast<int64_t>(cid) < sh.num_pairs) {
+        const int row_first = static_cast<int>(static_cast<int64_t>(cid) * 2 * kBM + rank * kBM);
+        for (int kb = 0; kb < kPrefetch && kb < k_blocks; ++kb)
+          tma_prefetch_2d(&tm_x, kb * kBK, row_first);
+      }
       for (int64_t pt = cid; pt < sh.num_pairs && ok; pt += ncl) {
         const int row0 = static_cast<int>(pt * 2 * kBM + rank * kBM);
         for (int kb = 0; kb < k_blocks; ++kb) {
@@ -250,6 +266,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * stage_bytes);
           const uint32_t a_dst = base + stage_bytes * stage;
           const uint32_t b_dst = a_dst + a_bytes;
+          // x comes from HBM: ask for the tile kPrefetch k-blocks ahead now,
+          // continuing into the pair's next tile near the end of this one
+          {
+            const int pk = kb + kPrefetch;
+            if (pk < k_blocks) {
+              tma_prefetch_2d(&tm_x, pk * kBK, row0);
+            } else if (pt + ncl < sh.num_pairs) {
+              tma_prefetch_2d(&tm_x, (pk - k_blocks) * kBK,
+                              static_cast<int>((pt + ncl) * 2 * kBM + rank * kBM));
+            }
+          }
           tma_load_2d_pair(a_dst, &tm_x, kb * kBK, row0, fb, pol_x);
           for (int c = 0; c < sh.nchunks; ++c)
             tma_load_2d_pair(b_dst + static_cast<uint32_t>(c * half_n) * (kBK * 2), &tm_w, kb * kBK,
@@ -279,11 +306,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = base + stage_bytes * stage;
           const uint32_t b_addr = a_addr + a_bytes;
           const uint64_t a_desc = sw128_desc(a_addr);
+          // one expert chunk at a time: back-to-back MMAs into the same
+          // accumulator run faster than alternating accumulators
+          for (int c = 0; c < sh.nchunks; ++c) {
+            const uint64_t b_desc =
+                sw128_desc(b_addr + static_cast<uint32_t>(c * half_n) * (kBK * 2));
 #pragma unroll
-          for (int ks = 0; ks < kBK / 16; ++ks) {
-            for (int c = 0; c < sh.nchunks; ++c) {
-              const uint64_t b_desc =
-                  sw128_desc(b_addr + static_cast<uint32_t>(c * half_n) * (kBK * 2));
+            for (int ks = 0; ks < kBK / 16; ++ks) {
               // 16 bf16 along K = 32 bytes inside the swizzle atom
               tc_mma_pair(tmem_base + static_cast<uint32_t>(c * sh.chunk_n), a_desc + 2u * ks,
                           b_desc + 2u * ks, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
@@ -304,7 +333,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // epilogue warps 2..5; TMEM lane quarter is fixed by warp % 4
     const int quarter = warp & 3;
     const int ew = warp - 2;
-    const uint32_t buf0 = staging + static_cast<uint32_t>(ew * 2 * kStageBuf);
+    const uint32_t buf0 = staging + static_cast<uint32_t>(ew * kEpiBufs * kStageBuf);
     const uint32_t empty_leader = map_to_rank(tmem_empty, 0);
     uint32_t acc_phase = 0;
     int nbuf = 0;
@@ -319,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         // staging buffer: 32 rows x 128 bytes, 16-byte chunks swizzled by row
         const uint32_t buf = buf0 + static_cast<uint32_t>(nbuf * kStageBuf);
-        if (lane == 0) bulk_wait_read_1();  // the store that last used this buffer has read it
+        if (lane == 0) bulk_wait_read_ring();  // the store that last used this buffer has read it
         __syncwarp();
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -334,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_store_2d(&tm_z, c0, row_base, buf);
           bulk_commit();
         }
-        nbuf ^= 1;
+        nbuf = (nbuf + 1 == kEpiBufs) ? 0 : nbuf + 1;
       }
       tc_fence_before();
       __syncwarp();
@@ -406,7 +435,7 @@ cudaError_t launch_router_logits(const void* x, const void* w, float* z, int64_t
   sh.tmem_cols = tc;
   const size_t stage_bytes =
       static_cast<size_t>(kBM) * kBK * 2 + static_cast<size_t>(cols / 2) * kBK * 2;
-  const size_t fixed = 1024 /*alignment slack*/ + kEpiWarps * 2 * kStageBuf + 8 * (2 * kMaxStages + 3);
+  const size_t fixed = 1024 /*alignment slack*/ + kEpiWarps * kEpiBufs * kStageBuf + 8 * (2 * kMaxStages + 3);
   int stages = static_cast<int>((kSmemLimit - fixed) / stage_bytes);
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return cudaErrorInvalidValue;
