@@ -34,6 +34,7 @@ SIGNATURES = {
     "kolibri_router_logits": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P]),
     "kolibri_router_topk": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P]),
     "kolibri_expert_permute": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
+    "kolibri_expert_permute_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P]),
     "kolibri_eqb_update": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _SZ, _P]),
     "kolibri_route_and_balance": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P, _P,
                                                  _SZ, _P]),
@@ -166,6 +167,29 @@ def kolibri_expert_permute(ids: torch.Tensor, E: int, ws: torch.Tensor | None = 
            load().kolibri_expert_permute(_ptr(ids), N, E, K, _ptr(counts), _ptr(offsets),
                                          _ptr(perm), _ptr(inv), _ptr(ws), ws.numel(),
                                          _stream(stream)))
+    return counts, offsets, perm, inv
+
+
+def kolibri_expert_permute_noalloc(ids: torch.Tensor, E: int, counts=None, offsets=None,
+                                   perm=None, inv=None, want_inv: bool = True, stream=None):
+    """kolibri_expert_permute without a workspace (library-held scratch).
+
+    For callers that cannot allocate device memory; see the header for the
+    size limit and the rule that calls must not overlap on the GPU."""
+    N, K = ids.shape
+    _need(ids, torch.int32, (N, K), "ids")
+    dev = ids.device
+    if counts is None:
+        counts = torch.empty((E,), dtype=torch.int32, device=dev)
+    if offsets is None:
+        offsets = torch.empty((E + 1,), dtype=torch.int64, device=dev)
+    if perm is None:
+        perm = torch.empty((N * K,), dtype=torch.int32, device=dev)
+    if inv is None and want_inv:
+        inv = torch.empty((N * K,), dtype=torch.int32, device=dev)
+    _check("kolibri_expert_permute_noalloc",
+           load().kolibri_expert_permute_noalloc(_ptr(ids), N, E, K, _ptr(counts), _ptr(offsets),
+                                                 _ptr(perm), _ptr(inv), _stream(stream)))
     return counts, offsets, perm, inv
 
 

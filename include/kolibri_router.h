@@ -129,6 +129,33 @@ KOLIBRI_API kolibri_status kolibri_expert_permute(const int32_t *ids, int64_t N,
                                       int32_t *inv, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * kolibri_expert_permute for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a deployment convenience.  Some
+ * callers may not call cudaMalloc at all: inference servers that reserve all
+ * of device memory for their own pool up front, plugins that run inside
+ * another runtime's memory budget, and code paths that must not risk the
+ * implicit synchronisation an allocation can cause.  This variant takes no
+ * workspace: its scratch is a fixed array of KOLIBRI_NOALLOC_SCRATCH_BYTES
+ * inside the library, which every GPU that loads the library holds until
+ * the process exits.
+ *   Arguments and results are those of kolibri_expert_permute, without ws.
+ *   Sizes whose scratch (kolibri_workspace_bytes(KOLIBRI_OP_PERMUTE, N, E,
+ *   K)) exceeds the array return KOLIBRI_ERR_WORKSPACE_TOO_SMALL and
+ *   enqueue nothing (at E = 384, up to 11,182,080 routed slots N*K fit).
+ *   The first call on each device looks up the array's device address with
+ *   that device current; make that first call before any stream capture.
+ *   Every call shares the one array: calls that can overlap on the GPU (on
+ *   different streams, or from different threads) race and must not be
+ *   issued.  The array keeps the previous call's contents; what must start
+ *   at zero is cleared on the stream by each call.
+ */
+#define KOLIBRI_NOALLOC_SCRATCH_BYTES (2u << 20)
+KOLIBRI_API kolibri_status kolibri_expert_permute_noalloc(const int32_t *ids, int64_t N,
+                                                          int32_t E, int32_t K, int32_t *counts,
+                                                          int64_t *offsets, int32_t *perm,
+                                                          int32_t *inv, void *stream);
+
+/*
  * Exact Quantile Balancing update ("Kolibri Pre-Training from Scratch" 7.1
  * update rule, 7.2 order of operations, 7.3 exactness):
  *   v_e  = Q_m(Z_:,e + alpha), the (m+1)-th largest entry of the fp32 sums,
