@@ -36,7 +36,6 @@ constexpr int kStoreCols = 32;           // fp32 columns per TMA store box
 constexpr int kStageBuf = kStoreCols * 32 * 4;  // 4 KB: 32 rows x 128 B
 constexpr int kEpiBufs = 4;              // staging buffers per epilogue warp
 constexpr int kSmemLimit = 227 * 1024;
-constexpr int kPrefetch = 8;             // x k-blocks warmed in L2 ahead of their load
 
 struct GemmShape {
   int64_t N;
@@ -93,14 +92,6 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster), "l"(policy)
       : "memory");
-}
-
-// Warm L2 with a tile that a later k-block will load (no shared memory).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int c0, int c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1)
-               : "memory");
 }
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int c0, int c1, uint32_t src) {
@@ -250,11 +241,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      if (static_cast<int64_t>(cid) < sh.num_pairs) {
-        const int row_first = static_cast<int>(static_cast<int64_t>(cid) * 2 * kBM + rank * kBM);
-        for (int kb = 0; kb < kPrefetch && kb < k_blocks; ++kb)
-          tma_prefetch_2d(&tm_x, kb * kBK, row_first);
-      }
       for (int64_t pt = cid; pt < sh.num_pairs && ok; pt += ncl) {
         const int row0 = static_cast<int>(pt * 2 * kBM + rank * kBM);
         for (int kb = 0; kb < k_blocks; ++kb) {
@@ -266,17 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (leader) mbar_arrive_expect_tx(full_bar(stage), 2u * stage_bytes);
           const uint32_t a_dst = base + stage_bytes * stage;
           const uint32_t b_dst = a_dst + a_bytes;
-          // x comes from HBM: ask for the tile kPrefetch k-blocks ahead now,
-          // continuing into the pair's next tile near the end of this one
-          {
-            const int pk = kb + kPrefetch;
-            if (pk < k_blocks) {
-              tma_prefetch_2d(&tm_x, pk * kBK, row0);
-            } else if (pt + ncl < sh.num_pairs) {
-              tma_prefetch_2d(&tm_x, (pk - k_blocks) * kBK,
-                              static_cast<int>((pt + ncl) * 2 * kBM + rank * kBM));
-            }
-          }
           tma_load_2d_pair(a_dst, &tm_x, kb * kBK, row0, fb, pol_x);
           for (int c = 0; c < sh.nchunks; ++c)
             tma_load_2d_pair(b_dst + static_cast<uint32_t>(c * half_n) * (kBK * 2), &tm_w, kb * kBK,
