@@ -80,6 +80,17 @@ def launches_per_step(N, E, K):
     return 1 + route_eqb + permute
 
 
+def reduce_max_over_ranks(value: float, device) -> float:
+    """The slowest rank's value (device time per step); identity on one rank."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return value
+    if torch.distributed.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -238,10 +249,7 @@ def run_ours(args, rank, world, local_rank):
     if st != B.KOLIBRI_OK:
         raise RuntimeError(f"device status after timing: {B.status_string(st)}")
 
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max_over_ranks(total_ms, device)
     ms_per_step = total_ms / args.steps
 
     # ---- end to end through the public API with host buffers
@@ -361,10 +369,7 @@ def run_e2e(args, step, stream, device, world):
     b.record(stream)
     b.synchronize()
     ms = a.elapsed_time(b) / n
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max_over_ranks(ms, device)
     return {"value": world * N / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms, "steps": n,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
