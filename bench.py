@@ -72,12 +72,13 @@ def gemm_bytes(N, d, E):
 
 
 def launches_per_step(N, E, K):
-    """Kernels of ours per step: logits 1; routing + EQB 4 (N <= 16384: route,
-    sample, select, bias) or 6 (sample, bracket, fused pass, select,
-    fallback check, bias); permutation 1 or 3."""
-    route_eqb = 4 if N <= 16384 else 7
+    """Kernels of ours per step: logits + selection 2 (the fused GEMM and the
+    check for rows it left to the row kernel); EQB update 3 (N <= 16384:
+    sample, exact select, bias) or 6 (sample, bracket, bracketed pass,
+    select, fallback check, bias); permutation 1 or 3."""
+    eqb = 3 if N <= 16384 else 6
     permute = 1 if N * K <= 4096 else 3
-    return 1 + route_eqb + permute
+    return 2 + eqb + permute
 
 
 def reduce_max_over_ranks(value: float, device) -> float:
@@ -186,15 +187,17 @@ class RouterStep:
         self.ws_eqb = B.workspace(B.KOLIBRI_OP_EQB, N, E, K, device)
 
     def run(self, stream, events=None):
-        """logits -> routing + EQB update (one call, one read of Z) -> permutation."""
+        """logits + routing (selection in the GEMM epilogue) -> EQB update of
+        beta from that alpha (one bracketed read of Z) -> permutation."""
         wl = self.wl
         if events:
             events[0].record(stream)
-        B.kolibri_router_logits(self.x, self.w, self.z, stream=stream)
+        B.kolibri_router_forward(self.x, self.w, self.beta, wl.K, z=self.z, ids=self.ids,
+                                 gates=self.gates, alpha=self.alpha, stream=stream)
         if events:
             events[1].record(stream)
-        B.kolibri_route_and_balance(self.z, self.beta, wl.K, self.ws_eqb, self.ids, self.gates,
-                                    self.alpha, self.q, stream=stream)
+        B.kolibri_eqb_update(self.z, self.alpha, self.beta, wl.K, self.ws_eqb, self.q,
+                             stream=stream)
         if events:
             events[2].record(stream)
         B.kolibri_expert_permute(self.ids, wl.E, self.ws_perm, self.counts, self.offsets,
@@ -262,7 +265,7 @@ def run_ours(args, rank, world, local_rank):
     peaks = _peaks()
     flops, bytes_ = algorithmic_work(N, d, E, K)
     roof_ms = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
-    gemm_ms = float(stage_ms[0])
+    gemm_ms = float(stage_ms[0])   # the fused GEMM + selection, and the row check after it
     gemm_tflops = 2.0 * N * d * E / (gemm_ms * 1e-3) / 1e12
     peak_t = peaks["bf16_tflops"]  # burst: the timed region is tens of ms at max clocks
     traffic = _traffic_from_profile(N)
@@ -282,14 +285,14 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": wl.name, "N": N, "d": d, "E": E, "K": K, "offsets": wl.offsets,
                    "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (x %.2f GB, Z %.2f GB)" % (2 * N * d / 1e9, 4 * N * E / 1e9)},
-        "roofline": {"bound": "tensor", "kernel": "router_gemm_pair_kernel",
+        "roofline": {"bound": "tensor", "kernel": "router_forward_kernel",
                      "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": gemm_tflops / peak_t, "traffic": traffic,
                      "peak_kind": f"bf16 burst (cuBLAS 8192^3), of {peaks['source']}", "sustained_frac": gemm_tflops / peaks["bf16_tflops_sustained"]},
         "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ms_per_step,
                           "flops": flops, "bytes": bytes_,
                           "peaks": f"bf16 burst {peaks['bf16_tflops']} TF/s, HBM {peaks['hbm_gbs']} GB/s, of {peaks['source']}"},
-        "stages_ms": {"logits": gemm_ms, "route_and_eqb": float(stage_ms[1]),
+        "stages_ms": {"logits_and_routing": gemm_ms, "eqb_update": float(stage_ms[1]),
                       "permute": float(stage_ms[2])},
         "gpu_launches": launches_per_step(N, E, K) * args.steps,
         "clocks": clocks,
@@ -300,18 +303,28 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
-GEMM_PROFILE = os.path.join(ROOT, "profiles", "router_gemm_pair_kolibri.md")
-GEMM_SOURCE = os.path.join(ROOT, "expert_load_balancing_b200", "csrc", "router_logits.cu")
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "router_forward_kolibri.md")
+GEMM_SOURCES = [os.path.join(ROOT, "expert_load_balancing_b200", "csrc", f)
+                for f in ("router_forward.cu", "gemm_pair.cuh")]
+
+
+def kernel_source_digest():
+    """sha256 over the fused kernel's source files, in a fixed order."""
+    import hashlib
+    h = hashlib.sha256()
+    for p in GEMM_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def _traffic_from_profile(N):
     """DRAM bytes per GEMM launch (read + write) from the committed ncu
     summary, scaled to N tokens; None if the kernel source changed since the
     counters were taken."""
-    import hashlib
     try:
         text = open(GEMM_PROFILE).read()
-        digest = hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest()
+        digest = kernel_source_digest()
     except OSError:
         return None
     fields = {}

@@ -11,7 +11,9 @@ from .binding import (  # noqa: F401
     kolibri_device_status,
     kolibri_eqb_update,
     kolibri_expert_permute,
+    kolibri_expert_permute_noalloc,
     kolibri_route_and_balance,
+    kolibri_router_forward,
     kolibri_router_logits,
     kolibri_router_topk,
     kolibri_workspace_bytes,

@@ -32,6 +32,7 @@ SIGNATURES = {
     "kolibri_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kolibri_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I32, _I32]),
     "kolibri_router_logits": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P]),
+    "kolibri_router_forward": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _P, _P, _P]),
     "kolibri_router_topk": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P]),
     "kolibri_expert_permute": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "kolibri_expert_permute_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P]),
@@ -116,6 +117,34 @@ def kolibri_router_logits(x: torch.Tensor, w: torch.Tensor, z: torch.Tensor | No
     _check("kolibri_router_logits",
            load().kolibri_router_logits(_ptr(x), _ptr(w), _ptr(z), N, d, E, _stream(stream)))
     return z
+
+
+def kolibri_router_forward(x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None, K: int,
+                           z: torch.Tensor | None = None, ids: torch.Tensor | None = None,
+                           gates: torch.Tensor | None = None, alpha: torch.Tensor | None = None,
+                           stream=None):
+    """Logits and selection in one call (the GEMM epilogue selects).
+
+    Returns (z [N,E] fp32, ids [N,K] int32, gates [N,K] fp32, alpha [N] fp32)."""
+    N, d = x.shape
+    E = w.shape[0]
+    _need(x, torch.bfloat16, (N, d), "x")
+    _need(w, torch.bfloat16, (E, d), "w")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    dev = x.device
+    z = torch.empty((N, E), dtype=torch.float32, device=dev) if z is None else z
+    ids = torch.empty((N, K), dtype=torch.int32, device=dev) if ids is None else ids
+    gates = torch.empty((N, K), dtype=torch.float32, device=dev) if gates is None else gates
+    alpha = torch.empty((N,), dtype=torch.float32, device=dev) if alpha is None else alpha
+    _need(z, torch.float32, (N, E), "z")
+    _need(ids, torch.int32, (N, K), "ids")
+    _need(gates, torch.float32, (N, K), "gates")
+    _need(alpha, torch.float32, (N,), "alpha")
+    _check("kolibri_router_forward",
+           load().kolibri_router_forward(_ptr(x), _ptr(w), _ptr(bias), _ptr(z), N, d, E, K,
+                                         _ptr(ids), _ptr(gates), _ptr(alpha), _stream(stream)))
+    return z, ids, gates, alpha
 
 
 def kolibri_router_topk(z: torch.Tensor, bias: torch.Tensor | None, K: int,

@@ -7,7 +7,7 @@
 
 namespace kolibri {
 
-__device__ unsigned int g_status = 0u;
+KOLIBRI_DEFINE_STATUS_TAKE(status_take_api)
 
 int device_sm_count() {
   int dev = 0, n = 0;
@@ -70,6 +70,29 @@ kolibri_status kolibri_router_logits(const void* x, const void* w, float* z, int
   return from_cuda(launch_router_logits(x, w, z, N, d, E, static_cast<cudaStream_t>(stream)));
 }
 
+kolibri_status kolibri_router_forward(const void* x, const void* w, const float* bias, float* z,
+                                      int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                      float* gates, float* alpha, void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!x || !w || !z || !ids || !gates || !alpha) return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(z) || (bias && !aligned16(bias)))
+    return KOLIBRI_ERR_INVALID_ARG;
+  if (d < 1) return KOLIBRI_ERR_INVALID_ARG;
+  if (d % 64 != 0 || E % 16 != 0) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (router_forward_supported(E, K)) {
+    const cudaError_t err = launch_router_forward(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+    if (err == cudaSuccess)
+      return from_cuda(launch_select_fixup(z, bias, N, E, K, ids, gates, alpha, s));
+    if (err != cudaErrorNotSupported) return KOLIBRI_ERR_CUDA;
+  }
+  // shapes outside the fused kernel: the two kernels one after the other
+  const cudaError_t err = launch_router_logits(x, w, z, N, d, E, s);
+  if (err != cudaSuccess) return KOLIBRI_ERR_CUDA;
+  return from_cuda(launch_topk(z, bias, N, E, K, ids, gates, alpha, s));
+}
+
 kolibri_status kolibri_router_topk(const float* z, const float* bias, int64_t N, int32_t E,
                                    int32_t K, int32_t* ids, float* gates, float* alpha,
                                    void* stream) {
@@ -124,10 +147,10 @@ kolibri_status kolibri_route_and_balance(const float* z, float* bias, int64_t N,
 kolibri_status kolibri_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KOLIBRI_ERR_CUDA;
-  unsigned int v = 0u, zero = 0u;
-  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return KOLIBRI_ERR_CUDA;
-  if (v != 0u && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
-    return KOLIBRI_ERR_CUDA;
+  const unsigned v = status_take_api() | status_take_eqb() | status_take_noalloc() |
+                     status_take_permute() | status_take_route() | status_take_logits() |
+                     status_take_forward();
+  if (v & kStatusReadFailed) return KOLIBRI_ERR_CUDA;
   if (v & kStatusTimeout) return KOLIBRI_ERR_TIMEOUT;
   if (v & kStatusBadInput) return KOLIBRI_ERR_DEVICE;
   return KOLIBRI_OK;

@@ -15,11 +15,25 @@ namespace kolibri {
 
 constexpr int kWarp = 32;
 
-// Device status word (one per device, module scope).  Bit 0: a bounded wait
-// expired; bit 1: a device-side argument check failed.
+// Device status word.  Bit 0: a bounded wait expired; bit 1: a device-side
+// argument check failed.  The library is built without relocatable device
+// code, so every translation unit holds its own word (one per device);
+// KOLIBRI_DEFINE_STATUS_TAKE gives each unit a host function that reads and
+// clears it, and kolibri_device_status ORs them.
 constexpr unsigned kStatusTimeout = 1u;
 constexpr unsigned kStatusBadInput = 2u;
-extern __device__ unsigned int g_status;
+constexpr unsigned kStatusReadFailed = 0x80000000u;
+static __device__ unsigned int g_status = 0u;
+
+#define KOLIBRI_DEFINE_STATUS_TAKE(fn)                                              \
+  unsigned fn() {                                                                   \
+    unsigned v = 0u, zero = 0u;                                                     \
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess)               \
+      return kStatusReadFailed;                                                     \
+    if (v != 0u && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) \
+      return kStatusReadFailed;                                                     \
+    return v;                                                                       \
+  }
 
 __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_status, bits); }
 

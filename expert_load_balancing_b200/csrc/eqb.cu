@@ -410,4 +410,6 @@ cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t
   return eqb_end(z, alpha_out, bias, N, E, K, quantiles, b, s);
 }
 
+KOLIBRI_DEFINE_STATUS_TAKE(status_take_eqb)
+
 }  // namespace kolibri

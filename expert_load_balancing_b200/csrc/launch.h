@@ -43,6 +43,16 @@ PermuteLayout permute_layout(int64_t N, int32_t E, int32_t K);
 cudaError_t launch_router_logits(const void* x, const void* w, float* z, int64_t N, int32_t d,
                                  int32_t E, cudaStream_t s);
 
+// Fused logits + selection (router_forward.cu).  Returns cudaErrorNotSupported
+// for shapes it does not cover; the caller then runs logits and top-K apart.
+// Rows it could not finish carry a NaN alpha; launch_select_fixup completes them.
+bool router_forward_supported(int32_t E, int32_t K);
+cudaError_t launch_router_forward(const void* x, const void* w, const float* bias, float* z,
+                                  int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                  float* gates, float* alpha, cudaStream_t s);
+cudaError_t launch_select_fixup(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
+                                int32_t* ids, float* gates, float* alpha, cudaStream_t s);
+
 cudaError_t launch_topk(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
                         int32_t* ids, float* gates, float* alpha, cudaStream_t s);
 
@@ -71,5 +81,14 @@ cudaError_t launch_route_window_pass(const float* z, const float* bias, const fl
                                      cudaStream_t s);
 
 int device_sm_count();
+
+// Read and clear the status word of one translation unit (see common.cuh).
+unsigned status_take_api();
+unsigned status_take_eqb();
+unsigned status_take_noalloc();
+unsigned status_take_permute();
+unsigned status_take_route();
+unsigned status_take_logits();
+unsigned status_take_forward();
 
 }  // namespace kolibri

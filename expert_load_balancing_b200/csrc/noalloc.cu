@@ -37,6 +37,8 @@ void* scratch_on_current_device() {
 }
 
 }  // namespace
+KOLIBRI_DEFINE_STATUS_TAKE(status_take_noalloc)
+
 }  // namespace kolibri
 
 using namespace kolibri;

@@ -345,4 +345,6 @@ cudaError_t launch_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K, 
   return cudaGetLastError();
 }
 
+KOLIBRI_DEFINE_STATUS_TAKE(status_take_permute)
+
 }  // namespace kolibri

@@ -309,6 +309,45 @@ __global__ void __launch_bounds__(kThreads) sample_keys_kernel(
   }
 }
 
+// Rows left unfinished by the fused logits + selection kernel carry a NaN
+// alpha (more candidates than its per-row buffer holds).  One warp checks 32
+// rows at a time and runs the exact row selection on each marked row.
+template <int Q, bool kFull, bool kBias>
+__global__ void __launch_bounds__(kThreads) select_fixup_kernel(
+    const float* __restrict__ z, const float* __restrict__ beta, int64_t N, int E, int K,
+    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha) {
+  __shared__ __align__(16) float beta_s[128 * Q];
+  __shared__ RowScratch<Q> scratch[kWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < 128 * Q; e += kThreads) beta_s[e] = (kBias && e < E) ? beta[e] : 0.f;
+  __syncthreads();
+  uint32_t valid = 0u;
+#pragma unroll
+  for (int j = 0; j < 4 * Q; ++j) valid |= (static_cast<int>(slot_expert(lane, j)) < E) ? (1u << j) : 0u;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kWarps * 32;
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * 32; base < N; base += step) {
+    const int64_t t = base + lane;
+    uint32_t m = __ballot_sync(0xffffffffu, t < N && isnan(alpha[t]));
+    while (m) {
+      const int i = __ffs(m) - 1;
+      m &= m - 1u;
+      const int64_t row = base + i;
+      float zr[4 * Q];
+      load_row<Q, kFull>(z + row * E, E, lane, zr);
+      int rank;
+      uint32_t key, id;
+      warp_select_row<Q, kFull, kBias>(zr, beta_s, valid, K, lane, scratch[warp], rank, key, id);
+      if (rank >= 0 && rank < K) {
+        const uint32_t e = id < static_cast<uint32_t>(E) ? id : 0u;
+        ids[row * K + rank] = static_cast<int32_t>(id);
+        gates[row * K + rank] = gate_sigmoid(scratch[warp].row[buffer_pos<Q>(e)]);
+      }
+      if (rank == K) alpha[row] = -key_to_float(key);
+      __syncwarp();
+    }
+  }
+}
+
 template <int Q, bool kFull, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
 cudaError_t launch_rows(const RouteParams& p, cudaStream_t s) {
   auto kern = route_rows_kernel<Q, kFull, kBias, kRoute, kAlphaOut, kAlphaIn, kWindow>;
@@ -401,6 +440,32 @@ cudaError_t launch_topk(const float* z, const float* bias, int64_t N, int32_t E,
   return dispatch(p, true, alpha != nullptr, false, false, s);
 }
 
+cudaError_t launch_select_fixup(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
+                                int32_t* ids, float* gates, float* alpha, cudaStream_t s) {
+  const int64_t rows_per_block = static_cast<int64_t>(kWarps) * 32;
+  int64_t blocks = (N + rows_per_block - 1) / rows_per_block;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 4;
+  if (blocks > cap) blocks = cap;
+  const bool full = (E % 128) == 0, b = bias != nullptr;
+  const dim3 grid(static_cast<unsigned>(blocks)), block(kThreads);
+#define KOLIBRI_FIXUP(Q)                                                                       \
+  if (full) {                                                                                  \
+    if (b) select_fixup_kernel<Q, true, true><<<grid, block, 0, s>>>(z, bias, N, E, K, ids, gates, alpha); \
+    else select_fixup_kernel<Q, true, false><<<grid, block, 0, s>>>(z, bias, N, E, K, ids, gates, alpha); \
+  } else {                                                                                     \
+    if (b) select_fixup_kernel<Q, false, true><<<grid, block, 0, s>>>(z, bias, N, E, K, ids, gates, alpha); \
+    else select_fixup_kernel<Q, false, false><<<grid, block, 0, s>>>(z, bias, N, E, K, ids, gates, alpha); \
+  }
+  switch ((E + 127) / 128) {
+    case 1: KOLIBRI_FIXUP(1) break;
+    case 2: KOLIBRI_FIXUP(2) break;
+    case 3: KOLIBRI_FIXUP(3) break;
+    default: return cudaErrorInvalidValue;   // the fused kernel covers E <= 384
+  }
+#undef KOLIBRI_FIXUP
+  return cudaGetLastError();
+}
+
 cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* bias, int64_t N,
                               int32_t E, int32_t K, int64_t S, int64_t stride, int64_t S_ld,
                               uint32_t* sample, cudaStream_t s) {
@@ -437,5 +502,7 @@ cudaError_t launch_route_window_pass(const float* z, const float* bias, const fl
   const bool route = ids != nullptr;
   return dispatch(p, route, alpha_out != nullptr, alpha_in != nullptr, true, s);
 }
+
+KOLIBRI_DEFINE_STATUS_TAKE(status_take_route)
 
 }  // namespace kolibri

@@ -96,6 +96,27 @@ KOLIBRI_API kolibri_status kolibri_router_logits(const void *x, const void *w, f
                                      int64_t N, int32_t d, int32_t E, void *stream);
 
 /*
+ * Router logits and selection in one call: kolibri_router_logits followed by
+ * kolibri_router_topk, with identical results ("Kolibri Pre-Training from
+ * Scratch" 6.1 and 7.1; "Kolibri 1 im Detail", routing steps 1 and 2).
+ *   x, w, z        as in kolibri_router_logits (z is still written in full)
+ *   bias           [E] fp32 selection bias beta, or NULL (B = Z exactly)
+ *   ids, gates     [N, K], written as by kolibri_router_topk
+ *   alpha          [N] fp32, written; required here (not NULL)
+ * For 16 <= E <= 384 with E >= 8 (K + 1) the selection runs inside the GEMM
+ * epilogue while the tensor cores compute the next tile, so Z is not read
+ * back for routing; rows with many tied scores are finished by a second
+ * kernel on the same stream.  Other shapes run the two kernels one after the
+ * other.  Shapes: d % 64 == 0, E % 16 == 0, plus the limits above.  Errors:
+ * KOLIBRI_ERR_INVALID_ARG for NULL or misaligned pointers (all 16-byte
+ * aligned), KOLIBRI_ERR_UNSUPPORTED_SHAPE otherwise; nothing is enqueued.
+ */
+KOLIBRI_API kolibri_status kolibri_router_forward(const void *x, const void *w, const float *bias,
+                                                  float *z, int64_t N, int32_t d, int32_t E,
+                                                  int32_t K, int32_t *ids, float *gates,
+                                                  float *alpha, void *stream);
+
+/*
  * Bias add, top-K selection and sigmoid gates ("Kolibri Pre-Training from
  * Scratch" 6.1 and 7.1; "Kolibri 1 im Detail", routing steps 1 and 2).
  *   z      [N, E] fp32 logits

@@ -1,0 +1,119 @@
+"""kolibri_router_forward (router GEMM with the selection in its epilogue).
+
+Z must equal kolibri_router_logits's Z bit for bit (the same tensor-core
+sums, the same order), and ids, gates and alpha must equal the oracle's
+selection on that Z bit for bit ("Kolibri Pre-Training from Scratch" 6.1 and
+7.1).  Covered: both column-group widths of the threshold, E that leaves
+epilogue warps without columns, ragged token tails, several tiles per CTA,
+heavy ties (rows finished by the row kernel) and the shapes that fall back
+to the two separate kernels."""
+import numpy as np
+import pytest
+import torch
+
+from expert_load_balancing_b200 import binding as B
+from expert_load_balancing_b200 import workloads
+
+from gpu_helpers import assert_bit_equal, check_status, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(kolibri_lib):
+    return kolibri_lib
+
+
+def _poisoned(N, E, K):
+    z = torch.full((N, E), float("nan"), device="cuda")
+    ids = torch.full((N, K), -7, dtype=torch.int32, device="cuda")
+    gates = torch.full((N, K), float("nan"), device="cuda")
+    alpha = torch.full((N,), 12345.0, device="cuda")
+    return z, ids, gates, alpha
+
+
+def _check(oracle_mod, x, w, beta, K):
+    N, E = x.shape[0], w.shape[0]
+    xd, wd = x.cuda(), w.cuda()
+    bd = None if beta is None else dev(beta)
+    z, ids, gates, alpha = _poisoned(N, E, K)
+    B.kolibri_router_forward(xd, wd, bd, K, z=z, ids=ids, gates=gates, alpha=alpha)
+    z_ref = B.kolibri_router_logits(xd, wd)
+    torch.cuda.synchronize()
+    check_status()
+    zf = host(z)
+    assert_bit_equal(zf, host(z_ref), "z")
+    oi, og, oa = oracle_mod.select(zf, beta, K)
+    assert_bit_equal(host(ids), oi, "ids")
+    assert_bit_equal(host(gates), og, "gates")
+    assert_bit_equal(host(alpha), oa, "alpha")
+
+
+CASES = [
+    # N, d, E, K, logit offsets, beta
+    (70001, 2560, 384, 6, "zipf1.1", "normal0.1"),   # Kolibri shape, ragged tail
+    (4099, 2048, 128, 8, "none", "normal0.1"),       # Origin shape: groups of 8 columns
+    (1000, 512, 384, 16, "collapsed8", "zeros"),     # largest K
+    (777, 256, 64, 6, "none", "normal0.1"),          # groups of 8, one warp of columns
+    (300, 640, 256, 2, "collapsed8", "normal0.1"),   # third column warp idle
+    (257, 1024, 336, 6, "zipf1.1", "normal0.1"),     # E % 32 == 16
+    (1, 2560, 384, 6, "none", "normal0.1"),
+    (255, 128, 384, 1, "none", "zeros"),
+    (77, 64, 16, 1, "none", "normal0.1"),           # smallest E: one 32-column TMEM block
+]
+
+
+@pytest.mark.parametrize("N,d,E,K,offsets,beta", CASES)
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_forward_matches_logits_and_oracle(oracle_mod, N, d, E, K, offsets, beta, with_bias):
+    wl = workloads.Workload("t", N, d, E, K, offsets=offsets, beta=beta)
+    b = workloads.make_beta(wl).numpy() if with_bias else None
+    _check(oracle_mod, workloads.make_x(wl), workloads.make_w(wl), b, K)
+
+
+def test_forward_many_tiles_per_cta(oracle_mod):
+    # more 256-token tiles than SM pairs: every CTA pair loops, and the
+    # per-row candidate counters are reused tile after tile
+    wl = workloads.Workload("t", 148 * 256 * 3 + 77, 256, 384, 6, offsets="zipf1.1", beta="normal0.1")
+    _check(oracle_mod, workloads.make_x(wl), workloads.make_w(wl), workloads.make_beta(wl).numpy(), 6)
+
+
+@pytest.mark.parametrize("E,K", [(400, 6), (48, 6)])
+def test_forward_fallback_shapes(oracle_mod, E, K):
+    # E > 384, or too few column groups for a (K+1)-th group maximum: the
+    # call runs the two kernels one after the other, with the same results
+    wl = workloads.Workload("t", 513, 512, E, K, beta="normal0.1")
+    _check(oracle_mod, workloads.make_x(wl), workloads.make_w(wl), workloads.make_beta(wl).numpy(), K)
+
+
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_forward_heavy_ties(oracle_mod, with_bias):
+    # identical router rows: every score of a token ties, far more candidates
+    # than the epilogue's per-row buffer, so the row kernel finishes them;
+    # zero tokens tie at exactly 0 (and +0 vs -0 never arises from sums)
+    N, d, E, K = 1500, 256, 384, 6
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(N, d, generator=g).to(torch.bfloat16)
+    x[::3] = 0
+    w = torch.randn(1, d, generator=g).repeat(E, 1)
+    w[E // 2:] = torch.randn(E - E // 2, d, generator=g)      # half the experts tie
+    w = (w / 16).to(torch.bfloat16)
+    beta = np.zeros(E, np.float32)
+    if with_bias:
+        beta[::5] = 0.25                                     # ties among biased scores too
+    _check(oracle_mod, x, w, beta if with_bias else None, K)
+
+
+def test_forward_rejects_bad_args():
+    x = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((16, 64), dtype=torch.bfloat16, device="cuda")
+    lib = B.load()
+    z = torch.empty((4, 16), device="cuda")
+    ids = torch.empty((4, 2), dtype=torch.int32, device="cuda")
+    g = torch.empty((4, 2), device="cuda")
+    p = lambda t: None if t is None else t.data_ptr()
+    st = lib.kolibri_router_forward(p(x), p(w), None, p(z), 4, 64, 16, 2, p(ids), p(g), None, None)
+    assert st == B.KOLIBRI_ERR_INVALID_ARG          # alpha is required
+    a = torch.empty((4,), device="cuda")
+    st = lib.kolibri_router_forward(p(x), p(w), None, p(z), 4, 96, 16, 2, p(ids), p(g), p(a), None)
+    assert st == B.KOLIBRI_ERR_UNSUPPORTED_SHAPE    # d % 64 != 0
