@@ -12,8 +12,8 @@
 // whole 256 x E accumulator tile out of TMEM into registers at once (thread
 // = token row, 128 fp32 columns per thread) and hands TMEM back to the MMA
 // before doing anything else, so selection overlaps the next tile's MMAs.
-// Z still goes to HBM (the EQB update reads it), through shared staging and
-// TMA stores.
+// Z still goes to HBM (the EQB update reads it): each 32 x 16 block passes
+// through shared memory so the global stores are coalesced.
 //
 // Warp roles (512 threads, setmaxnreg: warpgroup 0 at 32 registers, the
 // three epilogue warpgroups at 160):
@@ -52,13 +52,13 @@ constexpr int kRegsCtrl = 32;
 constexpr int kRegsEpi = 160;
 static_assert(kCtrlWarps * 32 * kRegsCtrl + kEpiWarps * 32 * kRegsEpi <= kThreads * 128,
               "register split exceeds what 512 threads are launched with");
-constexpr int kZCols = 16;               // fp32 columns per Z store box (16 or 32)
-constexpr int kZBuf = kZCols * 32 * 4;   // one staging buffer: 32 rows of the box
-constexpr int kZBufs = 1;                // staging buffers per epilogue warp
-static_assert(kZCols == 16 || kZCols == 32, "Z store boxes are 64- or 128-byte rows");
+constexpr int kZCols = 16;               // columns per block of the Z / candidate pass
+constexpr int kZBuf = kZCols * 32 * 4;   // per-warp copy of one block (2 KB)
 constexpr int kCap = 32;                 // candidate slots per row
+constexpr int kMaxRounds = KOLIBRI_MAX_TOPK + 1;
 
 struct FwdParams {
+  float* z;            // [N, E] logits, written
   const float* beta;   // null: B = Z
   int32_t* ids;
   float* gates;
@@ -75,7 +75,7 @@ __host__ __device__ inline FwdLayout fwd_layout(uint32_t ring_bytes, int groups_
   FwdLayout L;
   uint32_t o = ring_bytes;                 // multiple of 1 KB
   L.zstage = o;
-  o += kEpiWarps * kZBufs * kZBuf;
+  o += kEpiWarps * kZBuf;
   L.beta = o;
   o += kMaxE * 4;
   L.gsort = o;                             // f32 [3][groups][128]
@@ -95,12 +95,11 @@ __host__ __device__ inline FwdLayout fwd_layout(uint32_t ring_bytes, int groups_
   return L;
 }
 
-// Byte offset of 16-byte chunk `c` of staging row `row`, in the layout of
-// the TMA swizzle that matches the row length (64 B rows: chunk bits 4-5 are
-// XORed with address bits 7-8; 128 B rows: bits 4-6 with bits 7-9).
+// Byte offset of 16-byte chunk `c` of row `row` in a warp's 32 x 64 B block
+// copy.  The XOR keeps both access patterns free of bank conflicts: a lane
+// per row (writes, candidate reads) and four lanes per row (the copy-out).
 __device__ __forceinline__ uint32_t zstage_off(int row, int c) {
-  if constexpr (kZCols == 16) return static_cast<uint32_t>(row * 64 + ((c ^ ((row >> 1) & 3)) << 4));
-  return static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
+  return static_cast<uint32_t>(row * 64 + ((c ^ ((row >> 1) & 3)) << 4));
 }
 
 // 32 columns of TMEM into r[OFF .. OFF+31] (compile-time offsets only, so
@@ -146,6 +145,12 @@ __device__ __forceinline__ void sort_desc(float (&v)[n]) {
   }
 }
 
+// Candidate (k, c) precedes the running best (bk, bc): key descending, then
+// expert id ascending.
+__device__ __forceinline__ bool precedes(uint32_t k, uint32_t c, uint32_t bk, uint32_t bc) {
+  return k > bk || (k == bk && c < bc);
+}
+
 // Barrier of the three warps of one lane quarter (96 arrivals), bounded.
 __device__ __forceinline__ bool quarter_sync(uint32_t bar, uint32_t parity) {
   mbar_arrive(bar);
@@ -156,7 +161,7 @@ __device__ __forceinline__ bool quarter_sync(uint32_t bar, uint32_t parity) {
 
 template <int kG, bool kBias>
 __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdParams& p,
-                                                 const CUtensorMap* tm_z, const Ring& rg,
+                                                 const Ring& rg,
                                                  const FwdLayout& L, uint8_t* gbase,
                                                  uint32_t tmem_base, uint32_t rank, int warp,
                                                  int lane) {
@@ -173,8 +178,7 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
   const int col0 = j * kColsPerWarp;
   const int ncols = max(0, min(kColsPerWarp, sh.E - col0));  // multiple of 16
   const int rl = q * 32 + lane;              // row within the CTA's 128
-  const uint32_t zbuf0 = base + L.zstage + static_cast<uint32_t>((warp - 4) * kZBufs * kZBuf);
-  int nbuf = 0;
+  const uint32_t zbuf = base + L.zstage + static_cast<uint32_t>((warp - 4) * kZBuf);
   const uint32_t empty_leader = map_to_rank(rg.tmem_empty(), 0);
   const uint32_t bar_a = base + L.qbar + 16u * q, bar_b = bar_a + 8u;
   const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
@@ -251,14 +255,13 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
       }
     }
 
-    // 2. Z store (staging + TMA) and candidates, kZCols columns at a time
+    // 2. Z and the candidates, kZCols columns at a time.  The block goes to
+    // this warp's shared copy (a lane per row), then out to HBM with four
+    // lanes per row, so each store instruction writes eight whole 64-byte
+    // row segments; the candidates (scores >= T) are read from the copy.
 #pragma unroll
     for (int b = 0; b < kColsPerWarp / kZCols; ++b) {
       if (b * kZCols < ncols) {
-        const uint32_t zbuf = zbuf0 + static_cast<uint32_t>(nbuf * kZBuf);
-        nbuf = (nbuf + 1 == kZBufs) ? 0 : nbuf + 1;
-        if (lane == 0) bulk_wait_read<kZBufs - 1>();   // the store that last used zbuf has read it
-        __syncwarp();
 #pragma unroll
         for (int c = 0; c < kZCols / 4; ++c) {
           const int o = b * kZCols + 4 * c;
@@ -266,11 +269,19 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
                        "r"(r[o]), "r"(r[o + 1]), "r"(r[o + 2]), "r"(r[o + 3])
                        : "memory");
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(tm_z, col0 + b * kZCols, row_base, zbuf);
-          bulk_commit();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int rr = 8 * k + (lane >> 2), ch = lane & 3;
+          uint32_t v0, v1, v2, v3;
+          asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v0), "=r"(v1), "=r"(v2), "=r"(v3)
+                       : "r"(zbuf + zstage_off(rr, ch))
+                       : "memory");
+          const int64_t grow = static_cast<int64_t>(row_base) + rr;
+          if (grow < sh.N)
+            *reinterpret_cast<uint4*>(p.z + grow * sh.E + col0 + b * kZCols + 4 * ch) =
+                make_uint4(v0, v1, v2, v3);
         }
         uint32_t m = 0u;
 #pragma unroll
@@ -295,6 +306,7 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
             cc[slot * 128 + rl] = static_cast<uint16_t>(col0 + b * kZCols + i);
           }
         }
+        __syncwarp();   // every lane is done with the copy before the next block
       }
     }
     if (!quarter_sync(bar_b, qphase)) return;
@@ -325,35 +337,56 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
           }
         }
       }
-      uint32_t taken = 0u;
-      for (int t = 0; t <= K && n > 0u; ++t) {
-        uint32_t bk = 0u, bc = 0xffffu, bi = 0u;
+      // K+1 rounds (static, so winners stay in registers); each round scans
+      // the candidates in four independent chains and then combines them
+      uint32_t taken = 0u, akey = 0u;
+      uint32_t wc[kMaxRounds], wi[kMaxRounds];
 #pragma unroll
-        for (int c8 = 0; c8 < kCap / 8; ++c8) {
-          if (static_cast<uint32_t>(8 * c8) < nmax) {
+      for (int t = 0; t < kMaxRounds; ++t) {
+        wc[t] = 0u;
+        wi[t] = 0u;
+        if (t <= K) {
+          uint32_t bk[4] = {0u, 0u, 0u, 0u}, bc[4] = {0xffffu, 0xffffu, 0xffffu, 0xffffu};
+          uint32_t bi[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const int i = 8 * c8 + u;
-              const bool better =
-                  !((taken >> i) & 1u) && (ck[i] > bk || (ck[i] == bk && ci[i] < bc));
-              bk = better ? ck[i] : bk;
-              bc = better ? ci[i] : bc;
-              bi = better ? static_cast<uint32_t>(i) : bi;
+          for (int c8 = 0; c8 < kCap / 8; ++c8) {
+            if (static_cast<uint32_t>(8 * c8) < nmax) {
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const int i = 8 * c8 + u, ch = u & 3;
+                const bool better = !((taken >> i) & 1u) && precedes(ck[i], ci[i], bk[ch], bc[ch]);
+                bk[ch] = better ? ck[i] : bk[ch];
+                bc[ch] = better ? ci[i] : bc[ch];
+                bi[ch] = better ? static_cast<uint32_t>(i) : bi[ch];
+              }
             }
           }
+#pragma unroll
+          for (int ch = 1; ch < 4; ++ch) {
+            const bool better = precedes(bk[ch], bc[ch], bk[0], bc[0]);
+            bk[0] = better ? bk[ch] : bk[0];
+            bc[0] = better ? bc[ch] : bc[0];
+            bi[0] = better ? bi[ch] : bi[0];
+          }
+          taken |= 1u << bi[0];
+          wc[t] = bc[0];
+          wi[t] = bi[0];
+          if (t == K) akey = bk[0];
         }
-        taken |= 1u << bi;
-        if (t < K) {
-          p.ids[row * K + t] = static_cast<int32_t>(bc);
-          p.gates[row * K + t] = gate_sigmoid(cz[bi * 128 + rl]);
-        } else {
-          p.alpha[row] = -key_to_float(bk);
+      }
+      if (n > 0u) {
+#pragma unroll
+        for (int t = 0; t < kMaxRounds - 1; ++t) {
+          if (t < K) {
+            p.ids[row * K + t] = static_cast<int32_t>(wc[t]);
+            p.gates[row * K + t] = gate_sigmoid(cz[wi[t] * 128 + rl]);
+          }
         }
+        p.alpha[row] = -key_to_float(akey);
       }
       if (overflow && row < sh.N) p.alpha[row] = __uint_as_float(0x7fc00000u);  // finished by the row kernel
     }
   }
-  if (lane == 0) bulk_wait_all();
 }
 
 // ---- kernel ---------------------------------------------------------------
@@ -362,7 +395,7 @@ template <int kG, bool kBias>
 __global__ void __launch_bounds__(kThreads, 1)
     router_forward_kernel(const __grid_constant__ CUtensorMap tm_x,
                           const __grid_constant__ CUtensorMap tm_w,
-                          const __grid_constant__ CUtensorMap tm_z, const GemmShape sh,
+                          const GemmShape sh,
                           const FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -380,7 +413,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     init_barriers(sh, rg, 2 * kEpiWarps);
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_z)) : "memory");
   }
   {
     float* beta_s = reinterpret_cast<float*>(gbase + L.beta);
@@ -409,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEpi));
-    forward_epilogue<kG, kBias>(sh, p, &tm_z, rg, L, gbase, tmem_base, rank, warp, lane);
+    forward_epilogue<kG, kBias>(sh, p, rg, L, gbase, tmem_base, rank, warp, lane);
   }
 
   tc_fence_before();
@@ -425,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---- host -----------------------------------------------------------------
 
 template <int kG, bool kBias>
-cudaError_t launch_fwd(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const CUtensorMap& tm_z,
+cudaError_t launch_fwd(const CUtensorMap& tm_x, const CUtensorMap& tm_w,
                        const GemmShape& sh, const FwdParams& p, size_t smem, cudaStream_t s) {
   auto kern = router_forward_kernel<kG, kBias>;
   // setmaxnreg hands registers between warpgroups inside the block's launch
@@ -466,7 +498,7 @@ cudaError_t launch_fwd(const CUtensorMap& tm_x, const CUtensorMap& tm_w, const C
   }
   const int64_t clusters = sh.num_pairs < max_clusters ? sh.num_pairs : max_clusters;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  err = cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, tm_z, sh, p);
+  err = cudaLaunchKernelEx(&cfg, kern, tm_x, tm_w, sh, p);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
@@ -495,20 +527,16 @@ cudaError_t launch_router_forward(const void* x, const void* w, const float* bia
   sh.stages = stages;
   const size_t smem = fixed + stage_bytes * stages;
 
-  CUtensorMap tm_x, tm_w, tm_z;
+  CUtensorMap tm_x, tm_w;
   if (!encode_operands(sh, x, w, &tm_x, &tm_w)) return cudaErrorInvalidValue;
-  if (!encode_2d(&tm_z, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, z, static_cast<uint64_t>(E),
-                 static_cast<uint64_t>(N), kZCols, 32,
-                 kZCols == 16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
 
-  FwdParams p{bias, ids, gates, alpha, K};
+  FwdParams p{z, bias, ids, gates, alpha, K};
   const bool b = bias != nullptr;
   if (kg == 16)
-    return b ? launch_fwd<16, true>(tm_x, tm_w, tm_z, sh, p, smem, s)
-             : launch_fwd<16, false>(tm_x, tm_w, tm_z, sh, p, smem, s);
-  return b ? launch_fwd<8, true>(tm_x, tm_w, tm_z, sh, p, smem, s)
-           : launch_fwd<8, false>(tm_x, tm_w, tm_z, sh, p, smem, s);
+    return b ? launch_fwd<16, true>(tm_x, tm_w, sh, p, smem, s)
+             : launch_fwd<16, false>(tm_x, tm_w, sh, p, smem, s);
+  return b ? launch_fwd<8, true>(tm_x, tm_w, sh, p, smem, s)
+           : launch_fwd<8, false>(tm_x, tm_w, sh, p, smem, s);
 }
 
 KOLIBRI_DEFINE_STATUS_TAKE(status_take_forward)
