@@ -185,25 +185,38 @@ class RouterStep:
         self.q = torch.empty((E,), dtype=torch.float32, device=device)
         self.ws_perm = B.workspace(B.KOLIBRI_OP_PERMUTE, N, E, K, device)
         self.ws_eqb = B.workspace(B.KOLIBRI_OP_EQB, N, E, K, device)
+        # the permutation needs only ids: it runs on a second stream while
+        # the EQB update runs on the first
+        self.side = torch.cuda.Stream(device)
+        self.fork = torch.cuda.Event()
+        self.join = torch.cuda.Event()
 
     def run(self, stream, events=None):
-        """logits + routing (selection in the GEMM epilogue) -> EQB update of
-        beta from that alpha (one bracketed read of Z) -> permutation."""
+        """logits + routing (selection in the GEMM epilogue), then on two
+        streams: the EQB update of beta from that alpha (one bracketed read
+        of Z) and the permutation.  events (6, optional): start, forward
+        done, EQB done, permutation start and end (second stream), step end."""
         wl = self.wl
         if events:
             events[0].record(stream)
         B.kolibri_router_forward(self.x, self.w, self.beta, wl.K, z=self.z, ids=self.ids,
                                  gates=self.gates, alpha=self.alpha, stream=stream)
+        fork = events[1] if events else self.fork
+        fork.record(stream)
+        self.side.wait_event(fork)
         if events:
-            events[1].record(stream)
+            events[3].record(self.side)
+        B.kolibri_expert_permute(self.ids, wl.E, self.ws_perm, self.counts, self.offsets,
+                                 self.perm, self.inv, stream=self.side)
+        join = events[4] if events else self.join
+        join.record(self.side)
         B.kolibri_eqb_update(self.z, self.alpha, self.beta, wl.K, self.ws_eqb, self.q,
                              stream=stream)
         if events:
             events[2].record(stream)
-        B.kolibri_expert_permute(self.ids, wl.E, self.ws_perm, self.counts, self.offsets,
-                                 self.perm, self.inv, stream=stream)
+        stream.wait_event(join)
         if events:
-            events[3].record(stream)
+            events[5].record(stream)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -226,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device status after warm-up: {B.status_string(st)}")
 
     # ---- timed region: device time, CUDA events on the launching stream
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
@@ -246,7 +259,8 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     total_ms = t0.elapsed_time(t1)
-    stage_ms = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(3)]
+    stage_ms = np.array([[ev[i][0].elapsed_time(ev[i][1]), ev[i][1].elapsed_time(ev[i][2]),
+                          ev[i][3].elapsed_time(ev[i][4])]
                          for i in range(args.steps)]).mean(axis=0)
     st = B.kolibri_device_status(stream)
     if st != B.KOLIBRI_OK:
@@ -293,7 +307,7 @@ def run_ours(args, rank, world, local_rank):
                           "flops": flops, "bytes": bytes_,
                           "peaks": f"bf16 burst {peaks['bf16_tflops']} TF/s, HBM {peaks['hbm_gbs']} GB/s, of {peaks['source']}"},
         "stages_ms": {"logits_and_routing": gemm_ms, "eqb_update": float(stage_ms[1]),
-                      "permute": float(stage_ms[2])},
+                      "permute_concurrent": float(stage_ms[2])},
         "gpu_launches": launches_per_step(N, E, K) * args.steps,
         "clocks": clocks,
         "e2e": e2e,

@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     kolibri_expert_permute_noalloc,
     kolibri_route_and_balance,
     kolibri_router_forward,
+    kolibri_router_forward_eqb,
     kolibri_router_logits,
     kolibri_router_topk,
     kolibri_workspace_bytes,

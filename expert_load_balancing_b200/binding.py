@@ -33,6 +33,8 @@ SIGNATURES = {
     "kolibri_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I32, _I32]),
     "kolibri_router_logits": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P]),
     "kolibri_router_forward": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _P, _P, _P]),
+    "kolibri_router_forward_eqb": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _P,
+                                                  _P, _P, _P, _SZ, _P]),
     "kolibri_router_topk": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P]),
     "kolibri_expert_permute": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "kolibri_expert_permute_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P]),
@@ -145,6 +147,39 @@ def kolibri_router_forward(x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor 
            load().kolibri_router_forward(_ptr(x), _ptr(w), _ptr(bias), _ptr(z), N, d, E, K,
                                          _ptr(ids), _ptr(gates), _ptr(alpha), _stream(stream)))
     return z, ids, gates, alpha
+
+
+def kolibri_router_forward_eqb(x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor, K: int,
+                               ws: torch.Tensor | None = None, z: torch.Tensor | None = None,
+                               ids: torch.Tensor | None = None, gates: torch.Tensor | None = None,
+                               alpha: torch.Tensor | None = None,
+                               quantiles: torch.Tensor | None = None, stream=None):
+    """Logits, routing with ``bias`` and the EQB update of ``bias`` in place.
+
+    Returns (z, ids, gates, alpha, quantiles)."""
+    N, d = x.shape
+    E = w.shape[0]
+    _need(x, torch.bfloat16, (N, d), "x")
+    _need(w, torch.bfloat16, (E, d), "w")
+    _need(bias, torch.float32, (E,), "bias")
+    dev = x.device
+    if ws is None:
+        ws = workspace(KOLIBRI_OP_EQB, N, E, K, dev)
+    z = torch.empty((N, E), dtype=torch.float32, device=dev) if z is None else z
+    ids = torch.empty((N, K), dtype=torch.int32, device=dev) if ids is None else ids
+    gates = torch.empty((N, K), dtype=torch.float32, device=dev) if gates is None else gates
+    alpha = torch.empty((N,), dtype=torch.float32, device=dev) if alpha is None else alpha
+    quantiles = torch.empty((E,), dtype=torch.float32, device=dev) if quantiles is None else quantiles
+    _need(z, torch.float32, (N, E), "z")
+    _need(ids, torch.int32, (N, K), "ids")
+    _need(gates, torch.float32, (N, K), "gates")
+    _need(alpha, torch.float32, (N,), "alpha")
+    _need(quantiles, torch.float32, (E,), "quantiles")
+    _check("kolibri_router_forward_eqb",
+           load().kolibri_router_forward_eqb(_ptr(x), _ptr(w), _ptr(bias), _ptr(z), N, d, E, K,
+                                             _ptr(ids), _ptr(gates), _ptr(alpha), _ptr(quantiles),
+                                             _ptr(ws), ws.numel(), _stream(stream)))
+    return z, ids, gates, alpha, quantiles
 
 
 def kolibri_router_topk(z: torch.Tensor, bias: torch.Tensor | None, K: int,

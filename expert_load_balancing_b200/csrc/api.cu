@@ -80,17 +80,25 @@ kolibri_status kolibri_router_forward(const void* x, const void* w, const float*
     return KOLIBRI_ERR_INVALID_ARG;
   if (d < 1) return KOLIBRI_ERR_INVALID_ARG;
   if (d % 64 != 0 || E % 16 != 0) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (router_forward_supported(E, K)) {
-    const cudaError_t err = launch_router_forward(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
-    if (err == cudaSuccess)
-      return from_cuda(launch_select_fixup(z, bias, N, E, K, ids, gates, alpha, s));
-    if (err != cudaErrorNotSupported) return KOLIBRI_ERR_CUDA;
-  }
-  // shapes outside the fused kernel: the two kernels one after the other
-  const cudaError_t err = launch_router_logits(x, w, z, N, d, E, s);
-  if (err != cudaSuccess) return KOLIBRI_ERR_CUDA;
-  return from_cuda(launch_topk(z, bias, N, E, K, ids, gates, alpha, s));
+  return from_cuda(router_forward_any(x, w, bias, z, N, d, E, K, ids, gates, alpha,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_router_forward_eqb(const void* x, const void* w, float* bias, float* z,
+                                          int64_t N, int32_t d, int32_t E, int32_t K,
+                                          int32_t* ids, float* gates, float* alpha,
+                                          float* quantiles, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!x || !w || !bias || !z || !ids || !gates || !ws) return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(z) || !aligned16(bias) || !aligned16(ws))
+    return KOLIBRI_ERR_INVALID_ARG;
+  if (d < 1) return KOLIBRI_ERR_INVALID_ARG;
+  if (d % 64 != 0 || E % 16 != 0) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < eqb_layout(N, E, K).total) return KOLIBRI_ERR_WORKSPACE_TOO_SMALL;
+  return from_cuda(launch_forward_eqb(x, w, bias, z, N, d, E, K, ids, gates, alpha, quantiles, ws,
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 kolibri_status kolibri_router_topk(const float* z, const float* bias, int64_t N, int32_t E,

@@ -311,15 +311,12 @@ EqbBuffers eqb_buffers(int64_t N, int32_t E, int32_t K, void* ws) {
   return b;
 }
 
-// Steps 1-2: sample keys (token bias given, or computed from bias_in), then
-// either the exact quantile (small N) or the per-expert bracket.
-cudaError_t eqb_begin(const float* z, const float* alpha, const float* bias, int64_t N, int32_t E,
-                      int32_t K, const EqbBuffers& b, cudaStream_t s) {
+// Step 2 from the sample keys: either the exact quantile (small N) or the
+// per-expert bracket, with the full-pass counters cleared.
+cudaError_t eqb_brackets(int64_t N, int32_t E, int32_t K, const EqbBuffers& b, cudaStream_t s) {
   const EqbLayout& L = b.L;
   const int64_t m = (N * static_cast<int64_t>(K)) / E;
-  cudaError_t err = launch_eqb_sample(z, alpha, alpha ? nullptr : bias, N, E, K, L.S, L.stride,
-                                      L.S_ld, b.sample, s);
-  if (err != cudaSuccess) return err;
+  cudaError_t err;
   if (L.exact_small) {
     err = set_select_smem();
     if (err != cudaSuccess) return err;
@@ -344,6 +341,17 @@ cudaError_t eqb_begin(const float* z, const float* alpha, const float* bias, int
   sample_select_kernel<<<E, kSelThreads, select_smem(L.S), s>>>(b.sample, L.S, 0, r_hi, r_lo,
                                                                  L.S_ld, false, b.v, b.lo, b.hi);
   return cudaGetLastError();
+}
+
+// Steps 1-2: sample keys (token bias given, or computed from bias_in), then
+// the brackets (or the exact quantile for small N).
+cudaError_t eqb_begin(const float* z, const float* alpha, const float* bias, int64_t N, int32_t E,
+                      int32_t K, const EqbBuffers& b, cudaStream_t s) {
+  const EqbLayout& L = b.L;
+  cudaError_t err = launch_eqb_sample(z, alpha, alpha ? nullptr : bias, N, E, K, L.S, L.stride,
+                                      L.S_ld, b.sample, s);
+  if (err != cudaSuccess) return err;
+  return eqb_brackets(N, E, K, b, s);
 }
 
 // Steps 4-5 and the bias update.
@@ -381,6 +389,21 @@ cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t 
     if (!alpha) alpha_used = b.alpha_ws;
   }
   return eqb_end(z, alpha_used, bias, N, E, K, quantiles, b, s);
+}
+
+// Logits, routing and the EQB update from the tokens: the fused GEMM +
+// selection, then the update from the alpha it wrote.  (Running the
+// bracketed full pass inside the GEMM epilogue as well, from brackets taken
+// first on a sampled-row GEMM, measured slower on B200: the epilogue is
+// latency-bound and the separate pass streams Z near HBM speed.)
+cudaError_t launch_forward_eqb(const void* x, const void* w, float* bias, float* z, int64_t N,
+                               int32_t d, int32_t E, int32_t K, int32_t* ids, float* gates,
+                               float* alpha, float* quantiles, void* ws, cudaStream_t s) {
+  const EqbBuffers b = eqb_buffers(N, E, K, ws);
+  float* alpha_out = alpha ? alpha : b.alpha_ws;
+  const cudaError_t err = router_forward_any(x, w, bias, z, N, d, E, K, ids, gates, alpha_out, s);
+  if (err != cudaSuccess) return err;
+  return launch_eqb(z, alpha_out, bias, N, E, K, quantiles, ws, s);
 }
 
 cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t E, int32_t K,

@@ -63,6 +63,16 @@ cudaError_t launch_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K, 
 cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
                        int32_t K, float* quantiles, void* ws, cudaStream_t s);
 
+// Logits + selection by whichever path covers the shape (fused kernel and
+// its row check, or the GEMM then the row kernel).
+cudaError_t router_forward_any(const void* x, const void* w, const float* bias, float* z,
+                               int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                               float* gates, float* alpha, cudaStream_t s);
+
+cudaError_t launch_forward_eqb(const void* x, const void* w, float* bias, float* z, int64_t N,
+                               int32_t d, int32_t E, int32_t K, int32_t* ids, float* gates,
+                               float* alpha, float* quantiles, void* ws, cudaStream_t s);
+
 cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t E, int32_t K,
                                  int32_t* ids, float* gates, float* alpha, float* quantiles,
                                  void* ws, cudaStream_t s);

@@ -55,7 +55,6 @@ static_assert(kCtrlWarps * 32 * kRegsCtrl + kEpiWarps * 32 * kRegsEpi <= kThread
 constexpr int kZCols = 16;               // columns per block of the Z / candidate pass
 constexpr int kZBuf = kZCols * 32 * 4;   // per-warp copy of one block (2 KB)
 constexpr int kCap = 32;                 // candidate slots per row
-constexpr int kMaxRounds = KOLIBRI_MAX_TOPK + 1;
 
 struct FwdParams {
   float* z;            // [N, E] logits, written
@@ -68,7 +67,7 @@ struct FwdParams {
 
 // Shared memory after the operand ring (offsets from the 1 KB aligned base).
 struct FwdLayout {
-  uint32_t zstage, beta, gsort, cz, cc, rowcnt, qbar, bars, total;
+  uint32_t zstage, beta, gsort, cz, cc, rowcnt, alpha, qbar, bars, total;
 };
 
 __host__ __device__ inline FwdLayout fwd_layout(uint32_t ring_bytes, int groups_per_warp) {
@@ -86,9 +85,11 @@ __host__ __device__ inline FwdLayout fwd_layout(uint32_t ring_bytes, int groups_
   o += kCap * 128 * 2;
   L.rowcnt = o;                            // u32 [128]
   o += 128 * 4;
+  L.alpha = o;                             // f32 [128] this tile's token biases
+  o += 128 * 4;
   o = (o + 7u) & ~7u;
-  L.qbar = o;                              // per quarter: two mbarriers
-  o += 4 * 2 * 8;
+  L.qbar = o;                              // per quarter: three mbarriers
+  o += 4 * 3 * 8;
   L.bars = o;
   o += 8 * (2 * kMaxStages + 3);
   L.total = o;
@@ -172,6 +173,7 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
   float* cz = reinterpret_cast<float*>(gbase + L.cz);
   uint16_t* cc = reinterpret_cast<uint16_t*>(gbase + L.cc);
   uint32_t* rowcnt = reinterpret_cast<uint32_t*>(gbase + L.rowcnt);
+  float* alpha_s = reinterpret_cast<float*>(gbase + L.alpha);
 
   const int q = warp & 3;                    // TMEM lane quarter
   const int j = (warp - 4) >> 2;             // column third
@@ -180,7 +182,7 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
   const int rl = q * 32 + lane;              // row within the CTA's 128
   const uint32_t zbuf = base + L.zstage + static_cast<uint32_t>((warp - 4) * kZBuf);
   const uint32_t empty_leader = map_to_rank(rg.tmem_empty(), 0);
-  const uint32_t bar_a = base + L.qbar + 16u * q, bar_b = bar_a + 8u;
+  const uint32_t bar_a = base + L.qbar + 24u * q, bar_b = bar_a + 8u, bar_c = bar_a + 16u;
   const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
   uint32_t cl[4];
 #pragma unroll
@@ -310,7 +312,6 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
       }
     }
     if (!quarter_sync(bar_b, qphase)) return;
-    qphase ^= 1u;
 
     // 3. one warp per quarter ranks the row's candidates: their keys and
     // ids go to registers once, then K+1 rounds pick the best not yet taken
@@ -337,55 +338,55 @@ __device__ __forceinline__ void forward_epilogue(const GemmShape& sh, const FwdP
           }
         }
       }
-      // K+1 rounds (static, so winners stay in registers); each round scans
-      // the candidates in four independent chains and then combines them
+      // K+1 rounds, each a scan of the candidates in four independent
+      // chains; the winners' ids go out at once, their slots to the (now
+      // read) id buffer for the gate step below
       uint32_t taken = 0u, akey = 0u;
-      uint32_t wc[kMaxRounds], wi[kMaxRounds];
+#pragma unroll 1
+      for (int t = 0; t <= K; ++t) {
+        uint32_t bk[4] = {0u, 0u, 0u, 0u}, bc[4] = {0xffffu, 0xffffu, 0xffffu, 0xffffu};
+        uint32_t bi[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-      for (int t = 0; t < kMaxRounds; ++t) {
-        wc[t] = 0u;
-        wi[t] = 0u;
-        if (t <= K) {
-          uint32_t bk[4] = {0u, 0u, 0u, 0u}, bc[4] = {0xffffu, 0xffffu, 0xffffu, 0xffffu};
-          uint32_t bi[4] = {0u, 0u, 0u, 0u};
+        for (int c8 = 0; c8 < kCap / 8; ++c8) {
+          if (static_cast<uint32_t>(8 * c8) < nmax) {
 #pragma unroll
-          for (int c8 = 0; c8 < kCap / 8; ++c8) {
-            if (static_cast<uint32_t>(8 * c8) < nmax) {
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const int i = 8 * c8 + u, ch = u & 3;
-                const bool better = !((taken >> i) & 1u) && precedes(ck[i], ci[i], bk[ch], bc[ch]);
-                bk[ch] = better ? ck[i] : bk[ch];
-                bc[ch] = better ? ci[i] : bc[ch];
-                bi[ch] = better ? static_cast<uint32_t>(i) : bi[ch];
-              }
+            for (int u = 0; u < 8; ++u) {
+              const int i = 8 * c8 + u, ch = u & 3;
+              const bool better = !((taken >> i) & 1u) && precedes(ck[i], ci[i], bk[ch], bc[ch]);
+              bk[ch] = better ? ck[i] : bk[ch];
+              bc[ch] = better ? ci[i] : bc[ch];
+              bi[ch] = better ? static_cast<uint32_t>(i) : bi[ch];
             }
           }
+        }
 #pragma unroll
-          for (int ch = 1; ch < 4; ++ch) {
-            const bool better = precedes(bk[ch], bc[ch], bk[0], bc[0]);
-            bk[0] = better ? bk[ch] : bk[0];
-            bc[0] = better ? bc[ch] : bc[0];
-            bi[0] = better ? bi[ch] : bi[0];
-          }
-          taken |= 1u << bi[0];
-          wc[t] = bc[0];
-          wi[t] = bi[0];
-          if (t == K) akey = bk[0];
+        for (int ch = 1; ch < 4; ++ch) {
+          const bool better = precedes(bk[ch], bc[ch], bk[0], bc[0]);
+          bk[0] = better ? bk[ch] : bk[0];
+          bc[0] = better ? bc[ch] : bc[0];
+          bi[0] = better ? bi[ch] : bi[0];
+        }
+        taken |= 1u << bi[0];
+        if (t < K) {
+          if (n > 0u) p.ids[row * K + t] = static_cast<int32_t>(bc[0]);
+          cc[t * 128 + rl] = static_cast<uint16_t>(bi[0]);
+        } else {
+          akey = bk[0];
         }
       }
-      if (n > 0u) {
-#pragma unroll
-        for (int t = 0; t < kMaxRounds - 1; ++t) {
-          if (t < K) {
-            p.ids[row * K + t] = static_cast<int32_t>(wc[t]);
-            p.gates[row * K + t] = gate_sigmoid(cz[wi[t] * 128 + rl]);
-          }
-        }
-        p.alpha[row] = -key_to_float(akey);
-      }
+      if (n > 0u) p.alpha[row] = -key_to_float(akey);
       if (overflow && row < sh.N) p.alpha[row] = __uint_as_float(0x7fc00000u);  // finished by the row kernel
+      alpha_s[rl] = (n > 0u) ? -key_to_float(akey) : __uint_as_float(0x7fc00000u);
     }
+
+    // the three warps share the fp64 gates: warp j takes ranks t = j mod 3
+    if (!quarter_sync(bar_c, qphase)) return;
+    if (!isnan(alpha_s[rl])) {
+      for (int t = j; t < K; t += 3)
+        p.gates[row * K + t] = gate_sigmoid(cz[cc[t * 128 + rl] * 128 + rl]);
+    }
+
+    qphase ^= 1u;
   }
 }
 
@@ -409,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_rank();
 
   if (threadIdx.x == 0) {
-    for (int qq = 0; qq < 8; ++qq) mbar_init(base + L.qbar + 8u * qq, 96);
+    for (int qq = 0; qq < 12; ++qq) mbar_init(base + L.qbar + 8u * qq, 96);
     init_barriers(sh, rg, 2 * kEpiWarps);
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
@@ -420,6 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       beta_s[i] = (kBias && i < sh.E) ? p.beta[i] : 0.f;
     uint32_t* rowcnt = reinterpret_cast<uint32_t*>(gbase + L.rowcnt);
     for (int i = threadIdx.x; i < 128; i += kThreads) rowcnt[i] = 0u;
+
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(rg.holder()),
@@ -530,13 +532,27 @@ cudaError_t launch_router_forward(const void* x, const void* w, const float* bia
   CUtensorMap tm_x, tm_w;
   if (!encode_operands(sh, x, w, &tm_x, &tm_w)) return cudaErrorInvalidValue;
 
-  FwdParams p{z, bias, ids, gates, alpha, K};
+  const FwdParams p{z, bias, ids, gates, alpha, K};
   const bool b = bias != nullptr;
   if (kg == 16)
     return b ? launch_fwd<16, true>(tm_x, tm_w, sh, p, smem, s)
              : launch_fwd<16, false>(tm_x, tm_w, sh, p, smem, s);
   return b ? launch_fwd<8, true>(tm_x, tm_w, sh, p, smem, s)
            : launch_fwd<8, false>(tm_x, tm_w, sh, p, smem, s);
+}
+
+cudaError_t router_forward_any(const void* x, const void* w, const float* bias, float* z,
+                               int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                               float* gates, float* alpha, cudaStream_t s) {
+  if (router_forward_supported(E, K)) {
+    const cudaError_t err = launch_router_forward(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+    if (err == cudaSuccess) return launch_select_fixup(z, bias, N, E, K, ids, gates, alpha, s);
+    if (err != cudaErrorNotSupported) return err;
+  }
+  // shapes outside the fused kernel: the two kernels one after the other
+  const cudaError_t err = launch_router_logits(x, w, z, N, d, E, s);
+  if (err != cudaSuccess) return err;
+  return launch_topk(z, bias, N, E, K, ids, gates, alpha, s);
 }
 
 KOLIBRI_DEFINE_STATUS_TAKE(status_take_forward)

@@ -117,6 +117,25 @@ KOLIBRI_API kolibri_status kolibri_router_forward(const void *x, const void *w, 
                                                   float *alpha, void *stream);
 
 /*
+ * One training step's routing from the tokens: logits, selection with bias
+ * beta_in, and the EQB update of bias to beta_out ("Kolibri Pre-Training
+ * from Scratch" 6.1, 7.1 update rule, 7.2 order of operations, 7.3 exact
+ * quantile): kolibri_router_forward followed by kolibri_eqb_update with the
+ * alpha it produced, in one call on one stream.
+ *   x, w, z, ids, gates   as in kolibri_router_forward
+ *   bias                  [E] fp32, in: beta_in (routes), out: beta_out
+ *   alpha                 [N] fp32, written if not NULL (else kept in ws)
+ *   quantiles             [E] fp32, written if not NULL: v_e
+ *   ws, ws_bytes          kolibri_workspace_bytes(KOLIBRI_OP_EQB, N, E, K)
+ * Errors: as kolibri_router_forward and kolibri_eqb_update.
+ */
+KOLIBRI_API kolibri_status kolibri_router_forward_eqb(const void *x, const void *w, float *bias,
+                                                      float *z, int64_t N, int32_t d, int32_t E,
+                                                      int32_t K, int32_t *ids, float *gates,
+                                                      float *alpha, float *quantiles, void *ws,
+                                                      size_t ws_bytes, void *stream);
+
+/*
  * Bias add, top-K selection and sigmoid gates ("Kolibri Pre-Training from
  * Scratch" 6.1 and 7.1; "Kolibri 1 im Detail", routing steps 1 and 2).
  *   z      [N, E] fp32 logits
