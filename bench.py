@@ -278,10 +278,12 @@ def run_ours(args, rank, world, local_rank):
         return None
     peaks = _peaks()
     flops, bytes_ = algorithmic_work(N, d, E, K)
-    roof_ms = max(flops / (peaks["bf16_tflops"] * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    roof_ms = max(flops / (peaks["bf16_tflops_sustained"] * 1e12),
+                  bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
     gemm_ms = float(stage_ms[0])   # the fused GEMM + selection, and the row check after it
     gemm_tflops = 2.0 * N * d * E / (gemm_ms * 1e-3) / 1e12
-    peak_t = peaks["bf16_tflops"]  # burst: the timed region is tens of ms at max clocks
+    # the timed region runs ~1 s under the 1 kW power cap: the sustained peak
+    peak_t = peaks["bf16_tflops_sustained"]
     traffic = _traffic_from_profile(N)
     line = {
         "metric": METRIC,
@@ -302,10 +304,11 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "router_forward_kernel",
                      "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": gemm_tflops / peak_t, "traffic": traffic,
-                     "peak_kind": f"bf16 burst (cuBLAS 8192^3), of {peaks['source']}", "sustained_frac": gemm_tflops / peaks["bf16_tflops_sustained"]},
+                     "peak_kind": f"bf16 sustained (cuBLAS, seconds-long loop under the power cap), of {peaks['source']}",
+                     "burst_frac": gemm_tflops / peaks["bf16_tflops"]},
         "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ms_per_step,
                           "flops": flops, "bytes": bytes_,
-                          "peaks": f"bf16 burst {peaks['bf16_tflops']} TF/s, HBM {peaks['hbm_gbs']} GB/s, of {peaks['source']}"},
+                          "peaks": f"bf16 sustained {peaks['bf16_tflops_sustained']} TF/s, HBM {peaks['hbm_gbs']} GB/s, of {peaks['source']}"},
         "stages_ms": {"logits_and_routing": gemm_ms, "eqb_update": float(stage_ms[1]),
                       "permute_concurrent": float(stage_ms[2])},
         "gpu_launches": launches_per_step(N, E, K) * args.steps,
@@ -319,7 +322,7 @@ def run_ours(args, rank, world, local_rank):
 
 GEMM_PROFILE = os.path.join(ROOT, "profiles", "router_forward_kolibri.md")
 GEMM_SOURCES = [os.path.join(ROOT, "expert_load_balancing_b200", "csrc", f)
-                for f in ("router_forward.cu", "gemm_pair.cuh")]
+                for f in ("router_forward.cu", "gemm_pair.cuh", "common.cuh")]
 
 
 def kernel_source_digest():
@@ -466,7 +469,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=400)   # ~1 s timed: clock samples fall inside it
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="kolibri_n1m", choices=sorted(workloads.WORKLOADS))
