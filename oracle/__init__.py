@@ -67,6 +67,16 @@ def _load():
     lib.oracle_intervention_rate.argtypes = [P, P, i64, i32]
     lib.oracle_intervention_rate.restype = f64
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_bf16_round.argtypes = [f32]
+    lib.oracle_bf16_round.restype = ctypes.c_uint16
+    lib.oracle_bf16_key.argtypes = [ctypes.c_uint16]
+    lib.oracle_bf16_key.restype = ctypes.c_uint16
+    lib.oracle_column_quantiles_bf16.argtypes = [P, P, i64, i32, i64, P]
+    lib.oracle_tanh_spec.argtypes = [f64]
+    lib.oracle_tanh_spec.restype = f64
+    lib.oracle_lei_delta.argtypes = [P, i64, i32, i32, f64, f64, P]
+    lib.oracle_lei_inject.argtypes = [P, i64, i32, i32, f64, f64, P]
+    lib.oracle_score_grad_to_logits.argtypes = [P, P, i64, P]
     _lib = lib
     return lib
 
@@ -210,3 +220,53 @@ def order_key_array(v) -> np.ndarray:
     u = _c(v, np.float32).view(np.uint32)
     neg = (u & np.uint32(0x80000000)) != 0
     return np.where(neg, ~u, u | np.uint32(0x80000000)).astype(np.uint32)
+
+
+def bf16_round(v: float) -> int:
+    """16-bit pattern of the bf16 value nearest to the fp32 value v (ties to even)."""
+    return int(_load().oracle_bf16_round(ctypes.c_float(np.float32(v))))
+
+
+def bf16_key(b: int) -> int:
+    """Order-preserving 16-bit key of a bf16 pattern."""
+    return int(_load().oracle_bf16_key(ctypes.c_uint16(b)))
+
+
+def column_quantiles_bf16(z, alpha, m: int) -> np.ndarray:
+    """v_e = the (m+1)-th largest of bf16(Z[:,e] + alpha), as float (section 7.3, bf16 keys)."""
+    z = _c(z, np.float32)
+    N, E = z.shape
+    a = None if alpha is None else _c(alpha, np.float32)
+    v = np.empty((E,), dtype=np.float32)
+    _load().oracle_column_quantiles_bf16(_ptr(z), _ptr(a), N, E, int(m), _ptr(v))
+    return v
+
+
+def tanh_spec(x: float) -> float:
+    return float(_load().oracle_tanh_spec(float(x)))
+
+
+def lei_delta(counts, N: int, K: int, lam: float = 1e-5, tau: float = 1.0) -> np.ndarray:
+    """Per-expert Load-Error Injection increment of section 8 (fp32)."""
+    c = _c(counts, np.int32)
+    out = np.empty((c.shape[0],), dtype=np.float32)
+    _load().oracle_lei_delta(_ptr(c), int(N), c.shape[0], int(K), float(lam), float(tau), _ptr(out))
+    return out
+
+
+def lei_inject(counts, g, K: int, lam: float = 1e-5, tau: float = 1.0) -> np.ndarray:
+    """G[t, e] + delta_e for every token of the microbatch (section 8)."""
+    c = _c(counts, np.int32)
+    g = np.array(g, dtype=np.float32, copy=True, order="C")
+    N, E = g.shape
+    _load().oracle_lei_inject(_ptr(c), N, E, int(K), float(lam), float(tau), _ptr(g))
+    return g
+
+
+def score_grad_to_logits(z, gs) -> np.ndarray:
+    """dL/dZ = dL/dS * sigma(Z) (1 - sigma(Z)) (section 8, chain rule)."""
+    z = _c(z, np.float32)
+    gs = _c(gs, np.float32)
+    out = np.empty_like(z)
+    _load().oracle_score_grad_to_logits(_ptr(z), _ptr(gs), z.size, _ptr(out))
+    return out

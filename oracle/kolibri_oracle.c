@@ -299,6 +299,116 @@ uint64_t oracle_radix_select(const uint64_t *keys, const int64_t *chunk_sizes, i
     return prefix;
 }
 
+/* ------------------------------------- bf16 keys, as on the pages (7.3) */
+
+/* The bf16 value nearest to v (ties to the even mantissa), as its 16 bits.
+ * Inputs are finite (or infinite); an fp32 value past the largest bf16
+ * rounds to infinity, as IEEE rounding does. */
+uint16_t oracle_bf16_round(float v)
+{
+    uint32_t u = f32_to_bits(v);
+    uint32_t lsb = (u >> 16) & 1u;              /* last kept bit: ties go to even */
+    uint32_t r = u + 0x7fffu + lsb;            /* add just under half, or half */
+    return (uint16_t)(r >> 16);
+}
+
+/* Order-preserving 16-bit key of a bf16 pattern: the same total order as
+ * the fp32 key (negative: all 16 bits flipped; non-negative: sign bit set). */
+uint16_t oracle_bf16_key(uint16_t b)
+{
+    return (b & 0x8000u) ? (uint16_t)(~b & 0xffffu) : (uint16_t)(b | 0x8000u);
+}
+
+static int cmp_u16_desc(const void *pa, const void *pb)
+{
+    uint16_t a = *(const uint16_t *)pa, b = *(const uint16_t *)pb;
+    return (a < b) - (a > b);
+}
+
+/* [KPT] 7.3 with bfloat16 keys: per column, C = bf16(Z + alpha) (the fp32
+ * sum rounded once to bf16), and v_e = the (m+1)-th largest of C in the
+ * total order of the keys, returned as its float value.  The plain
+ * definition: round, sort, index. */
+void oracle_column_quantiles_bf16(const float *z, const float *alpha, int64_t N, int32_t E,
+                                  int64_t m, float *v)
+{
+#pragma omp parallel
+    {
+        uint16_t *col = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)N);
+#pragma omp for schedule(dynamic, 1)
+        for (int32_t e = 0; e < E; ++e) {
+            for (int64_t t = 0; t < N; ++t) {
+                float c = alpha ? z[t * E + e] + alpha[t] : z[t * E + e];
+                col[t] = oracle_bf16_key(oracle_bf16_round(c));
+            }
+            qsort(col, (size_t)N, sizeof(uint16_t), cmp_u16_desc);
+            uint16_t k = col[m];
+            uint16_t b = (k & 0x8000u) ? (uint16_t)(k & 0x7fffu) : (uint16_t)(~k & 0xffffu);
+            v[e] = (float)bf16_value(b);
+        }
+        free(col);
+    }
+}
+
+/* ------------------------------------- Load-Error Injection ([KPT] 8) */
+
+/* tanh from the gate's exp: tanh(x) = (1 - e^(-2x)) / (1 + e^(-2x)) for
+ * x >= 0, in fp64 IEEE operations (x is a norm, so never negative here). */
+double oracle_tanh_spec(double x)
+{
+    if (x > 350.0) return 1.0;                 /* e^(-2x) < 2^-1000: exactly 1 */
+    double t = oracle_exp_spec(-2.0 * x);
+    return (1.0 - t) / (1.0 + t);
+}
+
+/* The per-expert injection of [KPT] 8 for one microbatch of N tokens:
+ *   f_e = c_e / (K N / E),  rho_e = f_e - 1,  xi = max_e |rho_e| / tau,
+ *   delta_e = lambda * (tanh(xi) / xi) * rho_e   (the factor is 1 at xi = 0),
+ * all in fp64, delta rounded once to fp32.  Every token's score gradient
+ * then receives delta: G[t][e] += delta_e in fp32 (g may be NULL to get
+ * delta only). */
+void oracle_lei_delta(const int32_t *counts, int64_t N, int32_t E, int32_t K, double lambda,
+                      double tau, float *delta)
+{
+    double target = (double)K * (double)N / (double)E;
+    double xi = 0.0;
+    for (int32_t e = 0; e < E; ++e) {
+        double rho = (double)counts[e] / target - 1.0;
+        double a = rho < 0.0 ? -rho : rho;
+        if (a > xi) xi = a;
+    }
+    xi = xi / tau;
+    double factor = xi == 0.0 ? 1.0 : oracle_tanh_spec(xi) / xi;
+    for (int32_t e = 0; e < E; ++e) {
+        double rho = (double)counts[e] / target - 1.0;
+        delta[e] = (float)(lambda * factor * rho);
+    }
+}
+
+void oracle_lei_inject(const int32_t *counts, int64_t N, int32_t E, int32_t K, double lambda,
+                       double tau, float *g)
+{
+    float *delta = (float *)malloc(sizeof(float) * (size_t)E);
+    oracle_lei_delta(counts, N, E, K, lambda, tau, delta);
+    for (int64_t t = 0; t < N; ++t)
+        for (int32_t e = 0; e < E; ++e) g[t * E + e] = g[t * E + e] + delta[e];
+    free(delta);
+}
+
+/* The chain rule to the router logits ([KPT] 8, numerical check):
+ * dL/dZ = dL/dS * sigma(Z) (1 - sigma(Z)), with sigma in fp64 from the
+ * gate's exp, the product in fp64, rounded once to fp32. */
+void oracle_score_grad_to_logits(const float *z, const float *gs, int64_t n, float *gz)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        double s;                                 /* saturates as the gate does */
+        if (z[i] > 700.0f) s = 1.0;
+        else if (z[i] < -700.0f) s = 0.0;
+        else s = 1.0 / (1.0 + oracle_exp_spec(-(double)z[i]));
+        gz[i] = (float)((double)gs[i] * (s * (1.0 - s)));
+    }
+}
+
 /* ------------------------------------------------ measurements */
 
 /* MaxVio of [KPT] 6.2: max_e c_e / (K*N/E) - 1. */
