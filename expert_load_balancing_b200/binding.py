@@ -25,6 +25,7 @@ KOLIBRI_ERR_TIMEOUT = 5
 KOLIBRI_ERR_DEVICE = 6
 KOLIBRI_OP_PERMUTE = 1
 KOLIBRI_OP_EQB = 2
+KOLIBRI_OP_EQB_BF16 = 3
 
 # every symbol the header declares, with (restype, argtypes)
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
@@ -36,6 +37,13 @@ SIGNATURES = {
     "kolibri_router_forward_eqb": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _P,
                                                   _P, _P, _P, _SZ, _P]),
     "kolibri_router_topk": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P]),
+    "kolibri_eqb_update_bf16": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _SZ, _P]),
+    "kolibri_eqb_bf16_histogram": (ctypes.c_int, [_P, _P, _I64, _I32, _P, _P, _P]),
+    "kolibri_eqb_bf16_digit": (ctypes.c_int, [_P, _I32, _P, _P, _P]),
+    "kolibri_eqb_bf16_bias": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P]),
+    "kolibri_lei_inject": (ctypes.c_int, [_P, _I64, _I32, _I32, ctypes.c_double, ctypes.c_double, _P, _P]),
+    "kolibri_score_grad_to_logits": (ctypes.c_int, [_P, _P, _I64, _P, _P]),
+    "kolibri_intervention_rate": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P]),
     "kolibri_expert_permute": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P, _SZ, _P]),
     "kolibri_expert_permute_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _P, _P]),
     "kolibri_eqb_update": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _SZ, _P]),
@@ -311,3 +319,88 @@ def kolibri_route_and_balance(z: torch.Tensor, bias: torch.Tensor, K: int,
 def kolibri_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(load().kolibri_device_status(_stream(stream)))
+
+
+# ------------------------------------------------ bf16-key EQB, LEI, intervention
+
+def kolibri_eqb_update_bf16(z: torch.Tensor, alpha: torch.Tensor | None, bias: torch.Tensor, K: int,
+                            quantiles: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                            stream=None):
+    """EQB with bf16 keys (two 256-bin radix passes), in place on ``bias``.
+
+    Returns (bias, quantiles)."""
+    N, E = z.shape
+    _need(z, torch.float32, (N, E), "z")
+    _need(bias, torch.float32, (E,), "bias")
+    if alpha is not None:
+        _need(alpha, torch.float32, (N,), "alpha")
+    if ws is None:
+        ws = workspace(KOLIBRI_OP_EQB_BF16, N, E, K, z.device)
+    if quantiles is None:
+        quantiles = torch.empty((E,), dtype=torch.float32, device=z.device)
+    _check("kolibri_eqb_update_bf16",
+           load().kolibri_eqb_update_bf16(_ptr(z), _ptr(alpha), _ptr(bias), N, E, K, _ptr(quantiles),
+                                          _ptr(ws), ws.numel(), _stream(stream)))
+    return bias, quantiles
+
+
+def kolibri_eqb_bf16_histogram(z, alpha, prefix, hist, stream=None):
+    """Add this rank's bf16-key histogram (pass one: prefix None) into hist [E, 256] uint32."""
+    N, E = z.shape
+    _check("kolibri_eqb_bf16_histogram",
+           load().kolibri_eqb_bf16_histogram(_ptr(z), _ptr(alpha), N, E, _ptr(prefix), _ptr(hist),
+                                             _stream(stream)))
+    return hist
+
+
+def kolibri_eqb_bf16_digit(hist, rank, digit, stream=None):
+    E = hist.shape[0]
+    _check("kolibri_eqb_bf16_digit",
+           load().kolibri_eqb_bf16_digit(_ptr(hist), E, _ptr(rank), _ptr(digit), _stream(stream)))
+    return digit
+
+
+def kolibri_eqb_bf16_bias(d_hi, d_lo, bias, quantiles, stream=None):
+    E = bias.shape[0]
+    _check("kolibri_eqb_bf16_bias",
+           load().kolibri_eqb_bf16_bias(_ptr(d_hi), _ptr(d_lo), E, _ptr(bias), _ptr(quantiles),
+                                        _stream(stream)))
+    return bias, quantiles
+
+
+def kolibri_lei_inject(counts: torch.Tensor, g: torch.Tensor, K: int, lam: float = 1e-5,
+                       tau: float = 1.0, stream=None) -> torch.Tensor:
+    """Load-Error Injection on the score gradient g [N, E] (in place)."""
+    N, E = g.shape
+    _need(g, torch.float32, (N, E), "g")
+    _need(counts, torch.int32, (E,), "counts")
+    _check("kolibri_lei_inject",
+           load().kolibri_lei_inject(_ptr(counts), N, E, K, float(lam), float(tau), _ptr(g),
+                                     _stream(stream)))
+    return g
+
+
+def kolibri_score_grad_to_logits(z: torch.Tensor, gs: torch.Tensor, gz: torch.Tensor | None = None,
+                                 stream=None) -> torch.Tensor:
+    """dL/dZ = dL/dS * sigma(Z) (1 - sigma(Z))."""
+    _need(z, torch.float32, tuple(z.shape), "z")
+    _need(gs, torch.float32, tuple(z.shape), "gs")
+    if gz is None:
+        gz = torch.empty_like(z)
+    _check("kolibri_score_grad_to_logits",
+           load().kolibri_score_grad_to_logits(_ptr(z), _ptr(gs), z.numel(), _ptr(gz), _stream(stream)))
+    return gz
+
+
+def kolibri_intervention_rate(z: torch.Tensor, ids: torch.Tensor, stream=None):
+    """(rate [1] float64, overlaps [1] int64 as uint64 bits) on the device."""
+    N, E = z.shape
+    K = ids.shape[1]
+    _need(z, torch.float32, (N, E), "z")
+    _need(ids, torch.int32, (N, K), "ids")
+    rate = torch.empty((1,), dtype=torch.float64, device=z.device)
+    overlaps = torch.empty((1,), dtype=torch.int64, device=z.device)
+    _check("kolibri_intervention_rate",
+           load().kolibri_intervention_rate(_ptr(z), _ptr(ids), N, E, K, _ptr(rate), _ptr(overlaps),
+                                            _stream(stream)))
+    return rate, overlaps

@@ -57,6 +57,7 @@ size_t kolibri_workspace_bytes(int op, int64_t N, int32_t E, int32_t K) {
   if (check_ek(N, E, K) != KOLIBRI_OK) return 0;
   if (op == KOLIBRI_OP_PERMUTE) return permute_layout(N, E, K).total;
   if (op == KOLIBRI_OP_EQB) return eqb_layout(N, E, K).total;
+  if (op == KOLIBRI_OP_EQB_BF16) return eqb_bf16_ws_bytes(N, E, K);
   return 0;
 }
 
@@ -152,12 +153,74 @@ kolibri_status kolibri_route_and_balance(const float* z, float* bias, int64_t N,
                                         static_cast<cudaStream_t>(stream)));
 }
 
+kolibri_status kolibri_eqb_update_bf16(const float* z, const float* alpha, float* bias, int64_t N,
+                                       int32_t E, int32_t K, float* quantiles, void* ws,
+                                       size_t ws_bytes, void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!z || !bias || !ws) return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(z) || !aligned16(ws) || !aligned16(bias)) return KOLIBRI_ERR_INVALID_ARG;
+  if (ws_bytes < eqb_bf16_ws_bytes(N, E, K)) return KOLIBRI_ERR_WORKSPACE_TOO_SMALL;
+  return from_cuda(launch_eqb_bf16(z, alpha, bias, N, E, K, quantiles, ws,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_bf16_histogram(const float* z, const float* alpha, int64_t N, int32_t E,
+                                          const uint32_t* prefix, uint32_t* hist, void* stream) {
+  if (N < 1 || E < 4 || E > KOLIBRI_MAX_EXPERTS || (E % 4) != 0)
+    return N < 1 ? KOLIBRI_ERR_INVALID_ARG : KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (!z || !hist || !aligned16(z)) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_bf16_hist(z, alpha, N, E, prefix, hist, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_bf16_digit(const uint32_t* hist, int32_t E, int64_t* rank,
+                                      uint32_t* digit, void* stream) {
+  if (E < 1 || E > KOLIBRI_MAX_EXPERTS) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (!hist || !rank || !digit) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_bf16_digit(hist, E, rank, digit, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_bf16_bias(const uint32_t* digit_hi, const uint32_t* digit_lo, int32_t E,
+                                     float* bias, float* quantiles, void* stream) {
+  if (E < 1 || E > KOLIBRI_MAX_EXPERTS) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (!digit_hi || !digit_lo || !bias || !quantiles) return KOLIBRI_ERR_INVALID_ARG;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t err = launch_bf16_value(digit_hi, digit_lo, E, quantiles, s);
+  if (err != cudaSuccess) return KOLIBRI_ERR_CUDA;
+  return from_cuda(launch_bias_update(quantiles, E, bias, quantiles, s));
+}
+
+kolibri_status kolibri_lei_inject(const int32_t* counts, int64_t N, int32_t E, int32_t K,
+                                  double lambda, double tau, float* g, void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!counts || !g || !aligned16(g) || !(tau > 0.0)) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_lei_inject(counts, N, E, K, lambda, tau, g,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_score_grad_to_logits(const float* z, const float* gs, int64_t n, float* gz,
+                                            void* stream) {
+  if (n < 1 || !z || !gs || !gz) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_score_grad(z, gs, n, gz, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_intervention_rate(const float* z, const int32_t* ids, int64_t N, int32_t E,
+                                         int32_t K, double* rate, unsigned long long* overlaps,
+                                         void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!z || !ids || !rate || !overlaps || !aligned16(z)) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_intervention(z, ids, N, E, K, overlaps, rate,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 kolibri_status kolibri_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KOLIBRI_ERR_CUDA;
   const unsigned v = status_take_api() | status_take_eqb() | status_take_noalloc() |
                      status_take_permute() | status_take_route() | status_take_logits() |
-                     status_take_forward();
+                     status_take_forward() | status_take_balance();
   if (v & kStatusReadFailed) return KOLIBRI_ERR_CUDA;
   if (v & kStatusTimeout) return KOLIBRI_ERR_TIMEOUT;
   if (v & kStatusBadInput) return KOLIBRI_ERR_DEVICE;

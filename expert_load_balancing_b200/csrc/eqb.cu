@@ -374,6 +374,12 @@ cudaError_t eqb_end(const float* z, const float* alpha_used, float* bias, int64_
 
 }  // namespace
 
+cudaError_t launch_bias_update(const float* v, int32_t E, float* bias, float* quantiles,
+                               cudaStream_t s) {
+  bias_update_kernel<<<1, 512, 0, s>>>(v, E, bias, quantiles);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
                        int32_t K, float* quantiles, void* ws, cudaStream_t s) {
   const EqbBuffers b = eqb_buffers(N, E, K, ws);

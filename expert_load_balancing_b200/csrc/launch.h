@@ -90,6 +90,26 @@ cudaError_t launch_route_window_pass(const float* z, const float* bias, const fl
                                      uint32_t* above, uint32_t* cnt, uint32_t* cand, int64_t cap,
                                      cudaStream_t s);
 
+// beta = -v, centred (fp64 sum in ascending e, one rounding); quantiles (nullable) = v.
+cudaError_t launch_bias_update(const float* v, int32_t E, float* bias, float* quantiles,
+                               cudaStream_t s);
+
+// balance.cu: bf16-key EQB passes, Load-Error Injection, intervention rate.
+cudaError_t launch_bf16_hist(const float* z, const float* alpha, int64_t N, int32_t E,
+                             const uint32_t* prefix, uint32_t* hist, cudaStream_t s);
+cudaError_t launch_bf16_digit(const uint32_t* hist, int32_t E, int64_t* rank, uint32_t* digit,
+                              cudaStream_t s);
+cudaError_t launch_bf16_value(const uint32_t* d_hi, const uint32_t* d_lo, int32_t E, float* v,
+                              cudaStream_t s);
+size_t eqb_bf16_ws_bytes(int64_t N, int32_t E, int32_t K);
+cudaError_t launch_eqb_bf16(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
+                            int32_t K, float* quantiles, void* ws, cudaStream_t s);
+cudaError_t launch_lei_inject(const int32_t* counts, int64_t N, int32_t E, int32_t K, double lambda,
+                              double tau, float* g, cudaStream_t s);
+cudaError_t launch_score_grad(const float* z, const float* gs, int64_t n, float* gz, cudaStream_t s);
+cudaError_t launch_intervention(const float* z, const int32_t* ids, int64_t N, int32_t E, int32_t K,
+                                unsigned long long* total, double* rate, cudaStream_t s);
+
 int device_sm_count();
 
 // Read and clear the status word of one translation unit (see common.cuh).
@@ -100,5 +120,6 @@ unsigned status_take_permute();
 unsigned status_take_route();
 unsigned status_take_logits();
 unsigned status_take_forward();
+unsigned status_take_balance();
 
 }  // namespace kolibri

@@ -67,7 +67,8 @@ typedef enum kolibri_status {
 /* Operation selector for kolibri_workspace_bytes(). */
 enum {
     KOLIBRI_OP_PERMUTE = 1,
-    KOLIBRI_OP_EQB = 2
+    KOLIBRI_OP_EQB = 2,
+    KOLIBRI_OP_EQB_BF16 = 3
 };
 
 /* Limits.  E (experts) and K (top-K) must satisfy 1 <= K < E <= 512,
@@ -238,6 +239,89 @@ KOLIBRI_API kolibri_status kolibri_route_and_balance(const float *z, float *bias
                                                      int32_t E, int32_t K, int32_t *ids,
                                                      float *gates, float *alpha, float *quantiles,
                                                      void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * EQB with bfloat16 keys, as the pages run it ("Kolibri Pre-Training from
+ * Scratch" 7.3): per expert, C = bf16(Z_:,e + alpha) (the fp32 sum rounded
+ * once to bf16, ties to even), each value encoded as an order-preserving
+ * 16-bit key; v_e = the (m+1)-th largest C, m = floor(N K / E); then
+ * beta = -v, centred as in kolibri_eqb_update.  Rounding to bf16 is
+ * monotone, so v_e is exactly the bf16 rounding of kolibri_eqb_update's fp32
+ * quantile, and on one GPU that is how it is computed (one bracketed read of
+ * Z).  Across ranks the pages' two histogram passes below apply.
+ *   z [N, E] fp32, alpha [N] fp32 (NULL: alpha from bias, as
+ *   kolibri_eqb_update), bias [E] in/out, quantiles [E] out if not NULL,
+ *   ws: kolibri_workspace_bytes(KOLIBRI_OP_EQB_BF16, N, E, K) bytes.
+ * Errors as kolibri_eqb_update.
+ */
+KOLIBRI_API kolibri_status kolibri_eqb_update_bf16(const float *z, const float *alpha, float *bias,
+                                                   int64_t N, int32_t E, int32_t K,
+                                                   float *quantiles, void *ws, size_t ws_bytes,
+                                                   void *stream);
+
+/*
+ * The bf16-key EQB in pieces, for batches split over ranks (section 7.3:
+ * "the histograms are summed with one all-reduce"): each rank adds its
+ * histogram, the caller sums the histograms over ranks (an all-reduce of
+ * 256 E 32-bit counts, e.g. NCCL), and every rank then picks the same digit.
+ *   kolibri_eqb_bf16_histogram: ADDS this rank's counts into hist [E][256]
+ *     (uint32; zero it before each pass) for the keys of bf16(z + alpha)
+ *     (alpha NULL: of bf16(z)).  prefix NULL: pass one (bins of
+ *     the high byte of every key); else pass two (bins of the low byte of the
+ *     keys whose high byte is prefix[e]).  E % 4 == 0.
+ *   kolibri_eqb_bf16_digit: per expert, scans the summed hist from the top
+ *     bin to the one holding the rank[e]-th largest key (0-based; start with
+ *     rank[e] = m = floor(N_total K / E)); writes that bin to digit[e] and
+ *     subtracts the keys of the bins above it from rank[e].
+ *   kolibri_eqb_bf16_bias: v_e from the two digits (the key), written to
+ *     quantiles [E] (required), then bias = -v, centred.
+ * Sequence per update: zero h; histogram(NULL); all-reduce h; digit(h, rank,
+ * d_hi); zero h; histogram(d_hi); all-reduce h; digit(h, rank, d_lo);
+ * bias(d_hi, d_lo).  On one rank the all-reduces are skipped.
+ */
+KOLIBRI_API kolibri_status kolibri_eqb_bf16_histogram(const float *z, const float *alpha,
+                                                      int64_t N, int32_t E,
+                                                      const uint32_t *prefix, uint32_t *hist,
+                                                      void *stream);
+KOLIBRI_API kolibri_status kolibri_eqb_bf16_digit(const uint32_t *hist, int32_t E, int64_t *rank,
+                                                  uint32_t *digit, void *stream);
+KOLIBRI_API kolibri_status kolibri_eqb_bf16_bias(const uint32_t *digit_hi,
+                                                 const uint32_t *digit_lo, int32_t E,
+                                                 float *bias, float *quantiles, void *stream);
+
+/*
+ * Load-Error Injection ("Kolibri Pre-Training from Scratch" 8) on the score
+ * gradient of one microbatch of N tokens:
+ *   f_e = counts[e] / (K N / E), rho_e = f_e - 1, xi = max_e |rho_e| / tau,
+ *   delta_e = lambda (tanh(xi) / xi) rho_e (the factor is 1 at xi = 0), in
+ *   fp64, rounded once to fp32 (tanh from the gate's exp);
+ *   g[t][e] += delta_e for every token t and expert e (fp32).
+ * The pages use lambda = 1e-5 and tau = 1.  counts [E] int32 (e.g. from
+ * kolibri_expert_permute), g [N, E] fp32 in/out, 16-byte aligned.
+ */
+KOLIBRI_API kolibri_status kolibri_lei_inject(const int32_t *counts, int64_t N, int32_t E,
+                                              int32_t K, double lambda, double tau, float *g,
+                                              void *stream);
+
+/*
+ * The chain rule from the score gradient to the router logits (section 8,
+ * numerical check): gz[i] = gs[i] * sigma(z[i]) (1 - sigma(z[i])), sigma in
+ * fp64 from the gate's exp (saturating where the gate does), the product in
+ * fp64, rounded once to fp32.  n elements of each array.
+ */
+KOLIBRI_API kolibri_status kolibri_score_grad_to_logits(const float *z, const float *gs,
+                                                        int64_t n, float *gz, void *stream);
+
+/*
+ * Intervention rate ("Kolibri Pre-Training from Scratch" 9): the router's
+ * own choice I^u_t = TopK(Z_t,:) (no bias; ties to the lower id) against the
+ * routed ids; rate = 1 - (sum over tokens of |I^u_t and I_t|) / (N K).
+ * Random routing gives 1 - K/E.  rate [1] double and overlaps [1] (the
+ * summed overlap count) are device memory, written.
+ */
+KOLIBRI_API kolibri_status kolibri_intervention_rate(const float *z, const int32_t *ids, int64_t N,
+                                                     int32_t E, int32_t K, double *rate,
+                                                     unsigned long long *overlaps, void *stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word of

@@ -1,0 +1,142 @@
+"""EQB with bf16 keys over a batch split across ranks ("Kolibri Pre-Training
+from Scratch" 7.3): expert_load_balancing_b200.distributed sums the per-rank
+256-bin histograms with an all-reduce between the two passes.  Run here with
+two and three gloo ranks on the CPU; the three library calls are replaced by
+CPU stand-ins built from the oracle's bf16 rounding and key (the GPU kernels
+behind them are checked against the oracle in test_gpu_balance.py).  Every
+rank must end with the exact quantile of the union and the same bias; the
+pages' counter-example shows that averaging per-rank quantiles would not."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+class _CpuOps:
+    """The three per-rank calls on the CPU (test stand-ins)."""
+
+    def __init__(self, oracle):
+        self.o = oracle
+
+    def _keys(self, z, alpha):
+        zz = z.numpy()
+        a = np.zeros(zz.shape[0], np.float32) if alpha is None else alpha.numpy()
+        keys = np.empty(zz.shape, np.int64)
+        for t in range(zz.shape[0]):
+            for e in range(zz.shape[1]):
+                keys[t, e] = self.o.bf16_key(self.o.bf16_round(np.float32(zz[t, e] + a[t])))
+        return keys
+
+    def histogram(self, z, alpha, prefix, hist):
+        keys = self._keys(z, alpha)
+        for e in range(keys.shape[1]):
+            k = keys[:, e]
+            if prefix is None:
+                b = k >> 8
+            else:
+                b = (k & 0xff)[(k >> 8) == int(prefix[e])]
+            hist[e] += torch.from_numpy(np.bincount(b, minlength=256).astype(np.int32))
+        return hist
+
+    def digit(self, hist, rank, digit):
+        for e in range(hist.shape[0]):
+            r = int(rank[e])
+            above = 0
+            for b in range(255, -1, -1):
+                c = int(hist[e, b])
+                if above + c > r:
+                    digit[e] = b
+                    rank[e] = r - above
+                    break
+                above += c
+        return digit
+
+    def bias(self, d_hi, d_lo, bias, quantiles):
+        v = np.empty(bias.shape[0], np.float32)
+        for e in range(bias.shape[0]):
+            k = (int(d_hi[e]) << 8) | int(d_lo[e])
+            b = (k & 0x7fff) if (k & 0x8000) else (~k & 0xffff)
+            v[e] = np.frombuffer(np.uint32(b << 16).tobytes(), np.float32)[0]
+        quantiles.copy_(torch.from_numpy(v))
+        bias.copy_(torch.from_numpy(self.o.eqb_bias(v)))
+        return bias, quantiles
+
+
+def _worker(rank, world, port, z_parts, a_parts, K, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        from expert_load_balancing_b200 import distributed as D
+        z = torch.from_numpy(z_parts[rank])
+        a = torch.from_numpy(a_parts[rank])
+        n_total = sum(p.shape[0] for p in z_parts)
+        bias = torch.zeros(z.shape[1])
+        _, q = D.eqb_update_bf16_distributed(z, a, bias, K, n_total, ops=_CpuOps(oracle))
+        out[rank] = (q.numpy().copy(), bias.numpy().copy())
+    finally:
+        dist.destroy_process_group()
+
+
+def _run(z_parts, a_parts, K):
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    world = len(z_parts)
+    procs = [ctx.Process(target=_worker, args=(r, world, port, z_parts, a_parts, K, out))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(180)
+        assert p.exitcode == 0
+    return [out[r] for r in range(world)]
+
+
+def test_pages_counter_example_two_ranks(oracle_mod):
+    # 7.3: column e1 + alpha is (3.0, 1.5) on rank A and (0.5, 3.0) on rank B;
+    # the exact Q_2 of the union is 1.5, the average of local quantiles 1.0
+    za = np.array([[3.0, 0.0], [1.5, 0.0]], np.float32)
+    zb = np.array([[0.5, 0.0], [3.0, 0.0]], np.float32)
+    zero = np.zeros(2, np.float32)
+    res = _run([za, zb], [zero, zero], K=1)        # N = 4, E = 2, K = 1: m = 2
+    for q, b in res:
+        assert q[0] == np.float32(1.5)
+    np.testing.assert_array_equal(res[0][1], res[1][1])
+    local = [oracle_mod.column_quantiles_bf16(p, None, 1)[0] for p in (za, zb)]   # r = 1 each
+    assert np.mean(local) == 1.0 != 1.5
+
+
+def test_three_ranks_equal_the_union(oracle_mod):
+    rng = np.random.default_rng(0)
+    E, K = 6, 2
+    sizes = [17, 30, 9]
+    z_parts = [(rng.standard_normal((n, E)) * 2).astype(np.float32) for n in sizes]
+    z_parts[1][:, 2] = 0.5                         # ties across ranks
+    a_parts = [(rng.standard_normal(n) * 0.3).astype(np.float32) for n in sizes]
+    res = _run(z_parts, a_parts, K)
+    z = np.concatenate(z_parts)
+    a = np.concatenate(a_parts)
+    m = (z.shape[0] * K) // E
+    v = oracle_mod.column_quantiles_bf16(z, a, m)
+    for q, b in res:
+        np.testing.assert_array_equal(q, v)
+        np.testing.assert_array_equal(b, oracle_mod.eqb_bias(v))
