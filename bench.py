@@ -466,6 +466,128 @@ def run_reference(args, rank, world):
 
 # ---------------------------------------------------------------- main
 
+# ---------------------------------------------------------------- the balancing pieces
+
+PARTS = {
+    # name: (what, algorithmic bytes per token as a function of (E, K), note)
+    "eqb_bf16": ("EQB update with bf16 keys (one GPU: exact fp32 quantile, rounded)",
+                 lambda E, K: 4 * E + 4, "Z and alpha read once"),
+    "eqb_bf16_split": ("EQB with bf16 keys, the two histogram passes of the multi-rank form, one rank",
+                       lambda E, K: 8 * E + 8, "Z and alpha read twice"),
+    "lei": ("Load-Error Injection on the [N, E] score gradient",
+            lambda E, K: 8 * E, "G read and written"),
+    "score_grad": ("chain rule from the score gradient to the logits",
+                   lambda E, K: 12 * E, "Z and dS read, dZ written"),
+    "intervention": ("intervention rate (own top-K vs routed ids)",
+                     lambda E, K: 4 * E + 4 * K, "Z and ids read"),
+}
+
+
+def run_part(args):
+    """One of the balancing pieces on the kolibri_n1m shape, timed like the
+    step (CUDA events, clock samples), with its HBM roofline and the oracle
+    on a sample of the same data beside it."""
+    import oracle
+    from expert_load_balancing_b200 import distributed as D
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wl = workloads.WORKLOADS[args.workload]
+    N, d, E, K = wl.N, wl.d, wl.E, wl.K
+    step = RouterStep(wl, device)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        step.run(stream)
+    stream.synchronize()
+    g = torch.Generator(device=device)
+    g.manual_seed(7)
+    gs = torch.randn((N, E), generator=g, device=device) * 1e-4 if args.part in ("lei", "score_grad") else None
+    gz = torch.empty_like(gs) if gs is not None else None
+    ws16 = B.workspace(B.KOLIBRI_OP_EQB_BF16, N, E, K, device)
+    beta0 = step.beta.clone()
+    q = torch.empty((E,), dtype=torch.float32, device=device)
+
+    def once():
+        if args.part == "eqb_bf16":
+            step.beta.copy_(beta0)
+            B.kolibri_eqb_update_bf16(step.z, step.alpha, step.beta, K, q, ws16, stream=stream)
+        elif args.part == "eqb_bf16_split":
+            step.beta.copy_(beta0)
+            with torch.cuda.stream(stream):
+                D.eqb_update_bf16_distributed(step.z, step.alpha, step.beta, K, N, quantiles=q)
+        elif args.part == "lei":
+            B.kolibri_lei_inject(step.counts, gs, K, stream=stream)
+        elif args.part == "score_grad":
+            B.kolibri_score_grad_to_logits(step.z, gs, gz, stream=stream)
+        else:
+            B.kolibri_intervention_rate(step.z, step.ids, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            once()
+    stream.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0")
+    sampler.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            once()
+    t1.record(stream)
+    t1.synchronize()
+    clocks = sampler.stop()
+    st = B.kolibri_device_status(stream)
+    if st != B.KOLIBRI_OK:
+        raise RuntimeError(f"device status: {B.status_string(st)}")
+    ms = t0.elapsed_time(t1) / args.steps
+    what, bpt, note = PARTS[args.part]
+    peaks = _peaks()
+    bytes_ = bpt(E, K) * N
+    achieved = bytes_ / (ms * 1e-3) / 1e9
+    # the oracle on the first rows of the same data
+    n = min(N, 4096 if args.part in ("eqb_bf16", "eqb_bf16_split") else 2048)
+    zh = step.z[:n].cpu().numpy()
+    t = time.time()
+    if args.part in ("eqb_bf16", "eqb_bf16_split"):
+        oracle.column_quantiles_bf16(zh, step.alpha[:n].cpu().numpy(), (n * K) // E)
+    elif args.part == "lei":
+        oracle.lei_inject(step.counts.cpu().numpy(), gs[:n].cpu().numpy(), K)
+    elif args.part == "score_grad":
+        oracle.score_grad_to_logits(zh, gs[:n].cpu().numpy())
+    else:
+        ids_u, _, _ = oracle.select(zh, None, K)
+        oracle.intervention_rate(step.ids[:n].cpu().numpy(), ids_u)
+    reps = 1
+    cpu_s = time.time() - t
+    while cpu_s < 2.0:                 # repeat the sample to about 2 s of CPU work
+        t = time.time()
+        if args.part in ("eqb_bf16", "eqb_bf16_split"):
+            oracle.column_quantiles_bf16(zh, step.alpha[:n].cpu().numpy(), (n * K) // E)
+        elif args.part == "lei":
+            oracle.lei_inject(step.counts.cpu().numpy(), gs[:n].cpu().numpy(), K)
+        elif args.part == "score_grad":
+            oracle.score_grad_to_logits(zh, gs[:n].cpu().numpy())
+        else:
+            ids_u, _, _ = oracle.select(zh, None, K)
+            oracle.intervention_rate(step.ids[:n].cpu().numpy(), ids_u)
+        cpu_s += time.time() - t
+        reps += 1
+    return {
+        "metric": f"{what}: tokens/s at N=1M, E=384, K=6", "part": args.part,
+        "value": N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "fp32/f64",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "N": N, "E": E, "K": K, "inputs": "the step's own Z, ids, alpha, counts"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic": f"{bpt(E, K)} B per token ({note})",
+                     "peak_kind": f"HBM copy, of {peaks['source']}"},
+        "clocks": clocks,
+        "cpu_baseline": {"value": n * reps / cpu_s, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": f"first {n} tokens, {reps} times, {cpu_s:.1f} s"},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -479,6 +601,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--part", choices=sorted(PARTS), default=None,
+                    help="time one balancing piece instead of the routing step (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -486,6 +610,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.part and args.impl == "ours":
+        print(json.dumps(run_part(args)), flush=True)
+        return
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:
