@@ -588,6 +588,118 @@ def run_part(args):
     }
 
 
+# ---------------------------------------------------------------- decode
+
+def _decode_oracle(oracle, wl, layers, xs, ws, betas):
+    t = time.perf_counter()
+    for l in layers:
+        z = oracle.router_logits(xs[l], ws[l])
+        ids, _, _ = oracle.select(z, betas[l], wl.K)
+        oracle.permute(ids, wl.E)
+    return time.perf_counter() - t
+
+
+def run_decode(args):
+    """The decode sweep: per step, 50 layers of logits + top-K + gates + alpha
+    + counts + stable permutation for N in (1, 8, 64, 256) tokens, every layer
+    with its own x, W and beta.  Timed eager (one call per kernel per layer)
+    and as one CUDA graph per step; the forward alone and the logits alone are
+    timed the same way to show where the step goes.  The roofline is W
+    streamed once from HBM per layer (1.97 MB)."""
+    import oracle
+    oracle.build()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    B.load()
+    stream = torch.cuda.Stream(device)
+    peaks = _peaks()
+    per_n = {}
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0")
+    sampler.start()
+    for n_tok in workloads.DECODE_TOKENS:
+        wl = workloads.decode_workload(n_tok)
+        L, N, d, E, K = wl.layers, wl.N, wl.d, wl.E, wl.K
+        xs = [workloads.make_x(wl, l).to(device) for l in range(L)]
+        ws = [workloads.make_w(wl, l).to(device) for l in range(L)]
+        betas = [workloads.make_beta(wl, l).to(device) for l in range(L)]
+        z = torch.empty((N, E), dtype=torch.float32, device=device)
+        ids = torch.empty((N, K), dtype=torch.int32, device=device)
+        gates = torch.empty((N, K), dtype=torch.float32, device=device)
+        alpha = torch.empty((N,), dtype=torch.float32, device=device)
+        counts = torch.empty((E,), dtype=torch.int32, device=device)
+        offsets = torch.empty((E + 1,), dtype=torch.int64, device=device)
+        perm = torch.empty((N * K,), dtype=torch.int32, device=device)
+        inv = torch.empty((N * K,), dtype=torch.int32, device=device)
+        wsp = B.workspace(B.KOLIBRI_OP_PERMUTE, N, E, K, device)
+
+        def step(part="step"):
+            for l in range(L):
+                if part == "logits":
+                    B.kolibri_router_logits(xs[l], ws[l], z=z, stream=stream)
+                    continue
+                B.kolibri_router_forward(xs[l], ws[l], betas[l], K, z=z, ids=ids, gates=gates,
+                                         alpha=alpha, stream=stream)
+                if part == "step":
+                    B.kolibri_expert_permute(ids, E, wsp, counts, offsets, perm, inv, stream=stream)
+
+        def timed(fn, reps):
+            for _ in range(args.warmup):
+                fn()
+            stream.synchronize()
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            b.synchronize()
+            return a.elapsed_time(b) * 1e3 / reps
+
+        res = {}
+        with torch.cuda.stream(stream):
+            res["eager_us"] = timed(step, args.steps)
+            for part in ("step", "forward", "logits"):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    step(part)
+                res[f"graph_us" if part == "step" else f"graph_{part}_us"] = timed(gr.replay, args.steps)
+                del gr
+        st = B.kolibri_device_status(stream)
+        if st != B.KOLIBRI_OK:
+            raise RuntimeError(f"device status: {B.status_string(st)}")
+        res["graph_us_per_layer"] = res["graph_us"] / L
+        res["gpu_launches"] = 3 * L
+        res["w_bytes_per_step"] = 2 * E * d * L
+        per_n[str(n_tok)] = res
+    clocks = sampler.stop()
+    # the oracle: one whole decode step at N = 8 (all 50 layers)
+    wl = workloads.decode_workload(8)
+    xs = [workloads.bf16_bits(workloads.make_x(wl, l)) for l in range(wl.layers)]
+    wh = [workloads.bf16_bits(workloads.make_w(wl, l)) for l in range(wl.layers)]
+    bh = [workloads.make_beta(wl, l).numpy() for l in range(wl.layers)]
+    cpu_s = _decode_oracle(oracle, wl, range(wl.layers), xs, wh, bh)
+    top = per_n[str(workloads.DECODE_TOKENS[-1])]
+    w_bytes = top["w_bytes_per_step"]
+    achieved = w_bytes / (top["graph_us"] * 1e-6) / 1e9
+    return {
+        "metric": "decode step latency, 50 layers of logits + top-K + gates + permutation "
+                  f"(d=2560, E=384, K=6), N={workloads.DECODE_TOKENS[-1]} tokens, CUDA graph",
+        "part": "decode", "value": top["graph_us"], "unit": "us/step", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": top["graph_us"] * 1e-3,
+        "higher_is_better": False, "dtype": "bf16 in, fp32 accumulate", "data": "synthetic",
+        "config": {"workload": "decode", "layers": workloads.DECODE_LAYERS,
+                   "tokens": list(workloads.DECODE_TOKENS), "d": 2560, "E": 384, "K": 6,
+                   "inputs": "distinct x, W, beta per layer (98 MB of W per step, under L2 size)"},
+        "per_n": per_n,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "algorithmic": "W read once per layer: 2 E d bytes",
+                     "peak_kind": f"HBM copy, of {peaks['source']}"},
+        "clocks": clocks,
+        "cpu_baseline": {"value": cpu_s * 1e6, "unit": "us/step", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": "one whole step at N=8 (50 layers)"},
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -601,6 +713,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--decode", action="store_true",
+                    help="time the decode sweep (50 layers, N = 1, 8, 64, 256; one GPU)")
     ap.add_argument("--part", choices=sorted(PARTS), default=None,
                     help="time one balancing piece instead of the routing step (one GPU)")
     args = ap.parse_args()
@@ -610,6 +724,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.decode and args.impl == "ours":
+        print(json.dumps(run_decode(args)), flush=True)
+        return
     if args.part and args.impl == "ours":
         print(json.dumps(run_part(args)), flush=True)
         return

@@ -68,7 +68,9 @@ kolibri_status kolibri_router_logits(const void* x, const void* w, float* z, int
   if (N < 1 || d < 1 || E < 1) return KOLIBRI_ERR_INVALID_ARG;
   if (d % 64 != 0 || E % 16 != 0 || E > KOLIBRI_MAX_EXPERTS) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
   if (N >= (static_cast<int64_t>(1) << 31)) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
-  return from_cuda(launch_router_logits(x, w, z, N, d, E, static_cast<cudaStream_t>(stream)));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (router_small_preferred(N)) return from_cuda(launch_router_logits_small(x, w, z, N, d, E, s));
+  return from_cuda(launch_router_logits(x, w, z, N, d, E, s));
 }
 
 kolibri_status kolibri_router_forward(const void* x, const void* w, const float* bias, float* z,
@@ -220,7 +222,7 @@ kolibri_status kolibri_device_status(void* stream) {
     return KOLIBRI_ERR_CUDA;
   const unsigned v = status_take_api() | status_take_eqb() | status_take_noalloc() |
                      status_take_permute() | status_take_route() | status_take_logits() |
-                     status_take_forward() | status_take_balance();
+                     status_take_forward() | status_take_balance() | status_take_small();
   if (v & kStatusReadFailed) return KOLIBRI_ERR_CUDA;
   if (v & kStatusTimeout) return KOLIBRI_ERR_TIMEOUT;
   if (v & kStatusBadInput) return KOLIBRI_ERR_DEVICE;

@@ -43,6 +43,12 @@ PermuteLayout permute_layout(int64_t N, int32_t E, int32_t K);
 cudaError_t launch_router_logits(const void* x, const void* w, float* z, int64_t N, int32_t d,
                                  int32_t E, cudaStream_t s);
 
+// Small batches (decode): logits by router_small.cu instead of the pair GEMM.
+constexpr int64_t kSmallTokenLimit = 1024;
+bool router_small_preferred(int64_t N);
+cudaError_t launch_router_logits_small(const void* x, const void* w, float* z, int64_t N, int32_t d,
+                                       int32_t E, cudaStream_t s);
+
 // Fused logits + selection (router_forward.cu).  Returns cudaErrorNotSupported
 // for shapes it does not cover; the caller then runs logits and top-K apart.
 // Rows it could not finish carry a NaN alpha; launch_select_fixup completes them.
@@ -121,5 +127,6 @@ unsigned status_take_route();
 unsigned status_take_logits();
 unsigned status_take_forward();
 unsigned status_take_balance();
+unsigned status_take_small();
 
 }  // namespace kolibri

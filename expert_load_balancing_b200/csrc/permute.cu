@@ -128,22 +128,6 @@ __global__ void __launch_bounds__(kPermThreads) chunk_scan_kernel(
   if (threadIdx.x == 0) *ticket = 0u;  // ready for the next call
 }
 
-__device__ __forceinline__ void scatter_round(int32_t e, int64_t j, int lane, uint32_t* cursor,
-                                              int32_t* __restrict__ perm,
-                                              int32_t* __restrict__ inv) {
-  const unsigned lt = (1u << lane) - 1u;
-  unsigned peers = __match_any_sync(0xffffffffu, e);
-  if (e >= 0) {
-    unsigned rank = __popc(peers & lt);
-    uint32_t pos = cursor[e] + rank;
-    perm[pos] = static_cast<int32_t>(j);
-    if (inv) inv[j] = static_cast<int32_t>(pos);
-  }
-  __syncwarp();
-  if (e >= 0 && (peers & lt) == 0u) cursor[e] += __popc(peers);
-  __syncwarp();
-}
-
 // Exclusive prefix of n <= 2 * kPermThreads values held two per thread
 // (thread t owns v0 = element 2t, v1 = element 2t+1); returns the prefix of
 // element 2t and writes the grand total to *total.
@@ -254,40 +238,89 @@ __global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
   }
 }
 
-// All three steps in one block (small N*K).
-__global__ void __launch_bounds__(1024) permute_single_kernel(
+// All three steps in one block (small N*K, decode batches).  Each of the 16
+// warps ranks a contiguous segment of slots (stable inside the segment: the
+// lanes of a round are grouped by expert with __match_any_sync and a per-warp
+// counter per expert carries the rounds); one thread per expert turns the
+// per-warp counts into starts; a block scan gives the offsets.  Slot order is
+// segment order, then round order, then lane order, which is j order.
+constexpr int kSingleThreads = 512;
+constexpr int kSingleWarps = kSingleThreads / kWarp;
+constexpr int kSingleRounds = static_cast<int>(kSingleMax / (kSingleWarps * 32));   // 8
+static_assert(kSingleMax % (kSingleWarps * 32) == 0, "segments of whole rounds");
+static_assert(KOLIBRI_MAX_EXPERTS <= kSingleThreads, "one thread per expert");
+
+__global__ void __launch_bounds__(kSingleThreads) permute_single_kernel(
     const int32_t* __restrict__ ids, int64_t NK, int E, int32_t* __restrict__ counts,
     int64_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
-  __shared__ uint32_t hist[KOLIBRI_MAX_EXPERTS];
-  __shared__ uint32_t cursor[KOLIBRI_MAX_EXPERTS];
-  const int tid = threadIdx.x, lane = tid & 31;
-  for (int e = tid; e < E; e += blockDim.x) hist[e] = 0u;
-  __syncthreads();
+  __shared__ uint32_t cnt_w[kSingleWarps][KOLIBRI_MAX_EXPERTS];   // per-warp counts, then starts
+  __shared__ uint32_t start_e[KOLIBRI_MAX_EXPERTS];
+  __shared__ uint32_t warp_sums[kSingleWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t* my_cnt = cnt_w[warp];
+  for (int e = lane; e < E; e += 32) my_cnt[e] = 0u;
+  __syncwarp();
+  // ---- segment ranks: this warp's slots [w0, w0 + 32 * rounds)
+  const int64_t seg = ((NK + kSingleWarps * 32 - 1) / (kSingleWarps * 32)) * 32;
+  const int64_t w0 = static_cast<int64_t>(warp) * seg;
+  int32_t ex[kSingleRounds];
+  uint32_t rk[kSingleRounds];
   bool bad = false;
-  for (int64_t j = tid; j < NK; j += blockDim.x) {
-    int32_t x = __ldg(ids + j);
-    if (x >= 0 && x < E) atomicAdd(&hist[x], 1u);
-    else bad = true;
+#pragma unroll
+  for (int r = 0; r < kSingleRounds; ++r) {
+    const int64_t j = w0 + r * 32 + lane;
+    const bool in = r * 32 < seg && j < NK;
+    int32_t x = in ? __ldg(ids + j) : -1;
+    if (in && !(x >= 0 && x < E)) bad = true;
+    x = (x >= 0 && x < E) ? x : -1;
+    ex[r] = x;
+    const unsigned peers = __match_any_sync(0xffffffffu, x);
+    const uint32_t below = __popc(peers & lt);
+    rk[r] = (x >= 0) ? my_cnt[x] + below : 0u;
+    __syncwarp();
+    if (x >= 0 && below == 0u) my_cnt[x] += __popc(peers);
+    __syncwarp();
   }
   if (bad) raise_status(kStatusBadInput);
   __syncthreads();
-  if (tid == 0) {
-    int64_t run = 0;
-    for (int e = 0; e < E; ++e) {
-      offsets[e] = run;
-      counts[e] = static_cast<int32_t>(hist[e]);
-      cursor[e] = static_cast<uint32_t>(run);
-      run += hist[e];
+  // ---- per expert: warp starts inside the expert's run, and its total
+  uint32_t tot = 0u;
+  if (tid < E) {
+    for (int w = 0; w < kSingleWarps; ++w) {
+      const uint32_t c = cnt_w[w][tid];
+      cnt_w[w][tid] = tot;
+      tot += c;
     }
-    offsets[E] = run;
+  }
+  // ---- exclusive scan of the totals over experts (E <= kSingleThreads)
+  uint32_t incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  uint32_t wbase = 0;
+  for (int w = 0; w < warp; ++w) wbase += warp_sums[w];
+  const uint32_t excl = wbase + incl - tot;
+  if (tid < E) {
+    start_e[tid] = excl;
+    offsets[tid] = excl;
+    counts[tid] = static_cast<int32_t>(tot);
+    if (tid == E - 1) offsets[E] = excl + tot;
   }
   __syncthreads();
-  if (tid < 32) {
-    for (int64_t base = 0; base < NK; base += 32) {
-      int64_t j = base + lane;
-      int32_t x = j < NK ? __ldg(ids + j) : -1;
-      x = (x >= 0 && x < E) ? x : -1;
-      scatter_round(x, j, lane, cursor, perm, inv);
+  // ---- positions
+#pragma unroll
+  for (int r = 0; r < kSingleRounds; ++r) {
+    const int32_t e = ex[r];
+    if (e >= 0) {
+      const int64_t j = w0 + r * 32 + lane;
+      const uint32_t pos = start_e[e] + my_cnt[e] + rk[r];
+      perm[pos] = static_cast<int32_t>(j);
+      if (inv) inv[j] = static_cast<int32_t>(pos);
     }
   }
 }
@@ -322,7 +355,7 @@ cudaError_t launch_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K, 
   const int64_t NK = N * K;
   const PermuteLayout L = permute_layout(N, E, K);
   if (L.single_cta) {
-    permute_single_kernel<<<1, 1024, 0, s>>>(ids, NK, E, counts, offsets, perm, inv);
+    permute_single_kernel<<<1, kSingleThreads, 0, s>>>(ids, NK, E, counts, offsets, perm, inv);
     return cudaGetLastError();
   }
   char* base = static_cast<char*>(ws);

@@ -21,7 +21,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / kWarp;
-constexpr int kRowsPerWarp = 32;     // rows per warp between gather flushes
+constexpr int kRowsPerWarp = 32;     // most rows per warp between gather flushes
 constexpr int kStageSlots = 16;      // staged bracket keys per expert per block
 
 struct RouteParams {
@@ -29,6 +29,7 @@ struct RouteParams {
   const float* beta;  // may be null
   int64_t N;
   int E, K;
+  int rows_per_warp;  // 1 .. kRowsPerWarp: small batches spread one row per warp
   // selection outputs
   int32_t* ids;
   float* gates;
@@ -131,11 +132,11 @@ __global__ void __launch_bounds__(kThreads, kAlphaIn ? 4 : 3) route_rows_kernel(
   for (int j = 0; j < V; ++j) valid |= (static_cast<int>(slot_expert(lane, j)) < E) ? (1u << j) : 0u;
   int gate_n = 0;
 
-  const int64_t rows_per_block = static_cast<int64_t>(kWarps) * kRowsPerWarp;
+  const int64_t rows_per_block = static_cast<int64_t>(kWarps) * p.rows_per_warp;
   for (int64_t base = static_cast<int64_t>(blockIdx.x) * rows_per_block; base < p.N;
        base += static_cast<int64_t>(gridDim.x) * rows_per_block) {
-    const int64_t r0 = base + static_cast<int64_t>(warp) * kRowsPerWarp;
-    const int64_t r1 = (r0 + kRowsPerWarp < p.N) ? r0 + kRowsPerWarp : p.N;
+    const int64_t r0 = base + static_cast<int64_t>(warp) * p.rows_per_warp;
+    const int64_t r1 = (r0 + p.rows_per_warp < p.N) ? r0 + p.rows_per_warp : p.N;
     // per-lane counts of keys above the bracket, one byte per slot (<= 32 rows per batch)
     uint32_t above_b[kWindow ? Q : 1];
     if constexpr (kWindow) {
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(kThreads) select_fixup_kernel(
 }
 
 template <int Q, bool kFull, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
-cudaError_t launch_rows(const RouteParams& p, cudaStream_t s) {
+cudaError_t launch_rows(RouteParams p, cudaStream_t s) {
   auto kern = route_rows_kernel<Q, kFull, kBias, kRoute, kAlphaOut, kAlphaIn, kWindow>;
   const SmemLayout L = smem_layout<Q, kWindow>(p.E);
   cudaError_t err =
@@ -362,9 +363,16 @@ cudaError_t launch_rows(const RouteParams& p, cudaStream_t s) {
   err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, L.total);
   if (err != cudaSuccess) return err;
   if (per_sm < 1) per_sm = 1;
-  const int64_t rows_per_block = static_cast<int64_t>(kWarps) * kRowsPerWarp;
-  int64_t blocks = (p.N + rows_per_block - 1) / rows_per_block;
+  // each warp walks its rows one after another, so a batch that does not
+  // fill the resident warps gets fewer rows per warp (one, for decode sizes)
   const int64_t resident = static_cast<int64_t>(device_sm_count()) * per_sm;
+  const int64_t warps = resident * kWarps;
+  int64_t rpw = (p.N + warps - 1) / warps;
+  if (rpw < 1) rpw = 1;
+  if (rpw > kRowsPerWarp) rpw = kRowsPerWarp;
+  p.rows_per_warp = static_cast<int>(rpw);
+  const int64_t rows_per_block = static_cast<int64_t>(kWarps) * rpw;
+  int64_t blocks = (p.N + rows_per_block - 1) / rows_per_block;
   if (blocks > resident) blocks = resident;
   kern<<<static_cast<unsigned>(blocks), kThreads, L.total, s>>>(p);
   return cudaGetLastError();

@@ -1,5 +1,8 @@
-"""GPU router logits (tcgen05 GEMM) against the oracle's fp64 sums:
-|dZ| <= 1e-3 max(1, |Z|), plus closed-form special cases that must be exact."""
+"""GPU router logits against the oracle's fp64 sums: |dZ| <= 1e-3 max(1, |Z|),
+plus closed-form special cases that must be exact.  Batches of up to 1024
+tokens take the clustered split-d kernel (its tile changes at 16, 32, 512
+tokens and with d a multiple of 128 or not); larger ones the tcgen05 pair
+GEMM."""
 import numpy as np
 import pytest
 import torch
@@ -34,6 +37,31 @@ def test_logits_random(oracle_mod, N, d, E):
     err = assert_logits_close(z, zr)
     assert err < 1e-4, err     # fp32 accumulation of exact bf16 products
     check_status()
+
+
+@pytest.mark.parametrize("N", [1, 15, 16, 17, 32, 33, 64, 65, 511, 512, 513, 1024, 1025])
+@pytest.mark.parametrize("d,E", [(2560, 384), (320, 400), (1024, 48)])
+def test_logits_small_batches(oracle_mod, N, d, E):
+    wl = workloads.Workload("t", N, d, E, 4, offsets="collapsed8")
+    x = workloads.make_x(wl)
+    w = workloads.make_w(wl)
+    z = _run(x, w)
+    zr = oracle_mod.router_logits(workloads.bf16_bits(x), workloads.bf16_bits(w))
+    err = assert_logits_close(z, zr)
+    assert err < 1e-4, err
+    # the split sums are added in a fixed order: a second call repeats every bit
+    np.testing.assert_array_equal(_run(x, w), z)
+    check_status()
+
+
+def test_logits_small_constant_rows_exact():
+    d, E = 2560, 384
+    for N in (3, 40, 300):
+        x = torch.full((N, d), 0.5, dtype=torch.bfloat16)
+        w = ((torch.arange(E, dtype=torch.float32) % 7 + 1) / 16).repeat(d, 1).T.contiguous()
+        z = _run(x, w.to(torch.bfloat16))
+        expect = np.float32(d * 0.5) * ((np.arange(E) % 7 + 1) / 16).astype(np.float32)
+        np.testing.assert_array_equal(z, np.tile(expect, (N, 1)))
 
 
 def test_logits_one_hot_exact(oracle_mod):

@@ -132,7 +132,10 @@ def test_gates_unchanged_by_bias():
 # ------------------------------------------------ permutation, bit-exact
 
 @pytest.mark.parametrize("N,E,K", [(1, 384, 6), (256, 384, 6), (683, 384, 6), (5000, 384, 6),
-                                   (40000, 128, 8), (12345, 16, 3)])
+                                   (40000, 128, 8), (12345, 16, 3),
+                                   # one block up to N*K = 4096: its edges
+                                   (512, 512, 8), (4096, 16, 1), (1, 512, 16), (13, 48, 5),
+                                   (4097, 16, 1)])
 def test_permute(oracle_mod, N, E, K):
     rng = np.random.default_rng(N)
     ids = np.stack([rng.choice(E, size=K, replace=False) for _ in range(N)]).astype(np.int32)
@@ -145,6 +148,15 @@ def test_permute_skewed(oracle_mod):
     N, E, K = 30000, 384, 6
     ids = np.tile(np.array([5, 17, 0, 383, 200, 6], np.int32), (N, 1))
     _permute_case(oracle_mod, ids, E)
+
+
+def test_permute_skewed_one_block(oracle_mod):
+    # a decode batch on the same experts: one expert's run spans every warp's segment
+    N, E, K = 600, 384, 6
+    ids = np.tile(np.array([5, 17, 0, 383, 200, 6], np.int32), (N, 1))
+    ids[::7, 2] = 1
+    _permute_case(oracle_mod, ids, E)
+    check_status()
 
 
 def test_permute_bad_id_sets_device_status():
