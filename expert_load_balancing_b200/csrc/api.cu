@@ -83,7 +83,7 @@ kolibri_status kolibri_router_forward(const void* x, const void* w, const float*
     return KOLIBRI_ERR_INVALID_ARG;
   if (d < 1) return KOLIBRI_ERR_INVALID_ARG;
   if (d % 64 != 0 || E % 16 != 0) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
-  return from_cuda(router_forward_any(x, w, bias, z, N, d, E, K, ids, gates, alpha,
+  return from_cuda(router_forward_by_size(x, w, bias, z, N, d, E, K, ids, gates, alpha,
                                       static_cast<cudaStream_t>(stream)));
 }
 

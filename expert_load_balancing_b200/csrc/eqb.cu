@@ -407,7 +407,7 @@ cudaError_t launch_forward_eqb(const void* x, const void* w, float* bias, float*
                                float* alpha, float* quantiles, void* ws, cudaStream_t s) {
   const EqbBuffers b = eqb_buffers(N, E, K, ws);
   float* alpha_out = alpha ? alpha : b.alpha_ws;
-  const cudaError_t err = router_forward_any(x, w, bias, z, N, d, E, K, ids, gates, alpha_out, s);
+  const cudaError_t err = router_forward_by_size(x, w, bias, z, N, d, E, K, ids, gates, alpha_out, s);
   if (err != cudaSuccess) return err;
   return launch_eqb(z, alpha_out, bias, N, E, K, quantiles, ws, s);
 }

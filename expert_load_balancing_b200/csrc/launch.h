@@ -75,6 +75,12 @@ cudaError_t router_forward_any(const void* x, const void* w, const float* bias, 
                                int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
                                float* gates, float* alpha, cudaStream_t s);
 
+// The forward by batch size: small batches (router_small_preferred) take the
+// small logits kernel and the row kernel, the rest router_forward_any.
+cudaError_t router_forward_by_size(const void* x, const void* w, const float* bias, float* z,
+                                   int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                   float* gates, float* alpha, cudaStream_t s);
+
 cudaError_t launch_forward_eqb(const void* x, const void* w, float* bias, float* z, int64_t N,
                                int32_t d, int32_t E, int32_t K, int32_t* ids, float* gates,
                                float* alpha, float* quantiles, void* ws, cudaStream_t s);

@@ -18,6 +18,7 @@
 // Small inputs (decode) run the same steps inside one block.
 #include "launch.h"
 #include "common.cuh"
+#include "pdl.cuh"
 
 namespace kolibri {
 
@@ -261,6 +262,8 @@ __global__ void __launch_bounds__(kSingleThreads) permute_single_kernel(
   uint32_t* my_cnt = cnt_w[warp];
   for (int e = lane; e < E; e += 32) my_cnt[e] = 0u;
   __syncwarp();
+  pdl_wait();       // ids come from the kernel before this one
+  pdl_trigger();
   // ---- segment ranks: this warp's slots [w0, w0 + 32 * rounds)
   const int64_t seg = ((NK + kSingleWarps * 32 - 1) / (kSingleWarps * 32)) * 32;
   const int64_t w0 = static_cast<int64_t>(warp) * seg;
@@ -355,8 +358,8 @@ cudaError_t launch_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K, 
   const int64_t NK = N * K;
   const PermuteLayout L = permute_layout(N, E, K);
   if (L.single_cta) {
-    permute_single_kernel<<<1, kSingleThreads, 0, s>>>(ids, NK, E, counts, offsets, perm, inv);
-    return cudaGetLastError();
+    return launch_pdl(permute_single_kernel, dim3(1), dim3(kSingleThreads), 0, s, dim3(0, 0, 0), ids,
+                      NK, E, counts, offsets, perm, inv);
   }
   char* base = static_cast<char*>(ws);
   uint32_t* tile_counts = reinterpret_cast<uint32_t*>(base + L.off_chunk_counts);

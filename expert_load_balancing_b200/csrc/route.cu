@@ -14,6 +14,7 @@
 // one global atomic per expert.
 #include "launch.h"
 #include "route.cuh"
+#include "pdl.cuh"
 
 namespace kolibri {
 
@@ -115,6 +116,8 @@ __global__ void __launch_bounds__(kThreads, kAlphaIn ? 4 : 3) route_rows_kernel(
   uint32_t* stage_n = reinterpret_cast<uint32_t*>(smem + L.off_stage_n);
   uint32_t* stage = reinterpret_cast<uint32_t*>(smem + L.off_stage);
   WarpScratch<Q>& ws = reinterpret_cast<WarpScratch<Q>*>(smem + L.off_warp)[warp];
+  pdl_wait();       // Z comes from the kernel before this one
+  pdl_trigger();
 
   for (int e = threadIdx.x; e < E; e += kThreads) {
     if constexpr (kBias) beta_s[e] = p.beta[e];
@@ -374,8 +377,7 @@ cudaError_t launch_rows(RouteParams p, cudaStream_t s) {
   const int64_t rows_per_block = static_cast<int64_t>(kWarps) * rpw;
   int64_t blocks = (p.N + rows_per_block - 1) / rows_per_block;
   if (blocks > resident) blocks = resident;
-  kern<<<static_cast<unsigned>(blocks), kThreads, L.total, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), L.total, s, dim3(0, 0, 0), p);
 }
 
 // route: write ids/gates; alpha_out: write alpha; alpha_in: read alpha

@@ -544,12 +544,6 @@ cudaError_t launch_router_forward(const void* x, const void* w, const float* bia
 cudaError_t router_forward_any(const void* x, const void* w, const float* bias, float* z,
                                int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
                                float* gates, float* alpha, cudaStream_t s) {
-  if (router_small_preferred(N)) {
-    // decode batches: the many-CTA small GEMM, then the row selection
-    const cudaError_t err = launch_router_logits_small(x, w, z, N, d, E, s);
-    if (err != cudaSuccess) return err;
-    return launch_topk(z, bias, N, E, K, ids, gates, alpha, s);
-  }
   if (router_forward_supported(E, K)) {
     const cudaError_t err = launch_router_forward(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
     if (err == cudaSuccess) return launch_select_fixup(z, bias, N, E, K, ids, gates, alpha, s);

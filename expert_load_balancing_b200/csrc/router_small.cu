@@ -20,6 +20,7 @@
 
 #include "launch.h"
 #include "common.cuh"
+#include "pdl.cuh"
 
 namespace kolibri {
 
@@ -103,6 +104,8 @@ __global__ void __launch_bounds__(32 * kWarps) small_logits_kernel(
   const int k0 = static_cast<int>(rank) * ks;
   const int e0 = blockIdx.x * kX;
   const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kTok;
+  pdl_wait();       // x may come from the kernel before this one
+  pdl_trigger();
 
   // every load at once: one round trip per CTA
   const int pieces = ks / 8;                         // 16-byte pieces per row
@@ -185,21 +188,8 @@ cudaError_t launch_small(const __nv_bfloat16* x, const __nv_bfloat16* w, float* 
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = kS;
-  cfg.gridDim = dim3(static_cast<unsigned>((E + kX - 1) / kX), static_cast<unsigned>(ty), kS);
-  cfg.blockDim = dim3(32 * kWarps, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kern, x, w, z, N, d, E);
-  if (err != cudaSuccess) return err;
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>((E + kX - 1) / kX), static_cast<unsigned>(ty), kS),
+                    dim3(32 * kWarps), smem, s, dim3(1, 1, kS), x, w, z, N, d, E);
 }
 
 }  // namespace
@@ -223,6 +213,18 @@ cudaError_t launch_router_logits_small(const void* x, const void* w, float* z, i
   if (N <= 32) return launch_small<2, 16, 8>(xb, wb, z, N, d, E, s);
   if (N <= 512) return launch_small<4, 32, 8>(xb, wb, z, N, d, E, s);
   return launch_small<4, 64, 8>(xb, wb, z, N, d, E, s);
+}
+
+cudaError_t router_forward_by_size(const void* x, const void* w, const float* bias, float* z,
+                                   int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                   float* gates, float* alpha, cudaStream_t s) {
+  if (router_small_preferred(N)) {
+    // decode batches: the clustered logits kernel, then one row per warp
+    const cudaError_t err = launch_router_logits_small(x, w, z, N, d, E, s);
+    if (err != cudaSuccess) return err;
+    return launch_topk(z, bias, N, E, K, ids, gates, alpha, s);
+  }
+  return router_forward_any(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
 }
 
 KOLIBRI_DEFINE_STATUS_TAKE(status_take_small)
