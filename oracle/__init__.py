@@ -77,6 +77,11 @@ def _load():
     lib.oracle_lei_delta.argtypes = [P, i64, i32, i32, f64, f64, P]
     lib.oracle_lei_inject.argtypes = [P, i64, i32, i32, f64, f64, P]
     lib.oracle_score_grad_to_logits.argtypes = [P, P, i64, P]
+    lib.oracle_bf16_round_f64.argtypes = [f64]
+    lib.oracle_bf16_round_f64.restype = ctypes.c_uint16
+    lib.oracle_silu_spec.argtypes = [f64]
+    lib.oracle_silu_spec.restype = f64
+    lib.oracle_expert_ffn.argtypes = [P, P, P, P, P, P, P, i64, i32, i32, i32, i32, P, P, P, P]
     _lib = lib
     return lib
 
@@ -270,3 +275,52 @@ def score_grad_to_logits(z, gs) -> np.ndarray:
     out = np.empty_like(z)
     _load().oracle_score_grad_to_logits(_ptr(z), _ptr(gs), z.size, _ptr(out))
     return out
+
+
+def bf16_round_f64(v: float) -> int:
+    """bf16 bits of the nearest bf16 to the fp64 value v (one rounding)."""
+    return int(_load().oracle_bf16_round_f64(float(v)))
+
+
+def silu_spec(g: float) -> float:
+    """SiLU(g) = g * sigma(g) in fp64 with the gate's exp."""
+    return float(_load().oracle_silu_spec(float(g)))
+
+
+def expert_ffn(x_bf16_bits, ids, gates, wgu_bf16_bits, wd_bf16_bits, wgu_s_bf16_bits=None,
+               wd_s_bf16_bits=None, want_h=False):
+    """The MoE layer output of section 6.1 with SwiGLU experts.
+
+    x [N,d], wgu [E,2F,d] (gate rows then up rows), wd [E,d,F], optional
+    shared expert wgu_s [2F,d], wd_s [d,F] (all bf16 bit patterns, uint16);
+    ids [N,K] int32, gates [N,K] fp32.  Returns (y [N,d] fp32, mag [N,d] fp64)
+    and, with want_h, also h [N*K,F] (slot order) and h_s [N,F] as uint16."""
+    lib = _load()
+    x = _c(x_bf16_bits, np.uint16)
+    ids = _c(ids, np.int32)
+    gates = _c(gates, np.float32)
+    wgu = _c(wgu_bf16_bits, np.uint16)
+    wd = _c(wd_bf16_bits, np.uint16)
+    N, d = x.shape
+    K = ids.shape[1]
+    E, F2, d2 = wgu.shape
+    F = F2 // 2
+    assert d2 == d and wd.shape == (E, d, F) and gates.shape == ids.shape
+    if wgu_s_bf16_bits is not None:
+        wgu_s = _c(wgu_s_bf16_bits, np.uint16)
+        wd_s = _c(wd_s_bf16_bits, np.uint16)
+        assert wgu_s.shape == (2 * F, d) and wd_s.shape == (d, F)
+    else:
+        wgu_s = wd_s = None
+    y = np.empty((N, d), np.float32)
+    mag = np.empty((N, d), np.float64)
+    h = np.empty((N * K, F), np.uint16) if want_h else None
+    h_s = np.empty((N, F), np.uint16) if (want_h and wgu_s is not None) else None
+    lib.oracle_expert_ffn(_ptr(x), _ptr(ids), _ptr(gates), _ptr(wgu), _ptr(wd),
+                          None if wgu_s is None else _ptr(wgu_s),
+                          None if wd_s is None else _ptr(wd_s), N, d, F, E, K,
+                          None if h is None else _ptr(h), None if h_s is None else _ptr(h_s),
+                          _ptr(y), _ptr(mag))
+    if want_h:
+        return y, mag, h, h_s
+    return y, mag

@@ -14,9 +14,12 @@
  *           6.1 (routing equations), 6.2 (MaxVio), 7.1 (Quantile Balancing),
  *           7.2 (numerical check), 7.3 (exact quantile by radix selection),
  *           9 (intervention rate).
+ *           6.1 also defines the layer output y_t = f_shared(x_t) +
+ *           sum_e S_t,e f_e(x_t) that the experts compute.
  *   [K1D]  "Kolibri 1 im Detail: hybride RNoPE-Attention, Sparse MoE und
  *           FP8-Serving" -- section "Routing: Auswahl-Bias und Mischgewichte
- *           sind getrennt" (bf16 router, fp32 logits, two-step rule).
+ *           sind getrennt" (bf16 router, fp32 logits, two-step rule; every
+ *           routed or shared expert a SwiGLU MLP 2560 -> 2 x 512 -> 2560).
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - Total order on fp32: the order-preserving key of the bit pattern
@@ -30,6 +33,9 @@
  *     below, rounded once to fp32.
  *   - Permutation: experts ascending, and inside an expert the flat slot
  *     index t*K+k ascending (a stable counting sort).
+ *   - Experts: the SwiGLU activation h = SiLU(gate) * up is rounded once to
+ *     bf16 (the operand of the down projection); everything else is fp64,
+ *     and the layer output is rounded once to fp32.
  *
  * Build: plain C11, no fast-math, no FP contraction (the arithmetic must be
  * exactly the operations written).  OpenMP only splits independent rows or
@@ -406,6 +412,120 @@ void oracle_score_grad_to_logits(const float *z, const float *gs, int64_t n, flo
         else if (z[i] < -700.0f) s = 0.0;
         else s = 1.0 / (1.0 + oracle_exp_spec(-(double)z[i]));
         gz[i] = (float)((double)gs[i] * (s * (1.0 - s)));
+    }
+}
+
+/* ------------------------------------------- the experts ([KPT] 6.1) */
+
+/* The bf16 value nearest to the real number v (ties to the even last
+ * significand bit), as its 16 bits.  v is rounded once, straight from fp64:
+ * an 8-bit significand for normal values, a fixed step of 2^-133 below
+ * 2^-126; values at or past the midpoint to 2^128 become infinity. */
+uint16_t oracle_bf16_round_f64(double v)
+{
+    if (v == 0.0) return signbit(v) ? 0x8000u : 0x0000u;
+    const double a = fabs(v);
+    double r;
+    if (a < ldexp(1.0, -126)) {
+        r = ldexp(nearbyint(ldexp(a, 133)), -133);
+    } else {
+        int e;
+        const double m = frexp(a, &e);           /* a = m 2^e, 0.5 <= m < 1 */
+        r = ldexp(nearbyint(ldexp(m, 8)), e - 8);
+    }
+    uint16_t b;
+    if (r >= ldexp(1.0, 128)) b = 0x7f80u;
+    else b = (uint16_t)(f32_to_bits((float)r) >> 16);   /* r has at most 8 significant bits */
+    return (uint16_t)(signbit(v) ? (b | 0x8000u) : b);
+}
+
+/* SiLU(g) = g sigma(g) with sigma(g) = 1 / (1 + e^(-g)) in fp64, e^x from
+ * exp_spec; for g <= -700 the product is 0 (-0 for negative g). */
+double oracle_silu_spec(double g)
+{
+    if (g <= -700.0) return -0.0;
+    return g * (1.0 / (1.0 + oracle_exp_spec(-g)));
+}
+
+/* One SwiGLU expert of [K1D] ("two projections d -> F form SiLU(gate) x up,
+ * then F -> d") applied to one token x [d]:
+ *   g_j = sum_i x_i Wg[j,i],  u_j = sum_i x_i Wu[j,i]   (fp64, i ascending)
+ *   h_j = bf16(SiLU(g_j) u_j)                          (the activation the
+ *                                                       down projection reads)
+ *   Y_c = sum_j h_j Wd[c,j]                              (fp64, j ascending)
+ * wgu [2F, d]: rows 0..F-1 are Wg, rows F..2F-1 are Wu; wd [d, F].
+ * h [F] receives the bf16 bits; mag[c] += scale * sum_j |h_j Wd[c,j]|. */
+static void swiglu_expert(const uint16_t *x, const uint16_t *wgu, const uint16_t *wd, int32_t d,
+                          int32_t F, uint16_t *h, double *hv, double *y, double *mag,
+                          double scale)
+{
+    for (int32_t j = 0; j < F; ++j) {
+        const uint16_t *wg = wgu + (int64_t)j * d, *wu = wgu + (int64_t)(F + j) * d;
+        double g = 0.0, u = 0.0;
+        for (int32_t i = 0; i < d; ++i) {
+            const double xi = bf16_value(x[i]);
+            g += xi * bf16_value(wg[i]);
+            u += xi * bf16_value(wu[i]);
+        }
+        h[j] = oracle_bf16_round_f64(oracle_silu_spec(g) * u);
+        hv[j] = bf16_value(h[j]);
+    }
+    for (int32_t c = 0; c < d; ++c) {
+        const uint16_t *w = wd + (int64_t)c * F;
+        double acc = 0.0, m = 0.0;
+        for (int32_t j = 0; j < F; ++j) {
+            const double t = hv[j] * bf16_value(w[j]);
+            acc += t;
+            m += fabs(t);
+        }
+        y[c] = acc;
+        if (mag) mag[c] += scale * m;
+    }
+}
+
+/* The MoE output of [KPT] 6.1: y_t = f_shared(x_t) + sum_k S_t,k f_e(x_t)
+ * over the token's K routed experts e = ids[t,k] with their gates S (the
+ * unbiased sigmoid scores, not renormalised).  x [N,d], wgu [E,2F,d],
+ * wd [E,d,F] (bf16 bits); the shared expert (wgu_s [2F,d], wd_s [d,F]) is
+ * left out when wgu_s is NULL.  The sum is taken in fp64 in the order
+ * shared, k = 0..K-1, and rounded once to fp32 into y [N,d].
+ * Optional outputs: h [N*K, F] the routed activations in slot order t*K+k,
+ * h_s [N, F] the shared ones, mag [N,d] = sum of |each product| weighted by
+ * |S| (the scale of the rounding error of any summation order). */
+void oracle_expert_ffn(const uint16_t *x, const int32_t *ids, const float *gates,
+                       const uint16_t *wgu, const uint16_t *wd, const uint16_t *wgu_s,
+                       const uint16_t *wd_s, int64_t N, int32_t d, int32_t F, int32_t E,
+                       int32_t K, uint16_t *h, uint16_t *h_s, float *y, double *mag)
+{
+    #pragma omp parallel
+    {
+        uint16_t *hb = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)F);
+        double *hv = (double *)malloc(sizeof(double) * (size_t)F);
+        double *ye = (double *)malloc(sizeof(double) * (size_t)d);
+        double *acc = (double *)malloc(sizeof(double) * (size_t)d);
+        #pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < N; ++t) {
+            const uint16_t *xt = x + t * d;
+            double *mt = mag ? mag + t * d : NULL;
+            if (mt) memset(mt, 0, sizeof(double) * (size_t)d);
+            for (int32_t c = 0; c < d; ++c) acc[c] = 0.0;
+            if (wgu_s) {
+                swiglu_expert(xt, wgu_s, wd_s, d, F, hb, hv, ye, mt, 1.0);
+                if (h_s) memcpy(h_s + t * F, hb, sizeof(uint16_t) * (size_t)F);
+                for (int32_t c = 0; c < d; ++c) acc[c] += ye[c];
+            }
+            for (int32_t k = 0; k < K; ++k) {
+                const int32_t e = ids[t * K + k];
+                if (e < 0 || e >= E) abort();
+                const double s = (double)gates[t * K + k];
+                swiglu_expert(xt, wgu + (int64_t)e * 2 * F * d, wd + (int64_t)e * d * F, d, F, hb,
+                              hv, ye, mt, fabs(s));
+                if (h) memcpy(h + (t * K + k) * F, hb, sizeof(uint16_t) * (size_t)F);
+                for (int32_t c = 0; c < d; ++c) acc[c] += s * ye[c];
+            }
+            for (int32_t c = 0; c < d; ++c) y[t * d + c] = (float)acc[c];
+        }
+        free(hb); free(hv); free(ye); free(acc);
     }
 }
 
