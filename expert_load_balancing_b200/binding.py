@@ -49,6 +49,13 @@ SIGNATURES = {
     "kolibri_eqb_update": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _SZ, _P]),
     "kolibri_route_and_balance": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P, _P,
                                                  _SZ, _P]),
+    "kolibri_expert_ffn_workspace_size": (_SZ, [_I64, _I32, _I32, _I32, _I32]),
+    "kolibri_expert_ffn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32, _I32,
+                                          _I32, _I32, _P, _SZ, _P]),
+    "kolibri_expert_dispatch": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P]),
+    "kolibri_expert_gate_up": (ctypes.c_int, [_P, _I64, _P, _I32, _P, _P, _I32, _I32, _P]),
+    "kolibri_expert_down": (ctypes.c_int, [_P, _I64, _P, _I32, _P, _P, _I32, _I32, _P]),
+    "kolibri_expert_combine": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _P, _P]),
     "kolibri_device_status": (ctypes.c_int, [_P]),
 }
 
@@ -404,3 +411,117 @@ def kolibri_intervention_rate(z: torch.Tensor, ids: torch.Tensor, stream=None):
            load().kolibri_intervention_rate(_ptr(z), _ptr(ids), N, E, K, _ptr(rate), _ptr(overlaps),
                                             _stream(stream)))
     return rate, overlaps
+
+
+# ---------------------------------------------------------------- the experts
+
+def expert_ffn_workspace(N: int, d: int, F: int, K: int, shared: bool, device=None) -> torch.Tensor:
+    """Device workspace for kolibri_expert_ffn."""
+    n = int(load().kolibri_expert_ffn_workspace_size(N, d, F, K, 1 if shared else 0))
+    return torch.empty((max(n, 1),), dtype=torch.uint8, device=device or "cuda")
+
+
+def kolibri_expert_ffn(x: torch.Tensor, perm: torch.Tensor, offsets: torch.Tensor, inv: torch.Tensor,
+                       gates: torch.Tensor, w_gate_up: torch.Tensor, w_down: torch.Tensor,
+                       ws_gate_up: torch.Tensor | None = None, ws_down: torch.Tensor | None = None,
+                       y: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """y [N, d] fp32 = shared expert + sum_k gates[t,k] expert_{ids[t,k]}(x_t) (SwiGLU experts)."""
+    N, d = x.shape
+    K = gates.shape[1]
+    E, F2, _ = w_gate_up.shape
+    F = F2 // 2
+    _need(x, torch.bfloat16, (N, d), "x")
+    _need(perm, torch.int32, (N * K,), "perm")
+    _need(offsets, torch.int64, (E + 1,), "offsets")
+    _need(inv, torch.int32, (N * K,), "inv")
+    _need(gates, torch.float32, (N, K), "gates")
+    _need(w_gate_up, torch.bfloat16, (E, 2 * F, d), "w_gate_up")
+    _need(w_down, torch.bfloat16, (E, d, F), "w_down")
+    if ws_gate_up is not None:
+        _need(ws_gate_up, torch.bfloat16, (2 * F, d), "ws_gate_up")
+        _need(ws_down, torch.bfloat16, (d, F), "ws_down")
+    if y is None:
+        y = torch.empty((N, d), dtype=torch.float32, device=x.device)
+    _need(y, torch.float32, (N, d), "y")
+    if ws is None:
+        ws = expert_ffn_workspace(N, d, F, K, ws_gate_up is not None, x.device)
+    _check("kolibri_expert_ffn",
+           load().kolibri_expert_ffn(_ptr(x), _ptr(perm), _ptr(offsets), _ptr(inv), _ptr(gates),
+                                     _ptr(w_gate_up), _ptr(w_down), _ptr(ws_gate_up), _ptr(ws_down),
+                                     _ptr(y), N, d, F, E, K, _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def kolibri_expert_dispatch(x: torch.Tensor, perm: torch.Tensor, K: int,
+                            x_perm: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """x_perm [N*K, d] with x_perm[p] = x[perm[p] // K]."""
+    N, d = x.shape
+    _need(x, torch.bfloat16, (N, d), "x")
+    _need(perm, torch.int32, (N * K,), "perm")
+    if x_perm is None:
+        x_perm = torch.empty((N * K, d), dtype=torch.bfloat16, device=x.device)
+    _need(x_perm, torch.bfloat16, (N * K, d), "x_perm")
+    _check("kolibri_expert_dispatch",
+           load().kolibri_expert_dispatch(_ptr(x), _ptr(perm), N, d, K, _ptr(x_perm), _stream(stream)))
+    return x_perm
+
+
+def kolibri_expert_gate_up(a: torch.Tensor, offsets: torch.Tensor | None, w_gate_up: torch.Tensor,
+                           h: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """h [rows, F] bf16 = bf16(SiLU(a Wg^T) * (a Wu^T)), expert g on rows [offsets[g], offsets[g+1])."""
+    rows, d = a.shape
+    if w_gate_up.dim() == 2:
+        w_gate_up = w_gate_up.unsqueeze(0)
+    G, F2, _ = w_gate_up.shape
+    F = F2 // 2
+    _need(a, torch.bfloat16, (rows, d), "a")
+    _need(w_gate_up, torch.bfloat16, (G, 2 * F, d), "w_gate_up")
+    if offsets is not None:
+        _need(offsets, torch.int64, (G + 1,), "offsets")
+    if h is None:
+        h = torch.empty((rows, F), dtype=torch.bfloat16, device=a.device)
+    _need(h, torch.bfloat16, (rows, F), "h")
+    _check("kolibri_expert_gate_up",
+           load().kolibri_expert_gate_up(_ptr(a), rows, _ptr(offsets), G, _ptr(w_gate_up), _ptr(h),
+                                         d, F, _stream(stream)))
+    return h
+
+
+def kolibri_expert_down(h: torch.Tensor, offsets: torch.Tensor | None, w_down: torch.Tensor,
+                        y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [rows, d] fp32 = h Wd_g^T per group."""
+    rows, F = h.shape
+    if w_down.dim() == 2:
+        w_down = w_down.unsqueeze(0)
+    G, d, _ = w_down.shape
+    _need(h, torch.bfloat16, (rows, F), "h")
+    _need(w_down, torch.bfloat16, (G, d, F), "w_down")
+    if offsets is not None:
+        _need(offsets, torch.int64, (G + 1,), "offsets")
+    if y is None:
+        y = torch.empty((rows, d), dtype=torch.float32, device=h.device)
+    _need(y, torch.float32, (rows, d), "y")
+    _check("kolibri_expert_down",
+           load().kolibri_expert_down(_ptr(h), rows, _ptr(offsets), G, _ptr(w_down), _ptr(y), d, F,
+                                      _stream(stream)))
+    return y
+
+
+def kolibri_expert_combine(y_perm: torch.Tensor, y_shared: torch.Tensor | None, inv: torch.Tensor,
+                           gates: torch.Tensor, y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [N, d] = y_shared + sum_k gates[t,k] y_perm[inv[t*K+k]] (fp32, k ascending)."""
+    N, K = gates.shape
+    d = y_perm.shape[1]
+    _need(y_perm, torch.float32, (N * K, d), "y_perm")
+    if y_shared is not None:
+        _need(y_shared, torch.float32, (N, d), "y_shared")
+    _need(inv, torch.int32, (N * K,), "inv")
+    _need(gates, torch.float32, (N, K), "gates")
+    if y is None:
+        y = torch.empty((N, d), dtype=torch.float32, device=y_perm.device)
+    _need(y, torch.float32, (N, d), "y")
+    _check("kolibri_expert_combine",
+           load().kolibri_expert_combine(_ptr(y_perm), _ptr(y_shared), _ptr(inv), _ptr(gates), N, d, K,
+                                         _ptr(y), _stream(stream)))
+    return y

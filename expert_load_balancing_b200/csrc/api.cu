@@ -217,12 +217,83 @@ kolibri_status kolibri_intervention_rate(const float* z, const int32_t* ids, int
                                        static_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+constexpr int64_t kExpertRowLimit = (static_cast<int64_t>(1) << 31) - 512;
+}
+
+size_t kolibri_expert_ffn_workspace_size(int64_t N, int32_t d, int32_t F, int32_t K,
+                                         int32_t shared) {
+  if (N < 1 || K < 1 || d < 1 || F < 1) return 0;
+  return expert_layout(N, d, F, K, shared != 0).total;
+}
+
+kolibri_status kolibri_expert_ffn(const void* x, const int32_t* perm, const int64_t* offsets,
+                                  const int32_t* inv, const float* gates, const void* w_gate_up,
+                                  const void* w_down, const void* ws_gate_up, const void* ws_down,
+                                  float* y, int64_t N, int32_t d, int32_t F, int32_t E, int32_t K,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !perm || !offsets || !inv || !gates || !w_gate_up || !w_down || !y || !ws)
+    return KOLIBRI_ERR_INVALID_ARG;
+  if ((ws_gate_up == nullptr) != (ws_down == nullptr)) return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(y) ||
+      !aligned16(ws) || (ws_gate_up && (!aligned16(ws_gate_up) || !aligned16(ws_down))))
+    return KOLIBRI_ERR_INVALID_ARG;
+  if (N < 1 || K < 1 || K > 32 || K > E) return KOLIBRI_ERR_INVALID_ARG;
+  if (!expert_shape_supported(d, F, E) || N * K >= kExpertRowLimit) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < expert_layout(N, d, F, K, ws_gate_up != nullptr).total)
+    return KOLIBRI_ERR_WORKSPACE_TOO_SMALL;
+  return from_cuda(launch_expert_ffn(x, perm, offsets, inv, gates, w_gate_up, w_down, ws_gate_up,
+                                     ws_down, y, N, d, F, E, K, ws, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_expert_dispatch(const void* x, const int32_t* perm, int64_t N, int32_t d,
+                                       int32_t K, void* x_perm, void* stream) {
+  if (!x || !perm || !x_perm || !aligned16(x) || !aligned16(x_perm)) return KOLIBRI_ERR_INVALID_ARG;
+  if (N < 1 || K < 1 || d < 1) return KOLIBRI_ERR_INVALID_ARG;
+  if (d % 8 != 0 || N * K >= kExpertRowLimit) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(launch_expert_dispatch(x, perm, N, d, K, x_perm, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_expert_gate_up(const void* a, int64_t rows, const int64_t* offsets, int32_t G,
+                                      const void* w_gate_up, void* h, int32_t d, int32_t F,
+                                      void* stream) {
+  if (!a || !w_gate_up || !h || !aligned16(a) || !aligned16(w_gate_up) || !aligned16(h))
+    return KOLIBRI_ERR_INVALID_ARG;
+  if (rows < 1 || (offsets == nullptr && G != 1)) return KOLIBRI_ERR_INVALID_ARG;
+  if (!expert_shape_supported(d, F, G) || rows >= kExpertRowLimit) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(launch_expert_gate_up(a, rows, offsets, G, w_gate_up, h, d, F,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_expert_down(const void* h, int64_t rows, const int64_t* offsets, int32_t G,
+                                   const void* w_down, float* y, int32_t d, int32_t F, void* stream) {
+  if (!h || !w_down || !y || !aligned16(h) || !aligned16(w_down) || !aligned16(y))
+    return KOLIBRI_ERR_INVALID_ARG;
+  if (rows < 1 || (offsets == nullptr && G != 1)) return KOLIBRI_ERR_INVALID_ARG;
+  if (!expert_shape_supported(d, F, G) || rows >= kExpertRowLimit) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(launch_expert_down(h, rows, offsets, G, w_down, y, d, F,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_expert_combine(const float* y_perm, const float* y_shared, const int32_t* inv,
+                                      const float* gates, int64_t N, int32_t d, int32_t K, float* y,
+                                      void* stream) {
+  if (!y_perm || !inv || !gates || !y || !aligned16(y_perm) || !aligned16(y) ||
+      (y_shared && !aligned16(y_shared)))
+    return KOLIBRI_ERR_INVALID_ARG;
+  if (N < 1 || K < 1 || K > 32 || d < 4) return KOLIBRI_ERR_INVALID_ARG;
+  if (d % 4 != 0 || N * K >= kExpertRowLimit) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(launch_expert_combine(y_perm, y_shared, inv, gates, N, d, K, y,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 kolibri_status kolibri_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return KOLIBRI_ERR_CUDA;
   const unsigned v = status_take_api() | status_take_eqb() | status_take_noalloc() |
                      status_take_permute() | status_take_route() | status_take_logits() |
-                     status_take_forward() | status_take_balance() | status_take_small();
+                     status_take_forward() | status_take_balance() | status_take_small() |
+                     status_take_experts();
   if (v & kStatusReadFailed) return KOLIBRI_ERR_CUDA;
   if (v & kStatusTimeout) return KOLIBRI_ERR_TIMEOUT;
   if (v & kStatusBadInput) return KOLIBRI_ERR_DEVICE;

@@ -49,6 +49,28 @@ bool router_small_preferred(int64_t N);
 cudaError_t launch_router_logits_small(const void* x, const void* w, float* z, int64_t N, int32_t d,
                                        int32_t E, cudaStream_t s);
 
+// The expert layer (expert_ffn.cu): workspace regions and the stages.
+struct ExpertLayout {
+  size_t off_x_perm, off_h, off_y_perm, off_h_shared, off_y_shared, total;
+};
+bool expert_shape_supported(int32_t d, int32_t F, int32_t E);
+ExpertLayout expert_layout(int64_t N, int32_t d, int32_t F, int32_t K, bool shared);
+cudaError_t launch_expert_dispatch(const void* x, const int32_t* perm, int64_t N, int32_t d,
+                                   int32_t K, void* x_perm, cudaStream_t s);
+cudaError_t launch_expert_gate_up(const void* a, int64_t rows, const int64_t* offsets, int32_t G,
+                                  const void* w_gate_up, void* h, int32_t d, int32_t F,
+                                  cudaStream_t s);
+cudaError_t launch_expert_down(const void* h, int64_t rows, const int64_t* offsets, int32_t G,
+                               const void* w_down, float* y, int32_t d, int32_t F, cudaStream_t s);
+cudaError_t launch_expert_combine(const float* y_perm, const float* y_shared, const int32_t* inv,
+                                  const float* gates, int64_t N, int32_t d, int32_t K, float* y,
+                                  cudaStream_t s);
+cudaError_t launch_expert_ffn(const void* x, const int32_t* perm, const int64_t* offsets,
+                              const int32_t* inv, const float* gates, const void* w_gate_up,
+                              const void* w_down, const void* ws_gate_up, const void* ws_down,
+                              float* y, int64_t N, int32_t d, int32_t F, int32_t E, int32_t K,
+                              void* ws, cudaStream_t s);
+
 // Fused logits + selection (router_forward.cu).  Returns cudaErrorNotSupported
 // for shapes it does not cover; the caller then runs logits and top-K apart.
 // Rows it could not finish carry a NaN alpha; launch_select_fixup completes them.
@@ -134,5 +156,6 @@ unsigned status_take_logits();
 unsigned status_take_forward();
 unsigned status_take_balance();
 unsigned status_take_small();
+unsigned status_take_experts();
 
 }  // namespace kolibri

@@ -324,6 +324,67 @@ KOLIBRI_API kolibri_status kolibri_intervention_rate(const float *z, const int32
                                                      unsigned long long *overlaps, void *stream);
 
 /*
+ * The expert layer ("Kolibri Pre-Training from Scratch" 6.1, with the
+ * experts of "Kolibri 1 im Detail": every routed or shared expert a SwiGLU
+ * MLP, two d -> F projections forming SiLU(gate) x up, then F -> d):
+ *   y_t = f_shared(x_t) + sum_k S_t,k f_{e_t,k}(x_t),  f(x) = (SiLU(x Wg^T) * (x Wu^T)) Wd^T
+ * with the gates S of kolibri_router_forward (unbiased sigmoid scores, not
+ * renormalised) and the grouping of kolibri_expert_permute.
+ *
+ * Arithmetic: bf16 operands, fp32 accumulation on the tensor cores; the
+ * activation h = SiLU(g) u is formed in fp32 and rounded once to bf16 (the
+ * operand of the down projection); the routed outputs are kept in fp32 and
+ * combined in fp32 multiply-adds in the order shared, k = 0 .. K-1.
+ *
+ * Layouts (row-major, bf16 unless noted, all 16-byte aligned):
+ *   x [N, d]; perm [N*K] int32, offsets [E+1] int64, inv [N*K] int32 from
+ *   kolibri_expert_permute; gates [N, K] fp32;
+ *   w_gate_up [E, 2F, d]: per expert the F gate rows, then the F up rows;
+ *   w_down [E, d, F]; shared expert ws_gate_up [2F, d], ws_down [d, F], or
+ *   both NULL for a layer without one; y [N, d] fp32, written.
+ * Shapes: d a multiple of 256, F a multiple of 128, 1 <= E <= 512,
+ * N*K < 2^31 - 512.  Otherwise KOLIBRI_ERR_UNSUPPORTED_SHAPE.
+ * ws: kolibri_expert_ffn_workspace_size(N, d, F, K, shared) bytes of device
+ * memory (the gathered rows, h and the routed outputs; about
+ * N K (6 d + 2 F) bytes), owned by the caller.  Out-of-range entries of perm
+ * or inv are skipped and set KOLIBRI_ERR_DEVICE in kolibri_device_status.
+ */
+KOLIBRI_API size_t kolibri_expert_ffn_workspace_size(int64_t N, int32_t d, int32_t F, int32_t K,
+                                                     int32_t shared);
+KOLIBRI_API kolibri_status kolibri_expert_ffn(const void *x, const int32_t *perm,
+                                              const int64_t *offsets, const int32_t *inv,
+                                              const float *gates, const void *w_gate_up,
+                                              const void *w_down, const void *ws_gate_up,
+                                              const void *ws_down, float *y, int64_t N, int32_t d,
+                                              int32_t F, int32_t E, int32_t K, void *ws,
+                                              size_t ws_bytes, void *stream);
+
+/*
+ * The four stages of kolibri_expert_ffn, each callable on its own:
+ *   kolibri_expert_dispatch: x_perm [N*K, d] with x_perm[p] = x[perm[p] / K].
+ *   kolibri_expert_gate_up: h [rows, F] bf16 = bf16(SiLU(a Wg^T) * (a Wu^T))
+ *     where rows [offsets[g], offsets[g+1]) of a [rows, d] use expert g of
+ *     w_gate_up [G, 2F, d]; offsets NULL: one group of all rows (G = 1).
+ *   kolibri_expert_down: y [rows, d] fp32 = h Wd_g^T per group, w_down [G, d, F].
+ *   kolibri_expert_combine: y [N, d] = y_shared (or 0 when NULL) + sum_k
+ *     gates[t,k] y_perm[inv[t*K+k]] in fp32 multiply-adds, k ascending.
+ */
+KOLIBRI_API kolibri_status kolibri_expert_dispatch(const void *x, const int32_t *perm, int64_t N,
+                                                   int32_t d, int32_t K, void *x_perm,
+                                                   void *stream);
+KOLIBRI_API kolibri_status kolibri_expert_gate_up(const void *a, int64_t rows,
+                                                  const int64_t *offsets, int32_t G,
+                                                  const void *w_gate_up, void *h, int32_t d,
+                                                  int32_t F, void *stream);
+KOLIBRI_API kolibri_status kolibri_expert_down(const void *h, int64_t rows, const int64_t *offsets,
+                                               int32_t G, const void *w_down, float *y, int32_t d,
+                                               int32_t F, void *stream);
+KOLIBRI_API kolibri_status kolibri_expert_combine(const float *y_perm, const float *y_shared,
+                                                  const int32_t *inv, const float *gates,
+                                                  int64_t N, int32_t d, int32_t K, float *y,
+                                                  void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device: KOLIBRI_OK, KOLIBRI_ERR_TIMEOUT or KOLIBRI_ERR_DEVICE
  * (the first recorded), or KOLIBRI_ERR_CUDA if the synchronisation failed.
