@@ -588,6 +588,119 @@ def run_part(args):
     }
 
 
+# ---------------------------------------------------------------- the experts
+
+def run_experts(args):
+    """The expert layer after the router on one microbatch of N = 16384 tokens
+    (d = 2560, E = 384 routed experts of 2560 -> 2 x 512 -> 2560, K = 6, plus
+    the shared expert): dispatch, the grouped gate/up and down projections,
+    combine.  The routing is our own: logits, one EQB update, re-routing with
+    the new bias, permutation.  Timed region: kolibri_expert_ffn alone, inputs
+    resident.  Roofline: the layer's FLOPs against the measured bf16 peak (the
+    run is short, so the burst figure applies); the algorithmic bytes (every
+    weight once, x in, y out) would take less time at the HBM peak."""
+    import oracle
+    oracle.build()
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    B.load()
+    N, d, F, E, K = args.tokens or 16384, 2560, 512, 384, 6
+    g = torch.Generator(device=device)
+    g.manual_seed(11)
+    wgu = (torch.randn(E, 2 * F, d, generator=g, device=device) / math.sqrt(d)).to(torch.bfloat16)
+    wd = (torch.randn(E, d, F, generator=g, device=device) / math.sqrt(F)).to(torch.bfloat16)
+    wgu_s = (torch.randn(2 * F, d, generator=g, device=device) / math.sqrt(d)).to(torch.bfloat16)
+    wd_s = (torch.randn(d, F, generator=g, device=device) / math.sqrt(F)).to(torch.bfloat16)
+    wl = workloads.Workload("experts", N, d, E, K)
+    x = torch.randn(N, d, generator=g, device=device).to(torch.bfloat16)
+    w_router = workloads.make_w(wl).to(device)
+    beta = torch.zeros(E, dtype=torch.float32, device=device)
+    z = torch.empty((N, E), dtype=torch.float32, device=device)
+    ids = torch.empty((N, K), dtype=torch.int32, device=device)
+    gates = torch.empty((N, K), dtype=torch.float32, device=device)
+    alpha = torch.empty((N,), dtype=torch.float32, device=device)
+    B.kolibri_router_forward(x, w_router, beta, K, z=z, ids=ids, gates=gates, alpha=alpha)
+    B.kolibri_eqb_update(z, alpha, beta, K, B.workspace(B.KOLIBRI_OP_EQB, N, E, K, device))
+    B.kolibri_router_forward(x, w_router, beta, K, z=z, ids=ids, gates=gates, alpha=alpha)
+    counts = torch.empty((E,), dtype=torch.int32, device=device)
+    offsets = torch.empty((E + 1,), dtype=torch.int64, device=device)
+    perm = torch.empty((N * K,), dtype=torch.int32, device=device)
+    inv = torch.empty((N * K,), dtype=torch.int32, device=device)
+    B.kolibri_expert_permute(ids, E, B.workspace(B.KOLIBRI_OP_PERMUTE, N, E, K, device), counts,
+                             offsets, perm, inv)
+    ws = B.expert_ffn_workspace(N, d, F, K, True, device)
+    y = torch.empty((N, d), dtype=torch.float32, device=device)
+    stream = torch.cuda.Stream(device)
+
+    def once():
+        B.kolibri_expert_ffn(x, perm, offsets, inv, gates, wgu, wd, wgu_s, wd_s, y=y, ws=ws,
+                             stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            once()
+    stream.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0")
+    sampler.start()
+    time.sleep(0.3)
+    t0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            once()
+    t1.record(stream)
+    t1.synchronize()
+    clocks = sampler.stop()
+    st = B.kolibri_device_status(stream)
+    if st != B.KOLIBRI_OK:
+        raise RuntimeError(f"device status: {B.status_string(st)}")
+    ms = t0.elapsed_time(t1) / args.steps
+    c = counts.cpu().numpy()
+    flops = 6.0 * d * F * N * (K + 1)
+    bytes_alg = 2.0 * 3 * d * F * (E + 1) + 2.0 * N * d + 4.0 * N * d + 16.0 * N * K
+    peaks = _peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    # the oracle on a bounded sample: the first tokens of the same microbatch
+    n = 8
+    xs = x[:n].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    ids_h = ids[:n].cpu().numpy()
+    used = np.unique(ids_h)
+    remap = np.full(E, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    sl = torch.from_numpy(used).to(device)
+    wgu_h = wgu[sl].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    wd_h = wd[sl].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    wgu_sh = wgu_s.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    wd_sh = wd_s.cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    gates_h = gates[:n].cpu().numpy()
+    reps, cpu_s = 0, 0.0
+    while cpu_s < 2.0:
+        t = time.time()
+        oracle.expert_ffn(xs, remap[ids_h].astype(np.int32), gates_h, wgu_h, wd_h, wgu_sh, wd_sh)
+        cpu_s += time.time() - t
+        reps += 1
+    return {
+        "metric": "expert layer (dispatch + grouped SwiGLU gate/up + down + combine, shared + 6 routed "
+                  "experts of 2560 -> 2x512 -> 2560, E=384): tokens/s at N=16384",
+        "part": "experts", "value": N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "dtype": "bf16 in, fp32 accumulate", "data": "synthetic",
+        "config": {"workload": "experts", "N": N, "d": d, "F": F, "E": E, "K": K,
+                   "routing": "own forward after one EQB update",
+                   "load_min_max": [int(c.min()), int(c.max())]},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                     "algorithmic": f"{flops / 1e12:.3f} TFLOP per layer (6 d F per token-expert); "
+                                    f"{bytes_alg / 1e9:.2f} GB of weights, x and y "
+                                    f"({bytes_alg / peaks['hbm_gbs'] / 1e6:.3f} ms at the HBM peak)",
+                     "peak_kind": f"bf16 burst, of {peaks['source']}"},
+        "clocks": clocks,
+        "gpu_launches": 7,
+        "cpu_baseline": {"value": n * reps / cpu_s, "unit": "tokens/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": f"first {n} tokens, {reps} times, {cpu_s:.1f} s"},
+    }
+
+
 # ---------------------------------------------------------------- decode
 
 def _decode_oracle(oracle, wl, layers, xs, ws, betas):
@@ -715,7 +828,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--decode", action="store_true",
                     help="time the decode sweep (50 layers, N = 1, 8, 64, 256; one GPU)")
-    ap.add_argument("--part", choices=sorted(PARTS), default=None,
+    ap.add_argument("--part", choices=sorted(PARTS) + ["experts"], default=None,
                     help="time one balancing piece instead of the routing step (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
@@ -726,6 +839,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.decode and args.impl == "ours":
         print(json.dumps(run_decode(args)), flush=True)
+        return
+    if args.part == "experts" and args.impl == "ours":
+        print(json.dumps(run_experts(args)), flush=True)
         return
     if args.part and args.impl == "ours":
         print(json.dumps(run_part(args)), flush=True)

@@ -16,17 +16,20 @@
 // The shared expert runs the same two projections over x itself.
 //
 // The projections are one grouped GEMM kernel: a persistent kernel on SM
-// pairs (tcgen05.mma.cta_group::2, M = 256 rows, N = 256 columns, bf16 in,
-// fp32 accumulate in TMEM, two accumulators so the epilogue of one tile
-// runs under the MMAs of the next).  Tiles are (expert, 256-row block,
-// column block); the kernel maps a tile index to them on the device from
-// the offsets, so no host round trip is needed between the permutation and
-// the GEMMs.  A row block may run past its expert's segment: those rows are
-// loaded (or zero-filled past the end) but never stored.  In the gate/up
-// projection the leader CTA loads 128 gate rows and its partner the 128 up
-// rows of the same hidden units, so accumulator columns c and c + 128 of a
-// row are the gate and up value of one unit and the epilogue forms the
-// SwiGLU product in registers.  No load uses cluster multicast.
+// pairs (tcgen05.mma.cta_group::2, bf16 in, fp32 accumulate in TMEM, two
+// accumulators so the epilogue of one tile runs under the MMAs of the
+// next).  The weights are the MMA's M side (256 features per pair) and the
+// tokens its N side, so the last token block of an expert is an MMA of just
+// its rows rounded up to 32 (with balanced loads of about 256 rows an
+// expert, 256-row blocks of tokens on the M side would spend up to half of
+// the tensor time on empty rows).  Tiles are (expert, token block, feature
+// block)
+// from the offsets, so no host round trip is needed between the
+// permutation and the GEMMs.  In the gate/up projection a CTA stages the
+// gate rows and the up rows of the same 128 units and issues one MMA for
+// each into its own columns, so a thread holds both sums of its unit and
+// the epilogue forms SiLU(gate) * up in registers.  Stores are one token
+// row segment per warp instruction.  No load uses cluster multicast.
 #include <cuda_bf16.h>
 
 #include "launch.h"
@@ -40,23 +43,34 @@ using namespace gemm;
 
 constexpr int kThreads = 192;            // warp 0 TMA, warp 1 TMEM + MMA, warps 2..5 epilogue
 constexpr int kEpiWarps = 4;
-constexpr int kTileM = 2 * kBM;          // 256 rows per pair
-constexpr int kTileN = 256;              // accumulator columns per tile
-constexpr int kHalfN = kTileN / 2;       // B rows per CTA
-constexpr int kAccCols = 2 * kTileN;     // two accumulators
+constexpr int kFeat = 2 * kBM;           // weight rows per pair tile: the MMA's M
+constexpr int kAccCols = 512;            // two accumulator buffers of 256 columns
 constexpr int kMaxGroups = KOLIBRI_MAX_EXPERTS;
-constexpr uint32_t kStageBytes = kBM * kBK * 2 + kHalfN * kBK * 2;   // 32 KB
+constexpr uint32_t kWBytes = kBM * kBK * 2;        // 128 weight rows x 64 (16 KB)
+
+// Per projection: tokens per tile at most (the MMA's N), weight bytes and
+// token bytes a CTA stages per k-block.  Gate/up: 128 gate rows and the same
+// units' 128 up rows (two MMAs per k-step into two column ranges of one
+// accumulator buffer), up to 128 tokens; down: 128 weight rows, up to 256
+// tokens.
+template <bool kGateUp>
+struct Cfg {
+  static constexpr int kTok = kGateUp ? 128 : 256;
+  static constexpr uint32_t kW = kGateUp ? 2 * kWBytes : kWBytes;
+  static constexpr uint32_t kX = static_cast<uint32_t>(kTok / 2) * kBK * 2;
+  static constexpr uint32_t kStage = kW + kX;                    // 40 KB / 32 KB
+};
 
 struct GroupedParams {
-  const int64_t* offsets;   // [G + 1] row segments, or null: one group [0, rows)
-  int64_t rows;             // rows of A (N*K routed, N shared)
+  const int64_t* offsets;   // [G + 1] token segments, or null: one group [0, rows)
+  int64_t rows;             // token rows (N*K routed, N shared)
   int G;                    // groups (experts)
   int kdim;                 // reduction length (d, or F)
-  int n_tiles;              // column blocks per row block
+  int n_tiles;              // feature blocks per token block
   int ncols;                // output row length (F for gate/up, d for down)
-  int gate_up_rows;         // gate/up: 2F (B rows per expert); down: d
+  int w_rows;               // weight rows per group: 2F (gate/up) or d (down)
   int stages;
-  int b_stream;             // 1: weights read about once (routed), evict them first
+  int w_stream;             // 1: weights read about once (routed), evict them first
   void* out;                // bf16 h [rows, F] or fp32 y [rows, d]
 };
 
@@ -71,15 +85,22 @@ struct Bars {
 };
 constexpr int kBarBytes = 8 * (2 * kMaxStages + 5);
 
-// Row-block prefix over the groups, in shared memory: mt[g] = row blocks of
-// groups before g; mt[G] = all row blocks.
+// Tokens in the tile (the MMA's N): the rows left in the group, rounded up
+// to 32, at most tok.
+__device__ __forceinline__ int tile_tokens(int64_t left, int tok) {
+  const int64_t r = (left + 31) & ~static_cast<int64_t>(31);
+  return static_cast<int>(r < tok ? r : tok);
+}
+
+// Token-block prefix over the groups, in shared memory: mt[g] = token blocks
+// of the groups before g; mt[G] = all token blocks.
 struct TileMap {
   const int32_t* mt;
   const int64_t* offsets;
   int64_t rows;
-  int G, n_tiles;
+  int G, n_tiles, tok;
   __device__ __forceinline__ int64_t total() const { return static_cast<int64_t>(mt[G]) * n_tiles; }
-  // tile -> group, first row of its pair block, rows left in the group from there, column block
+  // tile -> group, first token row of its block, rows left in the group from there, feature block
   __device__ __forceinline__ void map(int64_t tile, int& g, int64_t& row0, int64_t& left, int& n) const {
     const int mb = static_cast<int>(tile / n_tiles);
     n = static_cast<int>(tile - static_cast<int64_t>(mb) * n_tiles);
@@ -92,13 +113,13 @@ struct TileMap {
     g = lo;
     const int64_t start = offsets ? offsets[g] : 0;
     const int64_t end = offsets ? offsets[g + 1] : rows;
-    row0 = start + static_cast<int64_t>(mb - mt[g]) * kTileM;
+    row0 = start + static_cast<int64_t>(mb - mt[g]) * tok;
     left = end - row0;
   }
 };
 
 // All threads: mt[0..G] from the offsets (a block-wide exclusive scan).
-__device__ void build_tile_prefix(const GroupedParams& p, int32_t* mt, int32_t* warp_tot) {
+__device__ void build_tile_prefix(const GroupedParams& p, int tok, int32_t* mt, int32_t* warp_tot) {
   constexpr int kPer = (kMaxGroups + kThreads - 1) / kThreads;   // 3
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t v[kPer];
@@ -109,7 +130,7 @@ __device__ void build_tile_prefix(const GroupedParams& p, int32_t* mt, int32_t* 
     int32_t c = 0;
     if (g < p.G) {
       const int64_t len = p.offsets ? (p.offsets[g + 1] - p.offsets[g]) : p.rows;
-      c = static_cast<int32_t>((len + kTileM - 1) / kTileM);
+      c = static_cast<int32_t>((len + tok - 1) / tok);
     }
     v[i] = c;
     sum += c;
@@ -134,31 +155,37 @@ __device__ void build_tile_prefix(const GroupedParams& p, int32_t* mt, int32_t* 
   __syncthreads();
 }
 
-__device__ __forceinline__ float silu_f32(float g) { return g / (1.0f + __expf(-g)); }
+// SiLU(g) = g / (1 + e^-g) with the fast exponential and division (errors of
+// a few fp32 units, far below the bf16 step h is rounded to).  Large |g|:
+// e^-g -> 0 gives g; e^-g -> inf gives -0.
+__device__ __forceinline__ float silu_f32(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  const __nv_bfloat16 a = __float2bfloat16_rn(lo), b = __float2bfloat16_rn(hi);
-  return static_cast<uint32_t>(__bfloat16_as_ushort(a)) |
-         (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
-}
 
 // ---- the grouped projection ---------------------------------------------
 
-// kGateUp: A = x rows [rows, d], B = the experts' stacked [gate; up]
-// weights [G * 2F, d], out = bf16 h [rows, F]; tile column block n covers
-// hidden units [128 n, 128 n + 128).  Otherwise: A = h [rows, F], B = the
-// down weights [G * d, F], out = fp32 [rows, d]; column block n covers
-// output columns [256 n, 256 n + 256).
+// The weights are the MMA's A operand (M = 256 weight rows per pair, 128
+// per CTA) and the tokens its B operand (N = the tile's tokens, a multiple
+// of 32, half staged by each CTA), so a group's last token block costs only
+// its own rows.  TMEM lane = weight row, column = token.
+//
+// kGateUp: tokens = x rows [rows, d]; weights = the experts' [gate; up]
+// rows [G * 2F, d].  A feature block is 256 hidden units (128 per CTA): per
+// k-step one MMA takes the CTA's 128 gate rows into columns [0, 128) of the
+// accumulator buffer and one its 128 up rows into [128, 256), so a thread
+// holds both sums of its unit for every token.  out = bf16 h [rows, F].
+// Otherwise: tokens = h [rows, F]; weights = the down rows [G * d, F]; a
+// feature block is 256 output columns; out = fp32 [rows, d].
 template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
-    expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                       const __grid_constant__ CUtensorMap tm_b, const GroupedParams p) {
+    expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
+                       const __grid_constant__ CUtensorMap tm_x, const GroupedParams p) {
+  using C = Cfg<kGateUp>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int32_t mt_s[kMaxGroups + 1];
   __shared__ int32_t warp_tot[kThreads / 32];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t ring = (raw + 1023u) & ~1023u;
-  Bars bars{ring + kStageBytes * static_cast<uint32_t>(p.stages)};
+  Bars bars{ring + C::kStage * static_cast<uint32_t>(p.stages)};
   uint8_t* const holder_ptr = smem_raw + (bars.holder() - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -174,8 +201,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars.tempty(a), 2 * kEpiWarps);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_a)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_b)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_w)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_x)) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(bars.holder()),
@@ -183,39 +210,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
-  build_tile_prefix(p, mt_s, warp_tot);
+  build_tile_prefix(p, C::kTok, mt_s, warp_tot);
   tc_fence_before();
   cluster_sync();          // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(holder_ptr);
-  const TileMap tmap{mt_s, p.offsets, p.rows, p.G, p.n_tiles};
+  const TileMap tmap{mt_s, p.offsets, p.rows, p.G, p.n_tiles, C::kTok};
   const int64_t tiles = tmap.total();
   const int k_blocks = p.kdim / kBK;
 
   if (warp == 0) {
     if (lane == 0) {
-      // TMA producer of this CTA; both CTAs' copies land on the leader's full barrier
-      // A row blocks are read by every column block; routed weights about once
-      const uint64_t pol_a = policy_evict_last();
-      const uint64_t pol_b = p.b_stream ? policy_evict_first() : policy_evict_last();
+      // TMA producer of this CTA; both CTAs' copies land on the leader's full barrier.
+      // Token rows are read by every feature block; routed weights about once.
+      const uint64_t pol_x = policy_evict_last();
+      const uint64_t pol_w = p.w_stream ? policy_evict_first() : policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       for (int64_t tile = cid; tile < tiles; tile += ncl) {
-        int g, n;
+        int g, fb;
         int64_t row0, left;
-        tmap.map(tile, g, row0, left, n);
-        const int a_row = static_cast<int>(row0 + rank * kBM);
-        const int b_row = kGateUp
-            ? g * p.gate_up_rows + static_cast<int>(rank) * (p.gate_up_rows / 2) + n * kHalfN
-            : g * p.gate_up_rows + n * kTileN + static_cast<int>(rank) * kHalfN;
+        tmap.map(tile, g, row0, left, fb);
+        const int nt = tile_tokens(left, C::kTok);
+        const int x_row = static_cast<int>(row0) + static_cast<int>(rank) * (nt / 2);
+        // first weight row of this CTA (gate/up: its first gate row; the up rows are F below)
+        const int w_row = g * p.w_rows + fb * kFeat + static_cast<int>(rank) * kBM;
         bool ok = true;
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(bars.empty(stage), phase ^ 1u)) { ok = false; break; }
-          const uint32_t fb = map_to_rank(bars.full(stage), 0);
-          if (rank == 0) mbar_arrive_expect_tx(bars.full(stage), 2u * kStageBytes);
-          const uint32_t a_dst = ring + kStageBytes * stage;
-          tma_load_2d_pair(a_dst, &tm_a, kb * kBK, a_row, fb, pol_a);
-          tma_load_2d_pair(a_dst + kBM * kBK * 2, &tm_b, kb * kBK, b_row, fb, pol_b);
+          const uint32_t fbar = map_to_rank(bars.full(stage), 0);
+          if (rank == 0) mbar_arrive_expect_tx(bars.full(stage), 2u * C::kStage);
+          const uint32_t w_dst = ring + C::kStage * stage;
+          tma_load_2d_pair(w_dst, &tm_w, kb * kBK, w_row, fbar, pol_w);
+          if constexpr (kGateUp)
+            tma_load_2d_pair(w_dst + kWBytes, &tm_w, kb * kBK, w_row + p.w_rows / 2, fbar, pol_w);
+          tma_load_2d_pair(w_dst + C::kW, &tm_x, kb * kBK, x_row, fbar, pol_x);
           if (++stage == p.stages) {
             stage = 0;
             phase ^= 1u;
@@ -226,24 +255,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (rank == 0 && lane == 0) {
-      // the pair's single MMA thread: M = 256, N = 256, 4 MMAs of K = 16 per k-block
-      const uint32_t idesc = make_idesc(kTileM, kTileN);
+      // the pair's single MMA thread: M = 256 weight rows, N = the tile's tokens
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       for (int64_t tile = cid; tile < tiles; tile += ncl) {
+        int g, fb;
+        int64_t row0, left;
+        tmap.map(tile, g, row0, left, fb);
+        const uint32_t idesc = make_idesc(kFeat, tile_tokens(left, C::kTok));
         if (!mbar_wait(bars.tempty(acc), acc_phase ^ 1u)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kTileN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * 256);
         bool ok = true;
         for (int kb = 0; kb < k_blocks; ++kb) {
           if (!mbar_wait(bars.full(stage), phase)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_addr = ring + kStageBytes * stage;
-          const uint64_t a_desc = sw128_desc(a_addr);
-          const uint64_t b_desc = sw128_desc(a_addr + kBM * kBK * 2);
+          const uint32_t w_addr = ring + C::kStage * stage;
+          const uint64_t a_desc = sw128_desc(w_addr);
+          const uint64_t b_desc = sw128_desc(w_addr + C::kW);
 #pragma unroll
           for (int ks = 0; ks < kBK / 16; ++ks)
             tc_mma_pair(d_tmem, a_desc + 2u * ks, b_desc + 2u * ks, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+          if constexpr (kGateUp) {
+            const uint64_t u_desc = sw128_desc(w_addr + kWBytes);
+#pragma unroll
+            for (int ks = 0; ks < kBK / 16; ++ks)
+              tc_mma_pair(d_tmem + 128u, u_desc + 2u * ks, b_desc + 2u * ks, idesc, (kb > 0 || ks > 0) ? 1u : 0u);
+          }
           tc_commit_pair(bars.empty(stage));
           if (++stage == p.stages) {
             stage = 0;
@@ -259,53 +297,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // epilogue warps 2..5: thread = row (TMEM lane); the lane quarter is warp % 4
+    // epilogue warps 2..5: thread = weight row (TMEM lane); the lane quarter is warp % 4
     const int quarter = warp & 3;
+    const int L = quarter * 32 + lane;                 // this CTA's weight row
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int64_t tile = cid; tile < tiles; tile += ncl) {
       if (!mbar_wait(bars.tfull(acc), acc_phase)) break;
       tc_fence_after();
-      int g, n;
+      int g, fb;
       int64_t row0, left;
-      tmap.map(tile, g, row0, left, n);
-      const int64_t local = static_cast<int64_t>(rank) * kBM + quarter * 32 + lane;
-      const bool valid = local < left;
-      const int64_t row = row0 + local;
-      const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(acc * kTileN);
+      tmap.map(tile, g, row0, left, fb);
+      const int nt = tile_tokens(left, C::kTok);
+      const int valid = static_cast<int>(left < nt ? left : nt);
+      const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(acc * 256);
+      const int64_t stride = p.ncols;
       if constexpr (kGateUp) {
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.ncols + n * kHalfN;
+        const int unit = fb * kFeat + static_cast<int>(rank) * kBM + L;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row0 * stride + unit;
 #pragma unroll 1
-        for (int c = 0; c < kHalfN; c += 32) {
+        for (int c = 0; c < nt; c += 32) {
           uint32_t gr[32], ur[32];
           tmem_ld32(t0 + static_cast<uint32_t>(c), gr);
-          tmem_ld32(t0 + static_cast<uint32_t>(kHalfN + c), ur);
+          tmem_ld32(t0 + 128u + static_cast<uint32_t>(c), ur);
           tmem_wait_ld();
-          uint32_t hv[16];
+          __nv_bfloat16* o = out + c * stride;
+          const int n_ok = valid - c;                  // tokens of this chunk that are stored
+          if (n_ok >= 32) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float h0 = silu_f32(__uint_as_float(gr[2 * i])) * __uint_as_float(ur[2 * i]);
-            const float h1 = silu_f32(__uint_as_float(gr[2 * i + 1])) * __uint_as_float(ur[2 * i + 1]);
-            hv[i] = pack_bf16x2(h0, h1);
-          }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+            for (int i = 0; i < 32; ++i)
+              o[i * stride] = __float2bfloat16_rn(silu_f32(__uint_as_float(gr[i])) * __uint_as_float(ur[i]));
+          } else {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+            for (int i = 0; i < 32; ++i)
+              if (i < n_ok)
+                o[i * stride] = __float2bfloat16_rn(silu_f32(__uint_as_float(gr[i])) * __uint_as_float(ur[i]));
           }
         }
       } else {
-        float* out = static_cast<float*>(p.out) + row * p.ncols + n * kTileN;
+        float* out = static_cast<float*>(p.out) + row0 * stride + fb * kFeat + static_cast<int>(rank) * kBM + L;
 #pragma unroll 1
-        for (int c = 0; c < kTileN; c += 32) {
+        for (int c = 0; c < nt; c += 32) {
           uint32_t r[32];
           tmem_ld32(t0 + static_cast<uint32_t>(c), r);
           tmem_wait_ld();
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+          float* o = out + c * stride;
+          const int n_ok = valid - c;
+          if (n_ok >= 32) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) dst[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+            for (int i = 0; i < 32; ++i) o[i * stride] = __uint_as_float(r[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < n_ok) o[i * stride] = __uint_as_float(r[i]);
           }
         }
       }
@@ -387,8 +432,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const float4* __restrict__
 }
 
 template <bool kGateUp>
-cudaError_t launch_expert_gemm(const void* a, int64_t rows, const int64_t* offsets, int G,
-                               const void* w, void* out, int kdim, int ncols, int w_rows_per_group,
+cudaError_t launch_expert_gemm(const void* x, int64_t rows, const int64_t* offsets, int G,
+                               const void* w, void* out, int kdim, int ncols, int w_rows,
                                cudaStream_t s) {
   GroupedParams p{};
   p.offsets = offsets;
@@ -396,15 +441,16 @@ cudaError_t launch_expert_gemm(const void* a, int64_t rows, const int64_t* offse
   p.G = G;
   p.kdim = kdim;
   p.ncols = ncols;
-  p.gate_up_rows = w_rows_per_group;
-  p.n_tiles = kGateUp ? ncols / kHalfN : ncols / kTileN;
-  p.b_stream = offsets != nullptr;
+  p.w_rows = w_rows;
+  p.n_tiles = ncols / kFeat;
+  p.w_stream = offsets != nullptr;
   p.out = out;
-  CUtensorMap tm_a, tm_b;
-  if (!encode_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a, static_cast<uint64_t>(kdim),
-                 static_cast<uint64_t>(rows), kBK, kBM) ||
-      !encode_2d(&tm_b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, static_cast<uint64_t>(kdim),
-                 static_cast<uint64_t>(G) * w_rows_per_group, kBK, kHalfN))
+  using C = Cfg<kGateUp>;
+  CUtensorMap tm_w, tm_x;
+  if (!encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, static_cast<uint64_t>(kdim),
+                 static_cast<uint64_t>(rows), kBK, C::kTok / 2) ||
+      !encode_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w, static_cast<uint64_t>(kdim),
+                 static_cast<uint64_t>(G) * w_rows, kBK, kBM))
     return cudaErrorInvalidValue;
   auto kern = expert_gemm_kernel<kGateUp>;
   cudaFuncAttributes fa;
@@ -412,11 +458,11 @@ cudaError_t launch_expert_gemm(const void* a, int64_t rows, const int64_t* offse
   if (err != cudaSuccess) return err;
   const size_t fixed = 1024 /*alignment slack*/ + kBarBytes;
   const size_t avail = static_cast<size_t>(kSmemLimit) - fa.sharedSizeBytes - fixed;
-  int stages = static_cast<int>(avail / kStageBytes);
+  int stages = static_cast<int>(avail / C::kStage);
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return cudaErrorInvalidValue;
   p.stages = stages;
-  const size_t smem = fixed + static_cast<size_t>(kStageBytes) * stages;
+  const size_t smem = fixed + static_cast<size_t>(C::kStage) * stages;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
 
@@ -439,11 +485,11 @@ cudaError_t launch_expert_gemm(const void* a, int64_t rows, const int64_t* offse
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = device_sm_count() / 2;
     mc = n;
   }
-  // at most one pair per tile: row blocks <= rows / 256 + G (one partial block per group)
-  const int64_t tiles_max = ((rows + kTileM - 1) / kTileM + G) * p.n_tiles;
+  // at most one pair per tile: token blocks <= rows / 256 + G (one partial block per group)
+  const int64_t tiles_max = ((rows + C::kTok - 1) / C::kTok + G) * p.n_tiles;
   const int64_t clusters = tiles_max < mc ? tiles_max : mc;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  err = cudaLaunchKernelEx(&cfg, kern, tm_a, tm_b, p);
+  err = cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, p);
   if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
@@ -453,7 +499,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 }  // namespace
 
 bool expert_shape_supported(int32_t d, int32_t F, int32_t E) {
-  return d >= kTileN && d % kTileN == 0 && F >= kHalfN && F % kHalfN == 0 && E >= 1 &&
+  return d >= kFeat && d % kFeat == 0 && F >= kFeat && F % kFeat == 0 && E >= 1 &&
          E <= kMaxGroups && static_cast<int64_t>(E) * 2 * F < (1LL << 31) &&
          static_cast<int64_t>(E) * d < (1LL << 31);
 }

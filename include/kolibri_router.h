@@ -342,7 +342,7 @@ KOLIBRI_API kolibri_status kolibri_intervention_rate(const float *z, const int32
  *   w_gate_up [E, 2F, d]: per expert the F gate rows, then the F up rows;
  *   w_down [E, d, F]; shared expert ws_gate_up [2F, d], ws_down [d, F], or
  *   both NULL for a layer without one; y [N, d] fp32, written.
- * Shapes: d a multiple of 256, F a multiple of 128, 1 <= E <= 512,
+ * Shapes: d and F multiples of 256, 1 <= E <= 512,
  * N*K < 2^31 - 512.  Otherwise KOLIBRI_ERR_UNSUPPORTED_SHAPE.
  * ws: kolibri_expert_ffn_workspace_size(N, d, F, K, shared) bytes of device
  * memory (the gathered rows, h and the routed outputs; about

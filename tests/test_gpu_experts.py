@@ -120,8 +120,8 @@ def _assert_y_close(y, y_ref, mag):
 
 
 @pytest.mark.parametrize("N,d,F,E,K,shared,skew", [
-    (37, 256, 128, 8, 2, True, False),
-    (300, 256, 128, 16, 3, False, True),       # expert 0 spans two row blocks
+    (37, 256, 256, 8, 2, True, False),
+    (300, 256, 256, 16, 3, False, True),       # expert 0 spans several token blocks
     (700, 512, 256, 40, 4, True, True),       # three row blocks for one expert, empty experts
     (64, 2560, 512, 24, 6, True, False),      # the pages' d and F
 ])
@@ -189,8 +189,8 @@ def _pad(a, shape):
 
 def test_expert_ffn_worked_example_exact(oracle_mod):
     # the oracle's hand-added example (d = 4, F = 2), zero-padded to d = 256,
-    # F = 128: padded units have g = 0, SiLU(0) = 0, h = 0; every value is exact
-    d, F, E = 256, 128, 3
+    # F = 256: padded units have g = 0, SiLU(0) = 0, h = 0; every value is exact
+    d, F, E = 256, 256, 3
     x = _pad(np.array([[1, 2, 4, 8], [8, 4, 2, 1]], np.float32), (2, d))
     wgu = np.zeros((E, 2 * F, d), np.float32)
     wd = np.zeros((E, d, F), np.float32)
@@ -223,7 +223,7 @@ def test_expert_ffn_worked_example_exact(oracle_mod):
 def test_gate_up_rounding_midpoint_exact():
     # g = 64 (SiLU(64) = 64 in fp32), u = 1 + 2^-8: h = 64.25, the midpoint of
     # bf16 64 and 64.5 -> 64 (even); u = 1 + 2^-8 + 2^-20 -> 64.5
-    d, F = 256, 128
+    d, F = 256, 256
     wgu = np.zeros((1, 2 * F, d), np.float32)
     wgu[0, 0, :2] = 32
     wgu[0, F, :3] = [1, 2.0 ** -8, 2.0 ** -20]
