@@ -96,7 +96,7 @@ __device__ __forceinline__ int tile_tokens(int64_t left, int tok) {
 // of the groups before g; mt[G] = all token blocks.
 struct TileMap {
   const int32_t* mt;
-  const int64_t* offsets;
+  const int64_t* offsets;   // shared-memory copy of the group offsets [G + 1]
   int64_t rows;
   int G, n_tiles, tok;
   __device__ __forceinline__ int64_t total() const { return static_cast<int64_t>(mt[G]) * n_tiles; }
@@ -111,15 +111,19 @@ struct TileMap {
       else hi = mid - 1;
     }
     g = lo;
-    const int64_t start = offsets ? offsets[g] : 0;
-    const int64_t end = offsets ? offsets[g + 1] : rows;
+    const int64_t start = offsets[g];
+    const int64_t end = offsets[g + 1];
     row0 = start + static_cast<int64_t>(mb - mt[g]) * tok;
     left = end - row0;
   }
 };
 
-// All threads: mt[0..G] from the offsets (a block-wide exclusive scan).
-__device__ void build_tile_prefix(const GroupedParams& p, int tok, int32_t* mt, int32_t* warp_tot) {
+// All threads: mt[0..G] from the offsets (a block-wide exclusive scan), and
+// a shared-memory copy of the offsets (off[0..G]; without offsets: 0, rows).
+__device__ void build_tile_prefix(const GroupedParams& p, int tok, int32_t* mt, int64_t* off,
+                                  int32_t* warp_tot) {
+  for (int g = threadIdx.x; g <= p.G; g += kThreads)
+    off[g] = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.rows);
   constexpr int kPer = (kMaxGroups + kThreads - 1) / kThreads;   // 3
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t v[kPer];
@@ -182,6 +186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = Cfg<kGateUp>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ int32_t mt_s[kMaxGroups + 1];
+  __shared__ int64_t off_s[kMaxGroups + 1];
   __shared__ int32_t warp_tot[kThreads / 32];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t ring = (raw + 1023u) & ~1023u;
@@ -210,12 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
-  build_tile_prefix(p, C::kTok, mt_s, warp_tot);
+  build_tile_prefix(p, C::kTok, mt_s, off_s, warp_tot);
   tc_fence_before();
   cluster_sync();          // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(holder_ptr);
-  const TileMap tmap{mt_s, p.offsets, p.rows, p.G, p.n_tiles, C::kTok};
+  const TileMap tmap{mt_s, off_s, p.rows, p.G, p.n_tiles, C::kTok};
   const int64_t tiles = tmap.total();
   const int k_blocks = p.kdim / kBK;
 
@@ -301,10 +306,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quarter = warp & 3;
     const int L = quarter * 32 + lane;                 // this CTA's weight row
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    int acc = 0;
+    // The buffer of a tile is handed back at the start of the next tile's
+    // epilogue, not right after its last TMEM read: the arrive is a release
+    // and would otherwise wait for this warp's stores of the tile.  The MMA
+    // of tile j + 2 still never waits for the epilogue of tile j + 1.
+    int acc = 0, held = -1;
     uint32_t acc_phase = 0;
     for (int64_t tile = cid; tile < tiles; tile += ncl) {
       if (!mbar_wait(bars.tfull(acc), acc_phase)) break;
+      if (held >= 0 && lane == 0) mbar_arrive_cluster(map_to_rank(bars.tempty(held), 0));
+      held = -1;
       tc_fence_after();
       int g, fb;
       int64_t row0, left;
@@ -356,12 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_rank(bars.tempty(acc), 0));
+      held = acc;
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
       }
     }
+    if (held >= 0 && lane == 0) mbar_arrive_cluster(map_to_rank(bars.tempty(held), 0));
   }
 
   tc_fence_before();
