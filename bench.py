@@ -604,7 +604,7 @@ def run_experts(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     B.load()
-    N, d, F, E, K = args.tokens or 16384, 2560, 512, 384, 6
+    N, d, F, E, K = args.tokens or 16384, 2560, 512, args.experts or 384, 6
     g = torch.Generator(device=device)
     g.manual_seed(11)
     wgu = (torch.randn(E, 2 * F, d, generator=g, device=device) / math.sqrt(d)).to(torch.bfloat16)
@@ -681,7 +681,7 @@ def run_experts(args):
         reps += 1
     return {
         "metric": "expert layer (dispatch + grouped SwiGLU gate/up + down + combine, shared + 6 routed "
-                  "experts of 2560 -> 2x512 -> 2560, E=384): tokens/s at N=16384",
+                  f"experts of 2560 -> 2x512 -> 2560, E={E}): tokens/s at N={N}",
         "part": "experts", "value": N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "dtype": "bf16 in, fp32 accumulate", "data": "synthetic",
@@ -822,6 +822,8 @@ def main():
     ap.add_argument("--workload", default="kolibri_n1m", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--tokens", type=int, default=0,
                     help="override N (smaller captures for the profiler only)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E for --part experts (smaller captures for the profiler only)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
