@@ -780,7 +780,8 @@ def run_decode(args):
         if st != B.KOLIBRI_OK:
             raise RuntimeError(f"device status: {B.status_string(st)}")
         res["graph_us_per_layer"] = res["graph_us"] / L
-        res["gpu_launches"] = 3 * L
+        # per layer: the forward (one launch up to 96 tokens, else logits + selection), the permutation
+        res["gpu_launches"] = (2 if N <= 96 else 3) * L
         res["w_bytes_per_step"] = 2 * E * d * L
         per_n[str(n_tok)] = res
     clocks = sampler.stop()

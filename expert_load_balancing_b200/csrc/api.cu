@@ -68,9 +68,7 @@ kolibri_status kolibri_router_logits(const void* x, const void* w, float* z, int
   if (N < 1 || d < 1 || E < 1) return KOLIBRI_ERR_INVALID_ARG;
   if (d % 64 != 0 || E % 16 != 0 || E > KOLIBRI_MAX_EXPERTS) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
   if (N >= (static_cast<int64_t>(1) << 31)) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (router_small_preferred(N)) return from_cuda(launch_router_logits_small(x, w, z, N, d, E, s));
-  return from_cuda(launch_router_logits(x, w, z, N, d, E, s));
+  return from_cuda(launch_router_logits_by_size(x, w, z, N, d, E, static_cast<cudaStream_t>(stream)));
 }
 
 kolibri_status kolibri_router_forward(const void* x, const void* w, const float* bias, float* z,
@@ -250,7 +248,7 @@ kolibri_status kolibri_expert_dispatch(const void* x, const int32_t* perm, int64
                                        int32_t K, void* x_perm, void* stream) {
   if (!x || !perm || !x_perm || !aligned16(x) || !aligned16(x_perm)) return KOLIBRI_ERR_INVALID_ARG;
   if (N < 1 || K < 1 || d < 1) return KOLIBRI_ERR_INVALID_ARG;
-  if (d % 8 != 0 || N * K >= kExpertRowLimit) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (d % 8 != 0 || d > 8192 || N * K >= kExpertRowLimit) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
   return from_cuda(launch_expert_dispatch(x, perm, N, d, K, x_perm, static_cast<cudaStream_t>(stream)));
 }
 
@@ -293,7 +291,7 @@ kolibri_status kolibri_device_status(void* stream) {
   const unsigned v = status_take_api() | status_take_eqb() | status_take_noalloc() |
                      status_take_permute() | status_take_route() | status_take_logits() |
                      status_take_forward() | status_take_balance() | status_take_small() |
-                     status_take_experts();
+                     status_take_experts() | status_take_decode();
   if (v & kStatusReadFailed) return KOLIBRI_ERR_CUDA;
   if (v & kStatusTimeout) return KOLIBRI_ERR_TIMEOUT;
   if (v & kStatusBadInput) return KOLIBRI_ERR_DEVICE;

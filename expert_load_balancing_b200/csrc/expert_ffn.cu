@@ -387,7 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- dispatch and combine -------------------------------------------------
 
-// x_perm[p] = x[perm[p] / K]: a warp per row, 16-byte pieces.
+// x_perm[p] = x[perm[p] / K]: a warp per row, 16-byte pieces; each lane
+// issues all of its loads of the row (up to kDispatchPieces) before its
+// stores, so a row is one memory round trip.
+constexpr int kDispatchPieces = 16;      // 16-byte pieces per lane: rows up to 8192 bf16
 __global__ void __launch_bounds__(256) dispatch_kernel(const uint4* __restrict__ x,
                                                        const int32_t* __restrict__ perm, int64_t NK,
                                                        int K, int64_t N, int row_pieces,
@@ -403,7 +406,17 @@ __global__ void __launch_bounds__(256) dispatch_kernel(const uint4* __restrict__
     }
     const uint4* src = x + t * row_pieces;
     uint4* dst = x_perm + p * row_pieces;
-    for (int i = lane; i < row_pieces; i += 32) dst[i] = __ldg(src + i);
+    uint4 v[kDispatchPieces];
+#pragma unroll
+    for (int u = 0; u < kDispatchPieces; ++u) {
+      const int i = lane + 32 * u;
+      if (i < row_pieces) v[u] = __ldg(src + i);
+    }
+#pragma unroll
+    for (int u = 0; u < kDispatchPieces; ++u) {
+      const int i = lane + 32 * u;
+      if (i < row_pieces) dst[i] = v[u];
+    }
   }
 }
 
@@ -511,7 +524,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 }  // namespace
 
 bool expert_shape_supported(int32_t d, int32_t F, int32_t E) {
-  return d >= kFeat && d % kFeat == 0 && F >= kFeat && F % kFeat == 0 && E >= 1 &&
+  return d >= kFeat && d % kFeat == 0 && d <= 8192 && F >= kFeat && F % kFeat == 0 && E >= 1 &&
          E <= kMaxGroups && static_cast<int64_t>(E) * 2 * F < (1LL << 31) &&
          static_cast<int64_t>(E) * d < (1LL << 31);
 }
@@ -540,8 +553,9 @@ cudaError_t launch_expert_dispatch(const void* x, const int32_t* perm, int64_t N
                                    int32_t K, void* x_perm, cudaStream_t s) {
   const int64_t NK = N * K;
   const int row_pieces = d / 8;
+  if (row_pieces > 32 * kDispatchPieces) return cudaErrorInvalidValue;
   int64_t blocks = (NK + 7) / 8;
-  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 16;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
   if (blocks > cap) blocks = cap;
   dispatch_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
       static_cast<const uint4*>(x), perm, NK, K, N, row_pieces, static_cast<uint4*>(x_perm));

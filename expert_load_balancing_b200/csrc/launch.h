@@ -97,8 +97,21 @@ cudaError_t router_forward_any(const void* x, const void* w, const float* bias, 
                                int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
                                float* gates, float* alpha, cudaStream_t s);
 
-// The forward by batch size: small batches (router_small_preferred) take the
-// small logits kernel and the row kernel, the rest router_forward_any.
+// Decode batches (router_decode.cu): logits and selection in one clustered
+// launch.  Returns cudaErrorNotSupported where it does not apply.
+constexpr int64_t kDecodeTokenLimit = 96;
+bool router_decode_supported(int64_t N, int32_t d, int32_t E, int32_t K);
+cudaError_t launch_router_decode(const void* x, const void* w, const float* bias, float* z,
+                                 int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                 float* gates, float* alpha, cudaStream_t s);
+
+// The logits by batch size, with the same choice of kernel as the forward.
+cudaError_t launch_router_logits_by_size(const void* x, const void* w, float* z, int64_t N,
+                                         int32_t d, int32_t E, cudaStream_t s);
+
+// The forward by batch size: decode batches take router_decode.cu, small
+// ones (router_small_preferred) the small logits kernel and the row kernel,
+// the rest router_forward_any.
 cudaError_t router_forward_by_size(const void* x, const void* w, const float* bias, float* z,
                                    int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
                                    float* gates, float* alpha, cudaStream_t s);
@@ -157,5 +170,6 @@ unsigned status_take_forward();
 unsigned status_take_balance();
 unsigned status_take_small();
 unsigned status_take_experts();
+unsigned status_take_decode();
 
 }  // namespace kolibri

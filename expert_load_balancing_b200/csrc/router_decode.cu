@@ -1,0 +1,297 @@
+// router_decode.cu -- the whole router forward of a decode batch in one
+// launch: logits Z = x W^T, then per token the bias add, top-K, gates and
+// token bias.
+//
+// "Kolibri Pre-Training from Scratch" 6.1 (routing equations) and 7.1
+// (alpha_t = -Q_K(Z_t,: + beta)); "Kolibri 1 im Detail", routing: bf16
+// router, fp32 logits, the two-step rule (select on Z + beta, weight with
+// sigma(Z)).
+//
+// A cluster of 16 CTAs owns 16 tokens and all E experts: CTA c holds the
+// full-width router rows of experts [c E/16, (c+1) E/16) and the 16 token
+// rows in shared memory (bulk copies, one memory round trip), and its four
+// warps each form the 16 x E/16 logits over a quarter of d with mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate); the quarters are added in a fixed
+// order.  After a cluster barrier CTA r takes token r: its warp 0 reads the
+// token's E logits out of the 16 CTAs' shared memory (distributed shared
+// memory) into the lane layout of the row selection (route.cuh) and writes
+// ids, gates and alpha.  No workspace, no second launch, results repeat
+// bit for bit.  Used for batches of at most a few dozen tokens, where the
+// separate logits and selection launches are each mostly latency.
+#include <cuda_bf16.h>
+
+#include "launch.h"
+#include "route.cuh"
+#include "pdl.cuh"
+
+namespace kolibri {
+
+namespace {
+
+constexpr int kDecTok = 16;              // tokens per cluster (one m16 tile)
+constexpr int kDecCtas = 16;             // CTAs per cluster (non-portable size)
+constexpr int kDecWarps = 4;
+constexpr int kDecThreads = 32 * kDecWarps;
+
+struct DecLayout {
+  int ld;                                // padded row length of x and W rows, in bf16
+  int ec;                                // experts per CTA
+  uint32_t off_x, off_w, off_zp, off_zc, off_beta, off_sc, off_bar, total;
+};
+
+template <int Q>
+__host__ __device__ inline DecLayout dec_layout(int d, int E) {
+  DecLayout L;
+  L.ld = d + 8;                          // 16 bytes of padding: ldmatrix rows on distinct banks
+  L.ec = E / kDecCtas;
+  uint32_t o = 0;
+  L.off_x = o;
+  o += static_cast<uint32_t>(kDecTok * L.ld * 2);
+  L.off_w = o;
+  o += static_cast<uint32_t>(L.ec * L.ld * 2);
+  L.off_zp = o;
+  o += static_cast<uint32_t>(kDecWarps * kDecTok * L.ec * 4);
+  L.off_zc = o;
+  o += static_cast<uint32_t>(kDecTok * L.ec * 4);
+  L.off_beta = o;
+  o += static_cast<uint32_t>(128 * Q * 4);
+  L.off_sc = o;
+  o += static_cast<uint32_t>((sizeof(RowScratch<Q>) + 15) & ~static_cast<size_t>(15));
+  L.off_bar = o;
+  o += 16;
+  L.total = o;
+  return L;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t dec_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void dec_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ float dsmem_ld_f32(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+// One row of bytes from global memory into this CTA's shared memory,
+// completing on the mbarrier at `bar`.
+__device__ __forceinline__ void bulk_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+template <int Q, bool kBias>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_forward_kernel(
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
+    const float* __restrict__ bias, float* __restrict__ z, int64_t N, int d, int E, int K,
+    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const DecLayout L = dec_layout<Q>(d, E);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = dec_rank();
+  const int ec = L.ec, e0 = static_cast<int>(rank) * ec;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.y) * kDecTok;
+  const int nv = static_cast<int>(N - t0 < kDecTok ? N - t0 : kDecTok);   // tokens of this tile
+  const uint32_t base = smem_u32(sm);
+  const uint32_t bar = base + L.off_bar;
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sm + L.off_x);
+  float* zp = reinterpret_cast<float*>(sm + L.off_zp);
+  float* zc = reinterpret_cast<float*>(sm + L.off_zc);
+  float* beta_s = reinterpret_cast<float*>(sm + L.off_beta);
+  RowScratch<Q>& sc = *reinterpret_cast<RowScratch<Q>*>(sm + L.off_sc);
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // token rows past the batch are zero (their logits are never stored)
+  for (int i = tid; i < (kDecTok - nv) * (L.ld / 8); i += kDecThreads) {
+    const int r = nv + i / (L.ld / 8), c = i % (L.ld / 8);
+    *reinterpret_cast<uint4*>(xs + r * L.ld + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncthreads();
+  pdl_wait();                            // x may come from the kernel before this one
+  pdl_trigger();
+  if constexpr (kBias) {
+    for (int e = tid; e < 128 * Q; e += kDecThreads) beta_s[e] = e < E ? bias[e] : 0.f;
+  }
+  const uint32_t row_bytes = static_cast<uint32_t>(d) * 2;
+  if (warp == 0) {
+    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nv + ec) * row_bytes);
+    __syncwarp();
+    for (int r = lane; r < nv + ec; r += 32) {
+      if (r < nv)
+        bulk_row(base + L.off_x + static_cast<uint32_t>(r * L.ld * 2), x + (t0 + r) * d, row_bytes, bar);
+      else
+        bulk_row(base + L.off_w + static_cast<uint32_t>((r - nv) * L.ld * 2),
+                 w + static_cast<int64_t>(e0 + r - nv) * d, row_bytes, bar);
+    }
+  }
+  const bool loaded = mbar_wait(bar, 0);
+
+  // ---- logits: warp w sums k in [w d/4, (w+1) d/4)
+  if (loaded) {
+    float acc[Q][4];
+#pragma unroll
+    for (int j = 0; j < Q; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    const int kq = d / kDecWarps;
+    const int k0 = warp * kq;
+    const uint32_t a_base =
+        base + L.off_x + static_cast<uint32_t>((((lane & 7) + ((lane >> 3) & 1) * 8) * L.ld + (lane >> 4) * 8 + k0) * 2);
+    const uint32_t b_base =
+        base + L.off_w + static_cast<uint32_t>(((lane & 7) * L.ld + ((lane >> 3) & 1) * 8 + k0) * 2);
+    for (int kk = 0; kk < kq; kk += 16) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(a_base + 2u * kk, a0, a1, a2, a3);
+#pragma unroll
+      for (int j = 0; j < Q; ++j) {
+        uint32_t b0, b1;
+        ldsm_x2(b_base + static_cast<uint32_t>(8 * j * L.ld * 2) + 2u * kk, b0, b1);
+        mma16816(acc[j], a0, a1, a2, a3, b0, b1);
+      }
+    }
+    // accumulator of n tile j: rows lane/4 and lane/4 + 8, columns 8j + 2 (lane % 4) and + 1
+    float* mine = zp + warp * kDecTok * ec;
+    const int rr = lane >> 2, cc = 2 * (lane & 3);
+#pragma unroll
+    for (int j = 0; j < Q; ++j) {
+      mine[rr * ec + 8 * j + cc] = acc[j][0];
+      mine[rr * ec + 8 * j + cc + 1] = acc[j][1];
+      mine[(rr + 8) * ec + 8 * j + cc] = acc[j][2];
+      mine[(rr + 8) * ec + 8 * j + cc + 1] = acc[j][3];
+    }
+  }
+  __syncthreads();
+  if (loaded) {
+    // the four quarters in order; then Z out
+    for (int i = tid; i < kDecTok * ec; i += kDecThreads) {
+      const int n = kDecTok * ec;
+      const float v = __fadd_rn(__fadd_rn(__fadd_rn(zp[i], zp[n + i]), zp[2 * n + i]), zp[3 * n + i]);
+      zc[i] = v;
+      const int r = i / ec, c = i - r * ec;
+      if (r < nv) z[(t0 + r) * E + e0 + c] = v;
+    }
+  }
+  dec_cluster_sync();                    // every CTA's logits are in its shared memory
+
+  // ---- selection: CTA r takes token r of the tile (ids null: logits only)
+  if (ids != nullptr && warp == 0 && static_cast<int>(rank) < nv && loaded) {
+    const int64_t t = t0 + rank;
+    float zr[4 * Q];
+#pragma unroll
+    for (int j = 0; j < 4 * Q; ++j) {
+      const uint32_t e = slot_expert(lane, j);     // < 128 Q = E: E is a multiple of 128
+      const uint32_t owner = e / static_cast<uint32_t>(ec);
+      const uint32_t col = e - owner * static_cast<uint32_t>(ec);
+      zr[j] = dsmem_ld_f32(base + L.off_zc + (rank * static_cast<uint32_t>(ec) + col) * 4u, owner);
+    }
+    int rk;
+    uint32_t key, id;
+    warp_select_row<Q, true, kBias>(zr, beta_s, 0xffffffffu, K, lane, sc, rk, key, id);
+    if (rk >= 0 && rk < K) {
+      const uint32_t e = id < static_cast<uint32_t>(E) ? id : 0u;
+      ids[t * K + rk] = static_cast<int32_t>(id);
+      gates[t * K + rk] = gate_sigmoid(sc.row[buffer_pos<Q>(e)]);
+    }
+    if (rk == K && alpha) alpha[t] = -key_to_float(key);
+  }
+  dec_cluster_sync();                    // no CTA leaves while its logits may still be read
+}
+
+template <int Q, bool kBias>
+cudaError_t launch_dec(const void* x, const void* w, const float* bias, float* z, int64_t N, int d,
+                       int E, int K, int32_t* ids, float* gates, float* alpha, cudaStream_t s) {
+  const DecLayout L = dec_layout<Q>(d, E);
+  auto kern = decode_forward_kernel<Q, kBias>;
+  static int checked = 0;                // 1: runs, -1: this device cannot place the cluster
+  if (checked == 0) {
+    checked = -1;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(L.total)) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kDecCtas;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(kDecCtas, 1, 1);
+      cfg.blockDim = dim3(kDecThreads, 1, 1);
+      cfg.dynamicSmemBytes = L.total;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n >= 1) checked = 1;
+    }
+    (void)cudaGetLastError();
+  }
+  if (checked < 0) return cudaErrorNotSupported;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(L.total));
+  if (err != cudaSuccess) return err;
+  const unsigned tiles = static_cast<unsigned>((N + kDecTok - 1) / kDecTok);
+  return launch_pdl(kern, dim3(kDecCtas, tiles, 1), dim3(kDecThreads), L.total, s, dim3(kDecCtas, 1, 1),
+                    static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w), bias, z, N,
+                    d, E, K, ids, gates, alpha);
+}
+
+}  // namespace
+
+// ids, gates and alpha null: the logits alone (the same sums as the forward).
+bool router_decode_supported(int64_t N, int32_t d, int32_t E, int32_t K) {
+  if (N < 1 || N > kDecodeTokenLimit || E % 128 != 0 || E > 512 || d % 64 != 0 || K + 1 > 32) return false;
+  const int Q = E / 128;
+  const size_t total = Q == 1 ? dec_layout<1>(d, E).total
+                     : Q == 2 ? dec_layout<2>(d, E).total
+                     : Q == 3 ? dec_layout<3>(d, E).total
+                              : dec_layout<4>(d, E).total;
+  return total <= 227u * 1024u;
+}
+
+cudaError_t launch_router_decode(const void* x, const void* w, const float* bias, float* z,
+                                 int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                 float* gates, float* alpha, cudaStream_t s) {
+  if (!router_decode_supported(N, d, E, K)) return cudaErrorNotSupported;
+  const bool b = bias != nullptr;
+  switch (E / 128) {
+    case 1: return b ? launch_dec<1, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s)
+                     : launch_dec<1, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+    case 2: return b ? launch_dec<2, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s)
+                     : launch_dec<2, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+    case 3: return b ? launch_dec<3, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s)
+                     : launch_dec<3, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+    default: return b ? launch_dec<4, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s)
+                      : launch_dec<4, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+  }
+}
+
+KOLIBRI_DEFINE_STATUS_TAKE(status_take_decode)
+
+}  // namespace kolibri

@@ -215,9 +215,24 @@ cudaError_t launch_router_logits_small(const void* x, const void* w, float* z, i
   return launch_small<4, 64, 8>(xb, wb, z, N, d, E, s);
 }
 
+cudaError_t launch_router_logits_by_size(const void* x, const void* w, float* z, int64_t N,
+                                         int32_t d, int32_t E, cudaStream_t s) {
+  // the same kernel, and so the same sums, as router_forward_by_size picks
+  if (router_decode_supported(N, d, E, 1)) {
+    const cudaError_t err = launch_router_decode(x, w, nullptr, z, N, d, E, 1, nullptr, nullptr, nullptr, s);
+    if (err != cudaErrorNotSupported) return err;
+  }
+  if (router_small_preferred(N)) return launch_router_logits_small(x, w, z, N, d, E, s);
+  return launch_router_logits(x, w, z, N, d, E, s);
+}
+
 cudaError_t router_forward_by_size(const void* x, const void* w, const float* bias, float* z,
                                    int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
                                    float* gates, float* alpha, cudaStream_t s) {
+  if (router_decode_supported(N, d, E, K)) {
+    const cudaError_t err = launch_router_decode(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+    if (err != cudaErrorNotSupported) return err;
+  }
   if (router_small_preferred(N)) {
     // decode batches: the clustered logits kernel, then one row per warp
     const cudaError_t err = launch_router_logits_small(x, w, z, N, d, E, s);

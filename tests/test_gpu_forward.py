@@ -71,6 +71,43 @@ def test_forward_matches_logits_and_oracle(oracle_mod, N, d, E, K, offsets, beta
     _check(oracle_mod, workloads.make_x(wl), workloads.make_w(wl), b, K)
 
 
+# decode batches: one clustered launch (16 tokens per cluster, E a multiple of
+# 128, up to 96 tokens); 97 tokens and E = 512 at d = 2560 take the other paths
+DECODE_CASES = [
+    (1, 2560, 384, 6), (15, 2560, 384, 6), (16, 2560, 384, 6), (17, 2560, 384, 6),
+    (33, 2560, 384, 6), (64, 2560, 384, 6), (95, 2560, 384, 6), (96, 2560, 384, 6), (97, 2560, 384, 6),
+    (5, 2048, 128, 8), (40, 1024, 256, 16), (9, 1024, 512, 16), (3, 2560, 512, 6), (20, 64, 128, 1),
+]
+
+
+@pytest.mark.parametrize("N,d,E,K", DECODE_CASES)
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_forward_decode_batches(oracle_mod, N, d, E, K, with_bias):
+    wl = workloads.Workload("t", N, d, E, K, offsets="collapsed8", beta="normal0.1")
+    b = workloads.make_beta(wl).numpy() if with_bias else None
+    x, w = workloads.make_x(wl), workloads.make_w(wl)
+    _check(oracle_mod, x, w, b, K)
+    # and the logits against the oracle's sums
+    from gpu_helpers import assert_logits_close
+    z = B.kolibri_router_logits(x.cuda(), w.cuda())
+    torch.cuda.synchronize()
+    assert_logits_close(host(z), oracle_mod.router_logits(workloads.bf16_bits(x), workloads.bf16_bits(w)))
+
+
+def test_forward_decode_heavy_ties(oracle_mod):
+    # identical router rows in a decode batch: the selection's slow path
+    N, d, E, K = 40, 256, 384, 6
+    g = torch.Generator().manual_seed(12)
+    x = torch.randn(N, d, generator=g).to(torch.bfloat16)
+    x[::4] = 0
+    w = torch.randn(1, d, generator=g).repeat(E, 1)
+    w[E // 2:] = torch.randn(E - E // 2, d, generator=g)
+    w = (w / 16).to(torch.bfloat16)
+    beta = np.zeros(E, np.float32)
+    beta[::5] = 0.25
+    _check(oracle_mod, x, w, beta, K)
+
+
 def test_forward_many_tiles_per_cta(oracle_mod):
     # more 256-token tiles than SM pairs: every CTA pair loops, and the
     # per-row candidate counters are reused tile after tile
