@@ -122,8 +122,11 @@ __global__ void __launch_bounds__(kThreads, kAlphaIn ? 4 : 3) route_rows_kernel(
   for (int e = threadIdx.x; e < E; e += kThreads) {
     if constexpr (kBias) beta_s[e] = p.beta[e];
     if constexpr (kWindow) {
-      lo_s[e] = p.lo[e];
-      hi_s[e] = p.hi[e];
+      // the bracket as fp32 values: the order key is monotone in the value
+      // except that it puts -0 below +0, so against a nonzero bound a float
+      // compare decides exactly what the key compare would
+      lo_s[e] = __float_as_uint(key_to_float(p.lo[e]));
+      hi_s[e] = __float_as_uint(key_to_float(p.hi[e]));
       above_s[e] = 0u;
       stage_n[e] = 0u;
     }
@@ -134,6 +137,16 @@ __global__ void __launch_bounds__(kThreads, kAlphaIn ? 4 : 3) route_rows_kernel(
 #pragma unroll
   for (int j = 0; j < V; ++j) valid |= (static_cast<int>(slot_expert(lane, j)) < E) ? (1u << j) : 0u;
   int gate_n = 0;
+  // a lane whose brackets include a zero bound compares keys (the exact -0 < +0 order)
+  bool zero_bound = false;
+  if constexpr (kWindow) {
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if (!kFull && !(valid & (1u << j))) continue;
+      const uint32_t e = slot_expert(lane, j);
+      zero_bound |= (__uint_as_float(hi_s[e]) == 0.f) || (__uint_as_float(lo_s[e]) == 0.f);
+    }
+  }
 
   const int64_t rows_per_block = static_cast<int64_t>(kWarps) * p.rows_per_warp;
   for (int64_t base = static_cast<int64_t>(blockIdx.x) * rows_per_block; base < p.N;
@@ -198,16 +211,26 @@ __global__ void __launch_bounds__(kThreads, kAlphaIn ? 4 : 3) route_rows_kernel(
         for (int q = 0; q < Q; ++q) {
           if (!kFull && !(valid & (1u << (4 * q)))) continue;
           const int e0 = 128 * q + 4 * lane;
-          const uint4 hq = *reinterpret_cast<const uint4*>(&hi_s[e0]);
-          const uint4 lq = *reinterpret_cast<const uint4*>(&lo_s[e0]);
-          const uint32_t hv[4] = {hq.x, hq.y, hq.z, hq.w};
-          const uint32_t lv[4] = {lq.x, lq.y, lq.z, lq.w};
+          const float4 hq = *reinterpret_cast<const float4*>(&hi_s[e0]);
+          const float4 lq = *reinterpret_cast<const float4*>(&lo_s[e0]);
+          const float hv[4] = {hq.x, hq.y, hq.z, hq.w};
+          const float lv[4] = {lq.x, lq.y, lq.z, lq.w};
+          if (!zero_bound) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t k = order_key(__fadd_rn(z[4 * q + i], alpha));
-            const bool ab = k > hv[i];
-            above_b[q] += ab ? (1u << (8 * i)) : 0u;
-            wmask |= (!ab && k >= lv[i]) ? (1u << (4 * q + i)) : 0u;
+            for (int i = 0; i < 4; ++i) {
+              const float f = __fadd_rn(z[4 * q + i], alpha);
+              const bool ab = f > hv[i];
+              above_b[q] += ab ? (1u << (8 * i)) : 0u;
+              wmask |= (!ab && f >= lv[i]) ? (1u << (4 * q + i)) : 0u;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint32_t k = order_key(__fadd_rn(z[4 * q + i], alpha));
+              const bool ab = k > order_key(hv[i]);
+              above_b[q] += ab ? (1u << (8 * i)) : 0u;
+              wmask |= (!ab && k >= order_key(lv[i])) ? (1u << (4 * q + i)) : 0u;
+            }
           }
         }
         while (wmask) {  // rare: keys inside the bracket
