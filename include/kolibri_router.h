@@ -361,7 +361,8 @@ KOLIBRI_API kolibri_status kolibri_expert_ffn(const void *x, const int32_t *perm
 
 /*
  * The four stages of kolibri_expert_ffn, each callable on its own:
- *   kolibri_expert_dispatch: x_perm [N*K, d] with x_perm[p] = x[perm[p] / K].
+ *   kolibri_expert_dispatch: x_perm [N*K, d] with x_perm[p] = x[perm[p] / K]
+ *     (d a multiple of 8, at most 8192).
  *   kolibri_expert_gate_up: h [rows, F] bf16 = bf16(SiLU(a Wg^T) * (a Wu^T))
  *     where rows [offsets[g], offsets[g+1]) of a [rows, d] use expert g of
  *     w_gate_up [G, 2F, d]; offsets NULL: one group of all rows (G = 1).
