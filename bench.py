@@ -474,6 +474,8 @@ PARTS = {
                  lambda E, K: 4 * E + 4, "Z and alpha read once"),
     "eqb_bf16_split": ("EQB with bf16 keys, the two histogram passes of the multi-rank form, one rank",
                        lambda E, K: 8 * E + 8, "Z and alpha read twice"),
+    "eqb_fp32_split": ("EQB with fp32 keys, the four histogram passes of the multi-rank form, one rank",
+                       lambda E, K: 16 * E + 16, "Z and alpha read four times"),
     "lei": ("Load-Error Injection on the [N, E] score gradient",
             lambda E, K: 8 * E, "G read and written"),
     "score_grad": ("chain rule from the score gradient to the logits",
@@ -514,6 +516,10 @@ def run_part(args):
             step.beta.copy_(beta0)
             with torch.cuda.stream(stream):
                 D.eqb_update_bf16_distributed(step.z, step.alpha, step.beta, K, N, quantiles=q)
+        elif args.part == "eqb_fp32_split":
+            step.beta.copy_(beta0)
+            with torch.cuda.stream(stream):
+                D.eqb_update_distributed(step.z, step.alpha, step.beta, K, N, quantiles=q)
         elif args.part == "lei":
             B.kolibri_lei_inject(step.counts, gs, K, stream=stream)
         elif args.part == "score_grad":
@@ -545,10 +551,12 @@ def run_part(args):
     bytes_ = bpt(E, K) * N
     achieved = bytes_ / (ms * 1e-3) / 1e9
     # the oracle on the first rows of the same data
-    n = min(N, 4096 if args.part in ("eqb_bf16", "eqb_bf16_split") else 2048)
+    n = min(N, 4096 if args.part.startswith("eqb") else 2048)
     zh = step.z[:n].cpu().numpy()
     t = time.time()
-    if args.part in ("eqb_bf16", "eqb_bf16_split"):
+    if args.part == "eqb_fp32_split":
+        oracle.column_quantiles(zh, step.alpha[:n].cpu().numpy(), (n * K) // E)
+    elif args.part in ("eqb_bf16", "eqb_bf16_split"):
         oracle.column_quantiles_bf16(zh, step.alpha[:n].cpu().numpy(), (n * K) // E)
     elif args.part == "lei":
         oracle.lei_inject(step.counts.cpu().numpy(), gs[:n].cpu().numpy(), K)
@@ -561,7 +569,9 @@ def run_part(args):
     cpu_s = time.time() - t
     while cpu_s < 2.0:                 # repeat the sample to about 2 s of CPU work
         t = time.time()
-        if args.part in ("eqb_bf16", "eqb_bf16_split"):
+        if args.part == "eqb_fp32_split":
+            oracle.column_quantiles(zh, step.alpha[:n].cpu().numpy(), (n * K) // E)
+        elif args.part in ("eqb_bf16", "eqb_bf16_split"):
             oracle.column_quantiles_bf16(zh, step.alpha[:n].cpu().numpy(), (n * K) // E)
         elif args.part == "lei":
             oracle.lei_inject(step.counts.cpu().numpy(), gs[:n].cpu().numpy(), K)

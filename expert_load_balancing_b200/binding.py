@@ -49,6 +49,9 @@ SIGNATURES = {
     "kolibri_eqb_update": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P, _P, _SZ, _P]),
     "kolibri_route_and_balance": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P, _P,
                                                  _SZ, _P]),
+    "kolibri_eqb_key_histogram": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P]),
+    "kolibri_eqb_key_digit": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P]),
+    "kolibri_eqb_key_bias": (ctypes.c_int, [_P, _I32, _P, _P, _P]),
     "kolibri_expert_ffn_workspace_size": (_SZ, [_I64, _I32, _I32, _I32, _I32]),
     "kolibri_expert_ffn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32, _I32,
                                           _I32, _I32, _P, _SZ, _P]),
@@ -372,6 +375,30 @@ def kolibri_eqb_bf16_bias(d_hi, d_lo, bias, quantiles, stream=None):
     _check("kolibri_eqb_bf16_bias",
            load().kolibri_eqb_bf16_bias(_ptr(d_hi), _ptr(d_lo), E, _ptr(bias), _ptr(quantiles),
                                         _stream(stream)))
+    return bias, quantiles
+
+
+def kolibri_eqb_key_histogram(z, alpha, pass_, prefix, hist, stream=None):
+    """Add this rank's fp32-key histogram of digit pass pass_ (0..3) into hist [E, 256] uint32."""
+    N, E = z.shape
+    _check("kolibri_eqb_key_histogram",
+           load().kolibri_eqb_key_histogram(_ptr(z), _ptr(alpha), N, E, int(pass_), _ptr(prefix),
+                                            _ptr(hist), _stream(stream)))
+    return hist
+
+
+def kolibri_eqb_key_digit(hist, pass_, rank, prefix, stream=None):
+    E = hist.shape[0]
+    _check("kolibri_eqb_key_digit",
+           load().kolibri_eqb_key_digit(_ptr(hist), E, int(pass_), _ptr(rank), _ptr(prefix),
+                                        _stream(stream)))
+    return prefix
+
+
+def kolibri_eqb_key_bias(key, bias, quantiles, stream=None):
+    E = bias.shape[0]
+    _check("kolibri_eqb_key_bias",
+           load().kolibri_eqb_key_bias(_ptr(key), E, _ptr(bias), _ptr(quantiles), _stream(stream)))
     return bias, quantiles
 
 

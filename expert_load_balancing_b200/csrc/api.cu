@@ -190,6 +190,32 @@ kolibri_status kolibri_eqb_bf16_bias(const uint32_t* digit_hi, const uint32_t* d
   return from_cuda(launch_bias_update(quantiles, E, bias, quantiles, s));
 }
 
+kolibri_status kolibri_eqb_key_histogram(const float* z, const float* alpha, int64_t N, int32_t E,
+                                         int32_t pass, const uint32_t* prefix, uint32_t* hist,
+                                         void* stream) {
+  if (N < 1 || pass < 0 || pass > 3) return KOLIBRI_ERR_INVALID_ARG;
+  if (E < 4 || E > KOLIBRI_MAX_EXPERTS || (E % 4) != 0) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (!z || !hist || !aligned16(z) || (pass > 0 && !prefix)) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_key_hist(z, alpha, N, E, pass, prefix, hist, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_key_digit(const uint32_t* hist, int32_t E, int32_t pass, int64_t* rank,
+                                     uint32_t* prefix, void* stream) {
+  if (E < 1 || E > KOLIBRI_MAX_EXPERTS) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (!hist || !rank || !prefix || pass < 0 || pass > 3) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_key_digit(hist, E, pass, rank, prefix, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_key_bias(const uint32_t* key, int32_t E, float* bias, float* quantiles,
+                                    void* stream) {
+  if (E < 1 || E > KOLIBRI_MAX_EXPERTS) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (!key || !bias || !quantiles) return KOLIBRI_ERR_INVALID_ARG;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t err = launch_key_value(key, E, quantiles, s);
+  if (err != cudaSuccess) return KOLIBRI_ERR_CUDA;
+  return from_cuda(launch_bias_update(quantiles, E, bias, quantiles, s));
+}
+
 kolibri_status kolibri_lei_inject(const int32_t* counts, int64_t N, int32_t E, int32_t K,
                                   double lambda, double tau, float* g, void* stream) {
   kolibri_status st = check_ek(N, E, K);

@@ -7,6 +7,9 @@
 //     the keys in that bin and reads off the exact key.  The histograms are
 //     the only thing that crosses ranks in a distributed batch (one
 //     all-reduce of 256 E counts per pass), so each pass is its own call.
+//   * The same two-pass-per-byte scheme on the fp32 keys of the main update
+//     (four passes), so that update too can run over a batch split across
+//     ranks with only histograms crossing.
 //   * Load-Error Injection (section 8): per-expert load error rho from the
 //     microbatch counts, xi = |rho|_inf / tau, and G += lambda tanh(xi)/xi rho
 //     on every token's score gradient; and the chain rule to the logits,
@@ -125,6 +128,95 @@ __global__ void bf16_value_kernel(const uint32_t* __restrict__ d_hi, const uint3
   const uint32_t k = ((d_hi[e] & 0xffu) << 8) | (d_lo[e] & 0xffu);
   const uint32_t b = (k & 0x8000u) ? (k & 0x7fffu) : (~k & 0xffffu);
   v[e] = __uint_as_float(b << 16);
+}
+
+// The same radix selection on the fp32 keys of the main update (the order
+// key of Z + alpha), four passes of 8-bit digits from the top: pass p bins
+// byte 3 - p of the keys whose top 8p bits equal prefix[e] (the digits of the
+// earlier passes).  As above, only the histograms cross ranks.
+__global__ void __launch_bounds__(kHistThreads) key_hist_kernel(
+    const float* __restrict__ z, const float* __restrict__ alpha, int64_t N, int E, int pass,
+    const uint32_t* __restrict__ prefix, uint32_t* __restrict__ hist) {
+  extern __shared__ uint32_t hist_smem[];
+  uint32_t* h = hist_smem;                               // [64][256], 64 KB
+  uint32_t* pre_s = hist_smem + kColsPerCta * kBins;     // [64]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int col0 = blockIdx.y * kColsPerCta;
+  const int shift = 24 - 8 * pass;                       // this pass's byte
+  for (int i = threadIdx.x; i < kColsPerCta * kBins; i += kHistThreads) h[i] = 0u;
+  for (int i = threadIdx.x; i < kColsPerCta; i += kHistThreads)
+    pre_s[i] = (pass > 0 && col0 + i < E) ? prefix[col0 + i] : 0u;
+  __syncthreads();
+  const int c4 = 2 * lane;
+  const bool active = col0 + c4 < E;
+  // keys match when their bits above this pass's byte equal the prefix's
+  const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
+  uint32_t pre[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) pre[i] = pre_s[(c4 + i) & (kColsPerCta - 1)] & hi_mask;
+  const int64_t rows_per_block = static_cast<int64_t>(kHistThreads / 32);
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * rows_per_block + warp; t < N;
+       t += static_cast<int64_t>(gridDim.x) * rows_per_block) {
+    if (!active) continue;
+    const float a = alpha ? __ldg(alpha + t) : 0.f;
+    const float2 v = __ldcs(reinterpret_cast<const float2*>(z + t * E + col0 + c4));
+    const float vv[2] = {v.x, v.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const uint32_t k = order_key(__fadd_rn(vv[i], a));
+      if ((k & hi_mask) == pre[i]) atomicAdd(&h[(c4 + i) * kBins + ((k >> shift) & 0xffu)], 1u);
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kColsPerCta * kBins; i += kHistThreads) {
+    const int c = i / kBins;
+    if (col0 + c < E && h[i]) atomicAdd(hist + static_cast<int64_t>(col0 + c) * kBins + (i % kBins), h[i]);
+  }
+}
+
+// Per expert: this pass's digit (as bf16_digit_kernel), then the prefix
+// gains it as byte 3 - pass (pass 0 starts the prefix).
+__global__ void key_digit_kernel(const uint32_t* __restrict__ hist, int E, int pass,
+                                 int64_t* __restrict__ rank, uint32_t* __restrict__ prefix) {
+  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (e >= E) return;
+  const uint32_t* he = hist + static_cast<int64_t>(e) * kBins;
+  uint32_t c[8];
+  uint64_t sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = he[255 - (8 * lane + i)];
+    sum += c[i];
+  }
+  uint64_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  uint64_t above = incl - sum;
+  const int64_t r = rank[e];
+  const bool mine = static_cast<int64_t>(above) <= r && r < static_cast<int64_t>(incl);
+  const uint32_t who = __ballot_sync(0xffffffffu, mine);
+  const int shift = 24 - 8 * pass;
+  if (mine) {
+    int i = 0;
+    while (i < 7 && static_cast<int64_t>(above + c[i]) <= r) {
+      above += c[i];
+      ++i;
+    }
+    const uint32_t dgt = static_cast<uint32_t>(255 - (8 * lane + i));
+    const uint32_t keep = pass == 0 ? 0u : (prefix[e] & (0xffffffffu << (shift + 8)));
+    prefix[e] = keep | (dgt << shift);
+    rank[e] = r - static_cast<int64_t>(above);
+  }
+  if (who == 0u && lane == 0) raise_status(kStatusBadInput);   // rank past the column
+}
+
+__global__ void key_value_kernel(const uint32_t* __restrict__ key, int E, float* __restrict__ v) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < E) v[e] = key_to_float(key[e]);
 }
 
 // rho_e = c_e / (K N / E) - 1, xi = max |rho| / tau, delta_e = lambda *
@@ -281,6 +373,35 @@ cudaError_t launch_bf16_digit(const uint32_t* hist, int32_t E, int64_t* rank, ui
 cudaError_t launch_bf16_value(const uint32_t* d_hi, const uint32_t* d_lo, int32_t E, float* v,
                               cudaStream_t s) {
   bf16_value_kernel<<<(E + 255) / 256, 256, 0, s>>>(d_hi, d_lo, E, v);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_key_hist(const float* z, const float* alpha, int64_t N, int32_t E, int32_t pass,
+                            const uint32_t* prefix, uint32_t* hist, cudaStream_t s) {
+  const int groups = (E + kColsPerCta - 1) / kColsPerCta;
+  int per_group = 3 * device_sm_count() / groups;
+  if (per_group < 1) per_group = 1;
+  const int64_t rows_per_block = kHistThreads / 32;
+  int64_t gx = (N + rows_per_block - 1) / rows_per_block;
+  if (gx > per_group) gx = per_group;
+  const int smem = static_cast<int>(sizeof(uint32_t) * (kColsPerCta * kBins + kColsPerCta));
+  cudaError_t err =
+      cudaFuncSetAttribute(key_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (err != cudaSuccess) return err;
+  key_hist_kernel<<<dim3(static_cast<unsigned>(gx), static_cast<unsigned>(groups)), kHistThreads, smem,
+                    s>>>(z, alpha, N, E, pass, prefix, hist);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_key_digit(const uint32_t* hist, int32_t E, int32_t pass, int64_t* rank,
+                             uint32_t* prefix, cudaStream_t s) {
+  const int warps = 8;
+  key_digit_kernel<<<(E + warps - 1) / warps, 32 * warps, 0, s>>>(hist, E, pass, rank, prefix);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_key_value(const uint32_t* key, int32_t E, float* v, cudaStream_t s) {
+  key_value_kernel<<<(E + 255) / 256, 256, 0, s>>>(key, E, v);
   return cudaGetLastError();
 }
 

@@ -160,6 +160,13 @@ cudaError_t launch_intervention(const float* z, const int32_t* ids, int64_t N, i
 int device_sm_count();
 
 // Read and clear the status word of one translation unit (see common.cuh).
+// fp32-key radix passes of the EQB quantile over a split batch (balance.cu).
+cudaError_t launch_key_hist(const float* z, const float* alpha, int64_t N, int32_t E, int32_t pass,
+                            const uint32_t* prefix, uint32_t* hist, cudaStream_t s);
+cudaError_t launch_key_digit(const uint32_t* hist, int32_t E, int32_t pass, int64_t* rank,
+                             uint32_t* prefix, cudaStream_t s);
+cudaError_t launch_key_value(const uint32_t* key, int32_t E, float* v, cudaStream_t s);
+
 unsigned status_take_api();
 unsigned status_take_eqb();
 unsigned status_take_noalloc();

@@ -290,6 +290,35 @@ KOLIBRI_API kolibri_status kolibri_eqb_bf16_bias(const uint32_t *digit_hi,
                                                  float *bias, float *quantiles, void *stream);
 
 /*
+ * The EQB quantile of kolibri_eqb_update (fp32 keys) over a batch split
+ * across ranks: the same radix selection in four passes of 8-bit digits
+ * (the design of the pages' section 7.3 applied to the 32-bit order key of
+ * Z + alpha, so the result is the exact fp32 quantile of the union, equal to
+ * kolibri_eqb_update's on one rank).
+ *   kolibri_eqb_key_histogram: pass p (0..3) adds to hist [E][256] (uint32,
+ *     zeroed by the caller before each pass) the count of keys, per expert
+ *     and byte 3 - p, among the keys whose top 8p bits equal prefix[e] (the
+ *     digits so far; prefix is not read at pass 0).  alpha may be NULL (0).
+ *   kolibri_eqb_key_digit: per expert, the bin holding the rank[e]-th
+ *     largest key (0-based; start with rank[e] = m = floor(N_total K / E));
+ *     writes it into prefix[e] as byte 3 - p (pass 0 overwrites prefix) and
+ *     subtracts the keys of the bins above it from rank[e].  A rank past the
+ *     column sets KOLIBRI_ERR_DEVICE.
+ *   kolibri_eqb_key_bias: v_e from the finished key, written to quantiles
+ *     [E] (required), then bias = -v, centred.
+ * Sequence per update: for p = 0..3 { zero hist; histogram(p); all-reduce
+ * hist; digit(p) }; bias.  On one rank the all-reduces are skipped.
+ */
+KOLIBRI_API kolibri_status kolibri_eqb_key_histogram(const float *z, const float *alpha, int64_t N,
+                                                     int32_t E, int32_t pass,
+                                                     const uint32_t *prefix, uint32_t *hist,
+                                                     void *stream);
+KOLIBRI_API kolibri_status kolibri_eqb_key_digit(const uint32_t *hist, int32_t E, int32_t pass,
+                                                 int64_t *rank, uint32_t *prefix, void *stream);
+KOLIBRI_API kolibri_status kolibri_eqb_key_bias(const uint32_t *key, int32_t E, float *bias,
+                                                float *quantiles, void *stream);
+
+/*
  * Load-Error Injection ("Kolibri Pre-Training from Scratch" 8) on the score
  * gradient of one microbatch of N tokens:
  *   f_e = counts[e] / (K N / E), rho_e = f_e - 1, xi = max_e |rho_e| / tau,

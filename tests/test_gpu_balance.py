@@ -79,6 +79,24 @@ def test_eqb_bf16_pieces_equal_one_call(oracle_mod):
     assert_bit_equal(host(b2), host(b1), "beta")
 
 
+@pytest.mark.parametrize("N,E,K,ties", [(1, 16, 2, False), (5000, 384, 6, False), (20000, 384, 6, True),
+                                        (4099, 128, 8, True), (777, 400, 6, False)])
+def test_eqb_fp32_key_passes_equal_one_call(oracle_mod, N, E, K, ties):
+    # the four fp32-key passes of the split form, on one rank (no all-reduce),
+    # give kolibri_eqb_update's exact quantile and bias bit for bit
+    z, a = _column_data(N, E, N + 3 * E, ties=ties)
+    zt, at = dev(z), dev(a)
+    b1 = dev(np.zeros(E, np.float32))
+    _, q1 = B.kolibri_eqb_update(zt, at, b1, K)
+    b2 = dev(np.zeros(E, np.float32))
+    _, q2 = D.eqb_update_distributed(zt, at, b2, K, N)
+    torch.cuda.synchronize()
+    check_status()
+    assert_bit_equal(host(q2), host(q1), "quantiles")
+    assert_bit_equal(host(b2), host(b1), "beta")
+    assert_bit_equal(host(q2), oracle_mod.column_quantiles(z, a, (N * K) // E), "oracle")
+
+
 def test_lei_pages_example(oracle_mod):
     # section 8: loads (4, 4, 0, 0), K = 2, four tokens
     counts = dev(np.array([4, 4, 0, 0], np.int32))

@@ -1,6 +1,7 @@
-"""EQB with bf16 keys over a batch split across ranks ("Kolibri Pre-Training
-from Scratch" 7.3): expert_load_balancing_b200.distributed sums the per-rank
-256-bin histograms with an all-reduce between the two passes.  Run here with
+"""EQB over a batch split across ranks ("Kolibri Pre-Training from Scratch"
+7.3): expert_load_balancing_b200.distributed sums the per-rank 256-bin
+histograms with an all-reduce between the passes (two for the pages' bf16
+keys, four for the fp32 keys of the main update).  Run here with
 two and three gloo ranks on the CPU; the three library calls are replaced by
 CPU stand-ins built from the oracle's bf16 rounding and key (the GPU kernels
 behind them are checked against the oracle in test_gpu_balance.py).  Every
@@ -74,7 +75,50 @@ class _CpuOps:
         return bias, quantiles
 
 
-def _worker(rank, world, port, z_parts, a_parts, K, out):
+class _CpuKeyOps:
+    """The three per-rank calls of the fp32-key passes on the CPU (test stand-ins)."""
+
+    def __init__(self, oracle):
+        self.o = oracle
+
+    def histogram(self, z, alpha, p, prefix, hist):
+        zz = z.numpy()
+        a = np.zeros(zz.shape[0], np.float32) if alpha is None else alpha.numpy()
+        keys = self.o.order_key_array((zz + a[:, None]).astype(np.float32)).astype(np.int64)
+        shift = 24 - 8 * p
+        for e in range(keys.shape[1]):
+            k = keys[:, e]
+            if p:
+                hi = (0xffffffff << (shift + 8)) & 0xffffffff
+                k = k[(k & hi) == (int(prefix[e]) & 0xffffffff & hi)]
+            hist[e] += torch.from_numpy(np.bincount((k >> shift) & 0xff, minlength=256).astype(np.int32))
+        return hist
+
+    def digit(self, hist, p, rank, prefix):
+        shift = 24 - 8 * p
+        for e in range(hist.shape[0]):
+            r = int(rank[e])
+            above = 0
+            for b in range(255, -1, -1):
+                c = int(hist[e, b])
+                if above + c > r:
+                    keep = 0 if p == 0 else (int(prefix[e]) & 0xffffffff) & ((0xffffffff << (shift + 8)) & 0xffffffff)
+                    prefix[e] = np.int64(keep | (b << shift)).astype(np.uint32).view(np.int32)
+                    rank[e] = r - above
+                    break
+                above += c
+        return prefix
+
+    def bias(self, key, bias, quantiles):
+        k = key.numpy().view(np.uint32)
+        u = np.where(k & 0x80000000, k & 0x7fffffff, ~k & 0xffffffff).astype(np.uint32)
+        v = u.view(np.float32)
+        quantiles.copy_(torch.from_numpy(v.copy()))
+        bias.copy_(torch.from_numpy(self.o.eqb_bias(v)))
+        return bias, quantiles
+
+
+def _worker(rank, world, port, z_parts, a_parts, K, out, fp32=False):
     import sys
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -89,19 +133,22 @@ def _worker(rank, world, port, z_parts, a_parts, K, out):
         a = torch.from_numpy(a_parts[rank])
         n_total = sum(p.shape[0] for p in z_parts)
         bias = torch.zeros(z.shape[1])
-        _, q = D.eqb_update_bf16_distributed(z, a, bias, K, n_total, ops=_CpuOps(oracle))
+        if fp32:
+            _, q = D.eqb_update_distributed(z, a, bias, K, n_total, ops=_CpuKeyOps(oracle))
+        else:
+            _, q = D.eqb_update_bf16_distributed(z, a, bias, K, n_total, ops=_CpuOps(oracle))
         out[rank] = (q.numpy().copy(), bias.numpy().copy())
     finally:
         dist.destroy_process_group()
 
 
-def _run(z_parts, a_parts, K):
+def _run(z_parts, a_parts, K, fp32=False):
     ctx = mp.get_context("spawn")
     manager = ctx.Manager()
     out = manager.dict()
     port = _free_port()
     world = len(z_parts)
-    procs = [ctx.Process(target=_worker, args=(r, world, port, z_parts, a_parts, K, out))
+    procs = [ctx.Process(target=_worker, args=(r, world, port, z_parts, a_parts, K, out, fp32))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -137,6 +184,37 @@ def test_three_ranks_equal_the_union(oracle_mod):
     a = np.concatenate(a_parts)
     m = (z.shape[0] * K) // E
     v = oracle_mod.column_quantiles_bf16(z, a, m)
+    for q, b in res:
+        np.testing.assert_array_equal(q, v)
+        np.testing.assert_array_equal(b, oracle_mod.eqb_bias(v))
+
+
+def test_fp32_keys_pages_counter_example(oracle_mod):
+    # the same counter-example through the fp32-key passes of the main update
+    za = np.array([[3.0, 0.0], [1.5, 0.0]], np.float32)
+    zb = np.array([[0.5, 0.0], [3.0, 0.0]], np.float32)
+    zero = np.zeros(2, np.float32)
+    res = _run([za, zb], [zero, zero], K=1, fp32=True)
+    for q, b in res:
+        assert q[0] == np.float32(1.5)
+    np.testing.assert_array_equal(res[0][1], res[1][1])
+
+
+def test_fp32_keys_three_ranks_equal_the_union(oracle_mod):
+    rng = np.random.default_rng(1)
+    E, K = 8, 3
+    sizes = [23, 11, 40]
+    z_parts = [(rng.standard_normal((n, E)) * 2).astype(np.float32) for n in sizes]
+    z_parts[0][:, 1] = -0.0                           # signed zeros and ties across ranks
+    z_parts[2][:5, 1] = 0.0
+    z_parts[1][:, 4] = 0.75
+    a_parts = [(rng.standard_normal(n) * 0.3).astype(np.float32) for n in sizes]
+    a_parts[0][:] = 0.0
+    res = _run(z_parts, a_parts, K, fp32=True)
+    z = np.concatenate(z_parts)
+    a = np.concatenate(a_parts)
+    m = (z.shape[0] * K) // E
+    v = oracle_mod.column_quantiles(z, a, m)
     for q, b in res:
         np.testing.assert_array_equal(q, v)
         np.testing.assert_array_equal(b, oracle_mod.eqb_bias(v))
