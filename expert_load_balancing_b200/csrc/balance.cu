@@ -27,6 +27,12 @@ namespace {
 
 constexpr int kBins = 256;
 constexpr int kColsPerCta = 64;          // a lane owns two columns of the group
+// A column's bins sit kBinLd words apart in shared memory: with 256 every
+// lane's column would start in the same bank, and the lanes of a warp (all
+// on different columns, mostly on the same bin) would serialise their
+// atomics 32-fold.
+constexpr int kBinLd = kBins + 1;
+constexpr int kRowBatch = 8;             // rows a warp loads before counting them
 constexpr int kHistThreads = 256;
 
 __device__ __forceinline__ uint32_t bf16_key_of(float z, float a) {
@@ -44,11 +50,11 @@ __global__ void __launch_bounds__(kHistThreads) bf16_hist_kernel(
     const float* __restrict__ z, const float* __restrict__ alpha, int64_t N, int E,
     const uint32_t* __restrict__ prefix, uint32_t* __restrict__ hist) {
   extern __shared__ uint32_t hist_smem[];
-  uint32_t* h = hist_smem;                               // [64][256], 64 KB
-  uint32_t* pre_s = hist_smem + kColsPerCta * kBins;     // [64]
+  uint32_t* h = hist_smem;                               // [64][kBinLd], 64 KB
+  uint32_t* pre_s = hist_smem + kColsPerCta * kBinLd;    // [64]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int col0 = blockIdx.y * kColsPerCta;
-  for (int i = threadIdx.x; i < kColsPerCta * kBins; i += kHistThreads) h[i] = 0u;
+  for (int i = threadIdx.x; i < kColsPerCta * kBinLd; i += kHistThreads) h[i] = 0u;
   for (int i = threadIdx.x; i < kColsPerCta; i += kHistThreads)
     pre_s[i] = (prefix && col0 + i < E) ? prefix[col0 + i] : 0u;
   __syncthreads();
@@ -57,27 +63,39 @@ __global__ void __launch_bounds__(kHistThreads) bf16_hist_kernel(
   uint32_t pre[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) pre[i] = pre_s[(c4 + i) & (kColsPerCta - 1)];
-  const int64_t rows_per_block = static_cast<int64_t>(kHistThreads / 32);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * rows_per_block + warp; t < N;
-       t += static_cast<int64_t>(gridDim.x) * rows_per_block) {
+  // a warp takes kRowBatch rows at a time and issues all their loads first
+  const int64_t rows_per_block = static_cast<int64_t>(kHistThreads / 32) * kRowBatch;
+  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * rows_per_block + warp * kRowBatch; t0 < N;
+       t0 += static_cast<int64_t>(gridDim.x) * rows_per_block) {
     if (!active) continue;
-    const float a = alpha ? __ldg(alpha + t) : 0.f;
-    const float2 v = __ldcs(reinterpret_cast<const float2*>(z + t * E + col0 + c4));
-    const float vv[2] = {v.x, v.y};
+    float2 v[kRowBatch];
+    float a[kRowBatch];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t k = alpha ? bf16_key_of(vv[i], a) : bf16_key_of(vv[i], 0.f);
-      if (prefix == nullptr) {
-        atomicAdd(&h[(c4 + i) * kBins + (k >> 8)], 1u);
-      } else if ((k >> 8) == pre[i]) {
-        atomicAdd(&h[(c4 + i) * kBins + (k & 0xffu)], 1u);
+    for (int r = 0; r < kRowBatch; ++r) {
+      const int64_t t = t0 + r < N ? t0 + r : N - 1;
+      a[r] = alpha ? __ldg(alpha + t) : 0.f;
+      v[r] = __ldcs(reinterpret_cast<const float2*>(z + t * E + col0 + c4));
+    }
+#pragma unroll
+    for (int r = 0; r < kRowBatch; ++r) {
+      if (t0 + r >= N) break;
+      const float vv[2] = {v[r].x, v[r].y};
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t k = bf16_key_of(vv[i], a[r]);
+        if (prefix == nullptr) {
+          atomicAdd(&h[(c4 + i) * kBinLd + (k >> 8)], 1u);
+        } else if ((k >> 8) == pre[i]) {
+          atomicAdd(&h[(c4 + i) * kBinLd + (k & 0xffu)], 1u);
+        }
       }
     }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kColsPerCta * kBins; i += kHistThreads) {
-    const int c = i / kBins;
-    if (col0 + c < E && h[i]) atomicAdd(hist + static_cast<int64_t>(col0 + c) * kBins + (i % kBins), h[i]);
+    const int c = i / kBins, b = i % kBins;
+    const uint32_t n = h[c * kBinLd + b];
+    if (col0 + c < E && n) atomicAdd(hist + static_cast<int64_t>(col0 + c) * kBins + b, n);
   }
 }
 
@@ -138,12 +156,12 @@ __global__ void __launch_bounds__(kHistThreads) key_hist_kernel(
     const float* __restrict__ z, const float* __restrict__ alpha, int64_t N, int E, int pass,
     const uint32_t* __restrict__ prefix, uint32_t* __restrict__ hist) {
   extern __shared__ uint32_t hist_smem[];
-  uint32_t* h = hist_smem;                               // [64][256], 64 KB
-  uint32_t* pre_s = hist_smem + kColsPerCta * kBins;     // [64]
+  uint32_t* h = hist_smem;                               // [64][kBinLd], 64 KB
+  uint32_t* pre_s = hist_smem + kColsPerCta * kBinLd;    // [64]
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int col0 = blockIdx.y * kColsPerCta;
   const int shift = 24 - 8 * pass;                       // this pass's byte
-  for (int i = threadIdx.x; i < kColsPerCta * kBins; i += kHistThreads) h[i] = 0u;
+  for (int i = threadIdx.x; i < kColsPerCta * kBinLd; i += kHistThreads) h[i] = 0u;
   for (int i = threadIdx.x; i < kColsPerCta; i += kHistThreads)
     pre_s[i] = (pass > 0 && col0 + i < E) ? prefix[col0 + i] : 0u;
   __syncthreads();
@@ -154,23 +172,34 @@ __global__ void __launch_bounds__(kHistThreads) key_hist_kernel(
   uint32_t pre[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) pre[i] = pre_s[(c4 + i) & (kColsPerCta - 1)] & hi_mask;
-  const int64_t rows_per_block = static_cast<int64_t>(kHistThreads / 32);
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * rows_per_block + warp; t < N;
-       t += static_cast<int64_t>(gridDim.x) * rows_per_block) {
+  const int64_t rows_per_block = static_cast<int64_t>(kHistThreads / 32) * kRowBatch;
+  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * rows_per_block + warp * kRowBatch; t0 < N;
+       t0 += static_cast<int64_t>(gridDim.x) * rows_per_block) {
     if (!active) continue;
-    const float a = alpha ? __ldg(alpha + t) : 0.f;
-    const float2 v = __ldcs(reinterpret_cast<const float2*>(z + t * E + col0 + c4));
-    const float vv[2] = {v.x, v.y};
+    float2 v[kRowBatch];
+    float a[kRowBatch];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const uint32_t k = order_key(__fadd_rn(vv[i], a));
-      if ((k & hi_mask) == pre[i]) atomicAdd(&h[(c4 + i) * kBins + ((k >> shift) & 0xffu)], 1u);
+    for (int r = 0; r < kRowBatch; ++r) {
+      const int64_t t = t0 + r < N ? t0 + r : N - 1;
+      a[r] = alpha ? __ldg(alpha + t) : 0.f;
+      v[r] = __ldcs(reinterpret_cast<const float2*>(z + t * E + col0 + c4));
+    }
+#pragma unroll
+    for (int r = 0; r < kRowBatch; ++r) {
+      if (t0 + r >= N) break;
+      const float vv[2] = {v[r].x, v[r].y};
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint32_t k = order_key(__fadd_rn(vv[i], a[r]));
+        if ((k & hi_mask) == pre[i]) atomicAdd(&h[(c4 + i) * kBinLd + ((k >> shift) & 0xffu)], 1u);
+      }
     }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kColsPerCta * kBins; i += kHistThreads) {
-    const int c = i / kBins;
-    if (col0 + c < E && h[i]) atomicAdd(hist + static_cast<int64_t>(col0 + c) * kBins + (i % kBins), h[i]);
+    const int c = i / kBins, b = i % kBins;
+    const uint32_t n = h[c * kBinLd + b];
+    if (col0 + c < E && n) atomicAdd(hist + static_cast<int64_t>(col0 + c) * kBins + b, n);
   }
 }
 
@@ -351,10 +380,10 @@ cudaError_t launch_bf16_hist(const float* z, const float* alpha, int64_t N, int3
   const int groups = (E + kColsPerCta - 1) / kColsPerCta;
   int per_group = 3 * device_sm_count() / groups;        // three 64 KB CTAs per SM
   if (per_group < 1) per_group = 1;
-  const int64_t rows_per_block = kHistThreads / 32;
+  const int64_t rows_per_block = (kHistThreads / 32) * kRowBatch;
   int64_t gx = (N + rows_per_block - 1) / rows_per_block;
   if (gx > per_group) gx = per_group;
-  const int smem = static_cast<int>(sizeof(uint32_t) * (kColsPerCta * kBins + kColsPerCta));
+  const int smem = static_cast<int>(sizeof(uint32_t) * (kColsPerCta * kBinLd + kColsPerCta));
   cudaError_t err =
       cudaFuncSetAttribute(bf16_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
@@ -381,10 +410,10 @@ cudaError_t launch_key_hist(const float* z, const float* alpha, int64_t N, int32
   const int groups = (E + kColsPerCta - 1) / kColsPerCta;
   int per_group = 3 * device_sm_count() / groups;
   if (per_group < 1) per_group = 1;
-  const int64_t rows_per_block = kHistThreads / 32;
+  const int64_t rows_per_block = (kHistThreads / 32) * kRowBatch;
   int64_t gx = (N + rows_per_block - 1) / rows_per_block;
   if (gx > per_group) gx = per_group;
-  const int smem = static_cast<int>(sizeof(uint32_t) * (kColsPerCta * kBins + kColsPerCta));
+  const int smem = static_cast<int>(sizeof(uint32_t) * (kColsPerCta * kBinLd + kColsPerCta));
   cudaError_t err =
       cudaFuncSetAttribute(key_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
