@@ -181,6 +181,60 @@ def test_expert_ffn_pages_shape(oracle_mod):
     np.testing.assert_array_equal(host(y2), host(y))
 
 
+def _device_weights(E, d, F, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    wgu = (torch.randn(E, 2 * F, d, generator=g, device="cuda") / math.sqrt(d)).to(torch.bfloat16)
+    wd = (torch.randn(E, d, F, generator=g, device="cuda") / math.sqrt(F)).to(torch.bfloat16)
+    wgu_s = (torch.randn(2 * F, d, generator=g, device="cuda") / math.sqrt(d)).to(torch.bfloat16)
+    wd_s = (torch.randn(d, F, generator=g, device="cuda") / math.sqrt(F)).to(torch.bfloat16)
+    return wgu, wd, wgu_s, wd_s
+
+
+def _oracle_on_tokens(o, rows, x, ids, gates, wgu, wd, wgu_s, wd_s):
+    """The oracle on a subset of tokens (they are independent), with the
+    slices of the experts those tokens use."""
+    ids_r = ids[rows]
+    used = np.unique(ids_r)
+    remap = np.full(wgu.shape[0], -1, np.int64)
+    remap[used] = np.arange(len(used))
+    sl = torch.from_numpy(used).cuda()
+    return o.expert_ffn(_bits(x[rows].cpu()), remap[ids_r].astype(np.int32), gates[rows],
+                        _bits(wgu[sl].cpu()), _bits(wd[sl].cpu()), _bits(wgu_s.cpu()), _bits(wd_s.cpu()))
+
+
+def test_expert_ffn_bench_size_sampled(oracle_mod):
+    # the bench's microbatch: N = 16384 tokens, E = 384, K = 6, d = 2560, F = 512
+    # plus the shared expert, the routing from the library's own permutation;
+    # a sample of tokens (first, last, ragged and random) against the oracle
+    N, d, F, E, K = 16384, 2560, 512, 384, 6
+    wgu, wd, wgu_s, wd_s = _device_weights(E, d, F, 21)
+    g = torch.Generator(device="cuda").manual_seed(22)
+    x = torch.randn(N, d, generator=g, device="cuda").to(torch.bfloat16)
+    rng = np.random.default_rng(22)
+    ids = np.argsort(rng.random((N, E)), axis=1)[:, :K].astype(np.int32)
+    gates = rng.uniform(0.05, 0.95, (N, K)).astype(np.float32)
+    counts, offsets, perm, inv = B.kolibri_expert_permute(dev(ids), E)
+    y = B.kolibri_expert_ffn(x, perm, offsets, inv, dev(gates), wgu, wd, wgu_s, wd_s)
+    torch.cuda.synchronize()
+    check_status()
+    rows = np.unique(np.concatenate([[0, 1, N - 1, N - 256, 4095, 4096],
+                                     rng.choice(N, 42, replace=False)]))
+    y_ref, mag = _oracle_on_tokens(oracle_mod, rows, x, ids, gates, wgu, wd, wgu_s, wd_s)
+    _assert_y_close(host(y)[rows], y_ref, mag)
+
+
+@pytest.mark.parametrize("N,E,K,skew", [(1, 16, 1, False), (3, 8, 1, False), (2000, 4, 2, True)])
+def test_expert_ffn_tiny_and_crowded(oracle_mod, N, E, K, skew):
+    # one token, K = 1; and four experts that take hundreds of rows each (many
+    # token blocks per group, both projections)
+    d, F = 256, 256
+    x, wgu, wd, wgu_s, wd_s, ids, gates = _case(N, d, F, E, K, seed=7 + N, shared=True, skew=skew)
+    y_ref, mag, _, _ = _oracle(oracle_mod, x, wgu, wd, wgu_s, wd_s, ids, gates)
+    y, _, _ = _gpu(x, wgu, wd, wgu_s, wd_s, ids, gates, oracle_mod)
+    check_status()
+    _assert_y_close(host(y), y_ref, mag)
+
+
 def _pad(a, shape):
     out = np.zeros(shape, np.float32)
     out[tuple(slice(0, s) for s in a.shape)] = a
