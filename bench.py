@@ -724,8 +724,8 @@ def _decode_oracle(oracle, wl, layers, xs, ws, betas):
 
 def run_decode(args):
     """The decode sweep: per step, 50 layers of logits + top-K + gates + alpha
-    + counts + stable permutation for N in (1, 8, 64, 256) tokens, every layer
-    with its own x, W and beta.  Timed eager (one call per kernel per layer)
+    + counts + stable permutation (kolibri_router_forward_permute) for N in
+    (1, 8, 64, 256) tokens, every layer with its own x, W and beta.  Timed eager (one call per kernel per layer)
     and as one CUDA graph per step; the forward alone and the logits alone are
     timed the same way to show where the step goes.  The roofline is W
     streamed once from HBM per layer (1.97 MB)."""
@@ -761,10 +761,13 @@ def run_decode(args):
                 if part == "logits":
                     B.kolibri_router_logits(xs[l], ws[l], z=z, stream=stream)
                     continue
-                B.kolibri_router_forward(xs[l], ws[l], betas[l], K, z=z, ids=ids, gates=gates,
-                                         alpha=alpha, stream=stream)
                 if part == "step":
-                    B.kolibri_expert_permute(ids, E, wsp, counts, offsets, perm, inv, stream=stream)
+                    B.kolibri_router_forward_permute(xs[l], ws[l], betas[l], K, z=z, ids=ids, gates=gates,
+                                                     alpha=alpha, counts=counts, offsets=offsets,
+                                                     perm=perm, inv=inv, ws=wsp, stream=stream)
+                else:
+                    B.kolibri_router_forward(xs[l], ws[l], betas[l], K, z=z, ids=ids, gates=gates,
+                                             alpha=alpha, stream=stream)
 
         def timed(fn, reps):
             for _ in range(args.warmup):
@@ -790,8 +793,9 @@ def run_decode(args):
         if st != B.KOLIBRI_OK:
             raise RuntimeError(f"device status: {B.status_string(st)}")
         res["graph_us_per_layer"] = res["graph_us"] / L
-        # per layer: the forward (one launch up to 96 tokens, else logits + selection), the permutation
-        res["gpu_launches"] = (2 if N <= 96 else 3) * L
+        # per layer: one launch up to 16 tokens (forward and grouping); else the forward (one launch
+        # up to 96 tokens, else logits + selection) and the permutation
+        res["gpu_launches"] = (1 if N <= 16 else 2 if N <= 96 else 3) * L
         res["w_bytes_per_step"] = 2 * E * d * L
         per_n[str(n_tok)] = res
     clocks = sampler.stop()

@@ -34,6 +34,8 @@ SIGNATURES = {
     "kolibri_workspace_bytes": (_SZ, [ctypes.c_int, _I64, _I32, _I32]),
     "kolibri_router_logits": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _P]),
     "kolibri_router_forward": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _P, _P, _P]),
+    "kolibri_router_forward_permute": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _P,
+                                                      _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "kolibri_router_forward_eqb": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _I32, _P, _P,
                                                   _P, _P, _P, _SZ, _P]),
     "kolibri_router_topk": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P]),
@@ -250,6 +252,36 @@ def kolibri_expert_permute(ids: torch.Tensor, E: int, ws: torch.Tensor | None = 
                                          _ptr(perm), _ptr(inv), _ptr(ws), ws.numel(),
                                          _stream(stream)))
     return counts, offsets, perm, inv
+
+
+def kolibri_router_forward_permute(x: torch.Tensor, w: torch.Tensor, bias: torch.Tensor | None, K: int,
+                                   z=None, ids=None, gates=None, alpha=None, counts=None, offsets=None,
+                                   perm=None, inv=None, ws: torch.Tensor | None = None, want_inv: bool = True,
+                                   stream=None):
+    """The forward and the permutation of its ids in one call (one launch for
+    decode batches of at most 16 tokens).  Returns (z, ids, gates, alpha,
+    counts, offsets, perm, inv)."""
+    N, d = x.shape
+    E = w.shape[0]
+    _need(x, torch.bfloat16, (N, d), "x")
+    _need(w, torch.bfloat16, (E, d), "w")
+    dev = x.device
+    z = torch.empty((N, E), dtype=torch.float32, device=dev) if z is None else z
+    ids = torch.empty((N, K), dtype=torch.int32, device=dev) if ids is None else ids
+    gates = torch.empty((N, K), dtype=torch.float32, device=dev) if gates is None else gates
+    alpha = torch.empty((N,), dtype=torch.float32, device=dev) if alpha is None else alpha
+    counts = torch.empty((E,), dtype=torch.int32, device=dev) if counts is None else counts
+    offsets = torch.empty((E + 1,), dtype=torch.int64, device=dev) if offsets is None else offsets
+    perm = torch.empty((N * K,), dtype=torch.int32, device=dev) if perm is None else perm
+    if inv is None and want_inv:
+        inv = torch.empty((N * K,), dtype=torch.int32, device=dev)
+    if ws is None:
+        ws = workspace(KOLIBRI_OP_PERMUTE, N, E, K, dev)
+    _check("kolibri_router_forward_permute",
+           load().kolibri_router_forward_permute(
+               _ptr(x), _ptr(w), _ptr(bias), _ptr(z), N, d, E, K, _ptr(ids), _ptr(gates), _ptr(alpha),
+               _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(inv), _ptr(ws), ws.numel(), _stream(stream)))
+    return z, ids, gates, alpha, counts, offsets, perm, inv
 
 
 def kolibri_expert_permute_noalloc(ids: torch.Tensor, E: int, counts=None, offsets=None,

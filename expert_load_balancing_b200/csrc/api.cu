@@ -85,6 +85,35 @@ kolibri_status kolibri_router_forward(const void* x, const void* w, const float*
                                       static_cast<cudaStream_t>(stream)));
 }
 
+kolibri_status kolibri_router_forward_permute(const void* x, const void* w, const float* bias,
+                                              float* z, int64_t N, int32_t d, int32_t E, int32_t K,
+                                              int32_t* ids, float* gates, float* alpha,
+                                              int32_t* counts, int64_t* offsets, int32_t* perm,
+                                              int32_t* inv, void* ws, size_t ws_bytes, void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!x || !w || !z || !ids || !gates || !alpha || !counts || !offsets || !perm)
+    return KOLIBRI_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(z) || (bias && !aligned16(bias)))
+    return KOLIBRI_ERR_INVALID_ARG;
+  if (d < 1) return KOLIBRI_ERR_INVALID_ARG;
+  if (d % 64 != 0 || E % 16 != 0) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  const PermuteLayout L = permute_layout(N, E, K);
+  if (!L.single_cta) {
+    if (!ws) return KOLIBRI_ERR_INVALID_ARG;
+    if (ws_bytes < L.total) return KOLIBRI_ERR_WORKSPACE_TOO_SMALL;
+  }
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (router_decode_permutes(N, d, E, K)) {
+    const cudaError_t err = launch_router_decode_permute(x, w, bias, z, N, d, E, K, ids, gates, alpha,
+                                                         counts, offsets, perm, inv, s);
+    if (err != cudaErrorNotSupported) return from_cuda(err);
+  }
+  cudaError_t err = router_forward_by_size(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+  if (err == cudaSuccess) err = launch_permute(ids, N, E, K, counts, offsets, perm, inv, ws, s);
+  return from_cuda(err);
+}
+
 kolibri_status kolibri_router_forward_eqb(const void* x, const void* w, float* bias, float* z,
                                           int64_t N, int32_t d, int32_t E, int32_t K,
                                           int32_t* ids, float* gates, float* alpha,

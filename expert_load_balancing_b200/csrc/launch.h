@@ -104,6 +104,14 @@ bool router_decode_supported(int64_t N, int32_t d, int32_t E, int32_t K);
 cudaError_t launch_router_decode(const void* x, const void* w, const float* bias, float* z,
                                  int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
                                  float* gates, float* alpha, cudaStream_t s);
+// Batches of one cluster (at most 16 tokens): the same launch also forms
+// counts, offsets, perm and inv (inv may be null).
+bool router_decode_permutes(int64_t N, int32_t d, int32_t E, int32_t K);
+cudaError_t launch_router_decode_permute(const void* x, const void* w, const float* bias, float* z,
+                                         int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                         float* gates, float* alpha, int32_t* counts,
+                                         int64_t* offsets, int32_t* perm, int32_t* inv,
+                                         cudaStream_t s);
 
 // The logits by batch size, with the same choice of kernel as the forward.
 cudaError_t launch_router_logits_by_size(const void* x, const void* w, float* z, int64_t N,

@@ -36,7 +36,17 @@ constexpr int kDecThreads = 32 * kDecWarps;
 struct DecLayout {
   int ld;                                // padded row length of x and W rows, in bf16
   int ec;                                // experts per CTA
-  uint32_t off_x, off_w, off_zp, off_zc, off_beta, off_sc, off_bar, total;
+  uint32_t off_x, off_w, off_zp, off_zc, off_beta, off_sc, off_pids, off_pcnt, off_poff, off_bar,
+      total;
+};
+
+// The permutation outputs when the forward also groups the slots (counts
+// null: it does not).
+struct DecPerm {
+  int32_t* counts;
+  int64_t* offsets;
+  int32_t* perm;
+  int32_t* inv;
 };
 
 template <int Q>
@@ -57,6 +67,12 @@ __host__ __device__ inline DecLayout dec_layout(int d, int E) {
   o += static_cast<uint32_t>(128 * Q * 4);
   L.off_sc = o;
   o += static_cast<uint32_t>((sizeof(RowScratch<Q>) + 15) & ~static_cast<size_t>(15));
+  L.off_pids = o;                        // CTA 0: every slot's expert (16 tokens x K <= 16)
+  o += 4 * kDecTok * 16;
+  L.off_pcnt = o;                        // CTA 0: counts per expert
+  o += 4 * 512;
+  L.off_poff = o;                        // CTA 0: starts per expert
+  o += 4 * 516;
   L.off_bar = o;
   o += 16;
   L.total = o;
@@ -91,6 +107,11 @@ __device__ __forceinline__ void dec_cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
 }
+__device__ __forceinline__ void dsmem_st_u32(uint32_t local_addr, uint32_t rank, uint32_t v) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
+}
 __device__ __forceinline__ float dsmem_ld_f32(uint32_t local_addr, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
@@ -111,7 +132,7 @@ template <int Q, bool kBias>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_forward_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
     const float* __restrict__ bias, float* __restrict__ z, int64_t N, int d, int E, int K,
-    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha) {
+    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha, const DecPerm pm) {
   extern __shared__ __align__(16) uint8_t sm[];
   const DecLayout L = dec_layout<Q>(d, E);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -219,15 +240,75 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_forward_kernel(
       const uint32_t e = id < static_cast<uint32_t>(E) ? id : 0u;
       ids[t * K + rk] = static_cast<int32_t>(id);
       gates[t * K + rk] = gate_sigmoid(sc.row[buffer_pos<Q>(e)]);
+      // the slot's expert, into CTA 0's list when this launch also groups the slots
+      if (pm.counts != nullptr && gridDim.y == 1)
+        dsmem_st_u32(base + L.off_pids + 4u * (rank * static_cast<uint32_t>(K) + static_cast<uint32_t>(rk)),
+                     0u, e);
     }
     if (rk == K && alpha) alpha[t] = -key_to_float(key);
   }
-  dec_cluster_sync();                    // no CTA leaves while its logits may still be read
+  dec_cluster_sync();                    // no CTA leaves while its logits may still be read; the
+                                         // slots' experts are in CTA 0
+
+  // ---- the permutation, when the batch is this one cluster: CTA 0 forms
+  // counts, offsets and the stable grouping (experts ascending, slot index
+  // j = t K + k ascending inside an expert)
+  const bool permute = pm.counts != nullptr && ids != nullptr && gridDim.y == 1 && rank == 0;
+  uint32_t* pid = reinterpret_cast<uint32_t*>(sm + L.off_pids);
+  const int nk = nv * K;
+  if (permute) {
+    uint32_t* cnt = reinterpret_cast<uint32_t*>(sm + L.off_pcnt);
+    uint32_t* start = reinterpret_cast<uint32_t*>(sm + L.off_poff);
+    for (int e = tid; e < E; e += kDecThreads) cnt[e] = 0u;
+    __syncthreads();
+    for (int j = tid; j < nk; j += kDecThreads) atomicAdd(&cnt[pid[j]], 1u);
+    __syncthreads();
+    // exclusive scan over the experts: four per thread (E <= 512)
+    uint32_t v[4], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = 4 * tid + i;
+      v[i] = e < E ? cnt[e] : 0u;
+      sum += v[i];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    uint32_t* wsum = reinterpret_cast<uint32_t*>(sm + L.off_poff) + 512;   // 4 words after the starts
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    uint32_t run = incl - sum;
+    for (int w2 = 0; w2 < warp; ++w2) run += wsum[w2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = 4 * tid + i;
+      if (e < E) {
+        start[e] = run;
+        pm.counts[e] = static_cast<int32_t>(v[i]);
+        pm.offsets[e] = run;
+      }
+      run += v[i];
+    }
+    if (tid == 0) pm.offsets[E] = nk;
+    __syncthreads();
+    for (int j = tid; j < nk; j += kDecThreads) {
+      const uint32_t e = pid[j];
+      uint32_t before = 0;                 // earlier slots of the same expert
+      for (int i = 0; i < j; ++i) before += (pid[i] == e) ? 1u : 0u;
+      const uint32_t pos = start[e] + before;
+      pm.perm[pos] = j;
+      if (pm.inv) pm.inv[j] = static_cast<int32_t>(pos);
+    }
+  }
 }
 
 template <int Q, bool kBias>
 cudaError_t launch_dec(const void* x, const void* w, const float* bias, float* z, int64_t N, int d,
-                       int E, int K, int32_t* ids, float* gates, float* alpha, cudaStream_t s) {
+                       int E, int K, int32_t* ids, float* gates, float* alpha, const DecPerm& pm,
+                       cudaStream_t s) {
   const DecLayout L = dec_layout<Q>(d, E);
   auto kern = decode_forward_kernel<Q, kBias>;
   static int checked = 0;                // 1: runs, -1: this device cannot place the cluster
@@ -259,7 +340,7 @@ cudaError_t launch_dec(const void* x, const void* w, const float* bias, float* z
   const unsigned tiles = static_cast<unsigned>((N + kDecTok - 1) / kDecTok);
   return launch_pdl(kern, dim3(kDecCtas, tiles, 1), dim3(kDecThreads), L.total, s, dim3(kDecCtas, 1, 1),
                     static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w), bias, z, N,
-                    d, E, K, ids, gates, alpha);
+                    d, E, K, ids, gates, alpha, pm);
 }
 
 }  // namespace
@@ -275,21 +356,41 @@ bool router_decode_supported(int64_t N, int32_t d, int32_t E, int32_t K) {
   return total <= 227u * 1024u;
 }
 
-cudaError_t launch_router_decode(const void* x, const void* w, const float* bias, float* z,
-                                 int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
-                                 float* gates, float* alpha, cudaStream_t s) {
+static cudaError_t decode_dispatch(const void* x, const void* w, const float* bias, float* z,
+                                   int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                   float* gates, float* alpha, const DecPerm& pm, cudaStream_t s) {
   if (!router_decode_supported(N, d, E, K)) return cudaErrorNotSupported;
   const bool b = bias != nullptr;
   switch (E / 128) {
-    case 1: return b ? launch_dec<1, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s)
-                     : launch_dec<1, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
-    case 2: return b ? launch_dec<2, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s)
-                     : launch_dec<2, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
-    case 3: return b ? launch_dec<3, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s)
-                     : launch_dec<3, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
-    default: return b ? launch_dec<4, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s)
-                      : launch_dec<4, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, s);
+    case 1: return b ? launch_dec<1, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, s)
+                     : launch_dec<1, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, s);
+    case 2: return b ? launch_dec<2, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, s)
+                     : launch_dec<2, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, s);
+    case 3: return b ? launch_dec<3, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, s)
+                     : launch_dec<3, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, s);
+    default: return b ? launch_dec<4, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, s)
+                      : launch_dec<4, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, s);
   }
+}
+
+cudaError_t launch_router_decode(const void* x, const void* w, const float* bias, float* z,
+                                 int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                 float* gates, float* alpha, cudaStream_t s) {
+  return decode_dispatch(x, w, bias, z, N, d, E, K, ids, gates, alpha, DecPerm{}, s);
+}
+
+bool router_decode_permutes(int64_t N, int32_t d, int32_t E, int32_t K) {
+  return N <= kDecTok && router_decode_supported(N, d, E, K);
+}
+
+cudaError_t launch_router_decode_permute(const void* x, const void* w, const float* bias, float* z,
+                                         int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                         float* gates, float* alpha, int32_t* counts,
+                                         int64_t* offsets, int32_t* perm, int32_t* inv,
+                                         cudaStream_t s) {
+  if (!router_decode_permutes(N, d, E, K)) return cudaErrorNotSupported;
+  return decode_dispatch(x, w, bias, z, N, d, E, K, ids, gates, alpha,
+                         DecPerm{counts, offsets, perm, inv}, s);
 }
 
 KOLIBRI_DEFINE_STATUS_TAKE(status_take_decode)

@@ -118,6 +118,25 @@ KOLIBRI_API kolibri_status kolibri_router_forward(const void *x, const void *w, 
                                                   float *alpha, void *stream);
 
 /*
+ * kolibri_router_forward followed by kolibri_expert_permute on its ids, in
+ * one call: the arguments and outputs of both ("Kolibri Pre-Training from
+ * Scratch" 6.1 and 7.1; loads and grouping 6.1/6.2).  A decode batch of at
+ * most 16 tokens with E a multiple of 128 (and the router rows fitting in
+ * shared memory: E/16 rows of d per CTA) takes a single launch in which one
+ * 16-CTA cluster forms the logits, the selection and the grouping; other
+ * batches run the forward and then the permutation.  ws / ws_bytes as for
+ * kolibri_expert_permute (ignored, and may be NULL, when N*K <= 4096).
+ * inv may be NULL.
+ */
+KOLIBRI_API kolibri_status kolibri_router_forward_permute(const void *x, const void *w,
+                                                          const float *bias, float *z, int64_t N,
+                                                          int32_t d, int32_t E, int32_t K,
+                                                          int32_t *ids, float *gates, float *alpha,
+                                                          int32_t *counts, int64_t *offsets,
+                                                          int32_t *perm, int32_t *inv, void *ws,
+                                                          size_t ws_bytes, void *stream);
+
+/*
  * One training step's routing from the tokens: logits, selection with bias
  * beta_in, and the EQB update of bias to beta_out ("Kolibri Pre-Training
  * from Scratch" 6.1, 7.1 update rule, 7.2 order of operations, 7.3 exact

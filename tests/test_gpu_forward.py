@@ -94,6 +94,29 @@ def test_forward_decode_batches(oracle_mod, N, d, E, K, with_bias):
     assert_logits_close(host(z), oracle_mod.router_logits(workloads.bf16_bits(x), workloads.bf16_bits(w)))
 
 
+@pytest.mark.parametrize("N,d,E,K", [(1, 2560, 384, 6), (5, 2560, 384, 6), (16, 2560, 384, 6),
+                                     (17, 2560, 384, 6), (64, 1024, 128, 8), (7, 1024, 512, 16),
+                                     (300, 512, 384, 6), (5000, 256, 384, 6)])
+@pytest.mark.parametrize("with_bias", [True, False])
+def test_forward_permute_equals_the_two_calls(oracle_mod, N, d, E, K, with_bias):
+    # up to 16 tokens the forward and the grouping come from one launch; every
+    # output must equal the forward followed by the permutation, bit for bit
+    wl = workloads.Workload("t", N, d, E, K, offsets="collapsed8", beta="normal0.1")
+    b = dev(workloads.make_beta(wl).numpy()) if with_bias else None
+    x, w = workloads.make_x(wl).cuda(), workloads.make_w(wl).cuda()
+    got = B.kolibri_router_forward_permute(x, w, b, K)
+    z, ids, gates, alpha = B.kolibri_router_forward(x, w, b, K)
+    counts, offsets, perm, inv = B.kolibri_expert_permute(ids, E)
+    torch.cuda.synchronize()
+    check_status()
+    for name, a, r in zip(("z", "ids", "gates", "alpha", "counts", "offsets", "perm", "inv"), got,
+                          (z, ids, gates, alpha, counts, offsets, perm, inv)):
+        assert_bit_equal(host(a), host(r), name)
+    c_o, o_o, p_o, i_o = oracle_mod.permute(host(ids), E)
+    assert_bit_equal(host(got[6]), p_o, "perm vs oracle")
+    assert_bit_equal(host(got[4]), c_o, "counts vs oracle")
+
+
 def test_forward_decode_heavy_ties(oracle_mod):
     # identical router rows in a decode batch: the selection's slow path
     N, d, E, K = 40, 256, 384, 6
