@@ -26,6 +26,7 @@
 
 #include "launch.h"
 #include "common.cuh"
+#include "pdl.cuh"
 
 namespace kolibri {
 
@@ -153,13 +154,23 @@ __device__ __forceinline__ int64_t stage_keys(const uint32_t* __restrict__ keys,
 }
 
 // Step 2 (or the whole selection when the sample is the column).
+// The bracket path also clears this expert's counters of the full pass
+// (clear non-null: above, cnt, flag).
 __global__ void __launch_bounds__(kSelThreads) sample_select_kernel(
     const uint32_t* __restrict__ sample, int64_t S, int64_t m_exact, int64_t r_hi, int64_t r_lo,
     int64_t S_ld, bool exact, float* __restrict__ v, uint32_t* __restrict__ lo,
-    uint32_t* __restrict__ hi) {
+    uint32_t* __restrict__ hi, uint32_t* __restrict__ clear_above, uint32_t* __restrict__ clear_cnt,
+    uint32_t* __restrict__ clear_flag) {
   __shared__ SelectSmem sm;
   extern __shared__ __align__(16) uint32_t keys_s[];
   const int e = blockIdx.x;
+  pdl_wait();       // the sample comes from the kernel before this one
+  pdl_trigger();
+  if (clear_above != nullptr && threadIdx.x == 0) {
+    clear_above[e] = 0u;
+    clear_cnt[e] = 0u;
+    clear_flag[e] = 0u;
+  }
   const uint32_t* keys = sample + static_cast<int64_t>(e) * S_ld;
   stage_keys(keys, S, keys_s);
   const bool in_smem = S <= kSmemKeys;
@@ -188,6 +199,8 @@ __global__ void __launch_bounds__(kSelThreads) bracket_select_kernel(
   __shared__ SelectSmem sm;
   extern __shared__ __align__(16) uint32_t keys_s[];
   const int e = blockIdx.x;
+  pdl_wait();       // counts and gathered keys come from the full pass
+  pdl_trigger();
   const int64_t c = cnt[e], ab = above[e];
   const bool ok = c <= cap && ab <= m && m < ab + c;
   if (!ok) {
@@ -214,6 +227,8 @@ __global__ void __launch_bounds__(kSelThreads) column_fallback_kernel(
     const uint32_t* __restrict__ flag, float* __restrict__ v) {
   __shared__ SelectSmem sm;
   const int e = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (flag[e] == 0u) return;
   auto at = [z, alpha, E, e](int64_t t) {
     return order_key(__fadd_rn(__ldg(z + t * E + e), __ldg(alpha + t)));
@@ -228,6 +243,8 @@ __global__ void bias_update_kernel(const float* __restrict__ v, int E, float* __
                                    float* __restrict__ quantiles) {
   __shared__ float mean_s;
   __shared__ float v_s[KOLIBRI_MAX_EXPERTS];
+  pdl_wait();       // v comes from the kernels before this one
+  pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) v_s[e] = v[e];
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -320,9 +337,10 @@ cudaError_t eqb_brackets(int64_t N, int32_t E, int32_t K, const EqbBuffers& b, c
   if (L.exact_small) {
     err = set_select_smem();
     if (err != cudaSuccess) return err;
-    sample_select_kernel<<<E, kSelThreads, select_smem(L.S), s>>>(b.sample, L.S, m, 0, 0, L.S_ld,
-                                                                   true, b.v, b.lo, b.hi);
-    return cudaGetLastError();
+    return launch_pdl(sample_select_kernel, dim3(E), dim3(kSelThreads), select_smem(L.S), s, dim3(0, 0, 0),
+                      b.sample, L.S, m, static_cast<int64_t>(0), static_cast<int64_t>(0), L.S_ld, true, b.v,
+                      b.lo, b.hi, static_cast<uint32_t*>(nullptr), static_cast<uint32_t*>(nullptr),
+                      static_cast<uint32_t*>(nullptr));
   }
   // bracket ranks in the sample, descending order: the target sits at
   // about q*S with q = (m+1)/N; margin 6 binomial standard deviations
@@ -334,13 +352,12 @@ cudaError_t eqb_brackets(int64_t N, int32_t E, int32_t K, const EqbBuffers& b, c
   int64_t r_lo = static_cast<int64_t>(std::ceil(center)) + margin;
   if (r_hi < 0) r_hi = 0;
   if (r_lo > L.S - 1) r_lo = L.S - 1;
-  err = cudaMemsetAsync(b.base + L.off_above, 0, L.off_v - L.off_above, s);  // above, cnt, flag
-  if (err != cudaSuccess) return err;
   err = set_select_smem();
   if (err != cudaSuccess) return err;
-  sample_select_kernel<<<E, kSelThreads, select_smem(L.S), s>>>(b.sample, L.S, 0, r_hi, r_lo,
-                                                                 L.S_ld, false, b.v, b.lo, b.hi);
-  return cudaGetLastError();
+  // the select also clears the full pass's counters (above, cnt, flag)
+  return launch_pdl(sample_select_kernel, dim3(E), dim3(kSelThreads), select_smem(L.S), s, dim3(0, 0, 0),
+                    b.sample, L.S, static_cast<int64_t>(0), r_hi, r_lo, L.S_ld, false, b.v, b.lo, b.hi,
+                    b.above, b.cnt, b.flag);
 }
 
 // Steps 1-2: sample keys (token bias given, or computed from bias_in), then
@@ -362,22 +379,21 @@ cudaError_t eqb_end(const float* z, const float* alpha_used, float* bias, int64_
   if (!b.L.exact_small) {
     err = set_select_smem();
     if (err != cudaSuccess) return err;
-    bracket_select_kernel<<<E, kSelThreads, select_smem(kSmemKeys), s>>>(b.cand, b.cnt, b.above,
-                                                                          kCandCap, m, b.v, b.flag);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    column_fallback_kernel<<<E, kSelThreads, 0, s>>>(z, alpha_used, N, E, m, b.flag, b.v);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_pdl(bracket_select_kernel, dim3(E), dim3(kSelThreads), select_smem(kSmemKeys), s,
+                     dim3(0, 0, 0), b.cand, b.cnt, b.above, static_cast<int64_t>(kCandCap), m, b.v, b.flag);
+    if (err != cudaSuccess) return err;
+    err = launch_pdl(column_fallback_kernel, dim3(E), dim3(kSelThreads), 0, s, dim3(0, 0, 0), z, alpha_used, N,
+                     E, m, b.flag, b.v);
+    if (err != cudaSuccess) return err;
   }
-  bias_update_kernel<<<1, 512, 0, s>>>(b.v, E, bias, quantiles);
-  return cudaGetLastError();
+  return launch_pdl(bias_update_kernel, dim3(1), dim3(512), 0, s, dim3(0, 0, 0), b.v, E, bias, quantiles);
 }
 
 }  // namespace
 
 cudaError_t launch_bias_update(const float* v, int32_t E, float* bias, float* quantiles,
                                cudaStream_t s) {
-  bias_update_kernel<<<1, 512, 0, s>>>(v, E, bias, quantiles);
-  return cudaGetLastError();
+  return launch_pdl(bias_update_kernel, dim3(1), dim3(512), 0, s, dim3(0, 0, 0), v, E, bias, quantiles);
 }
 
 cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,

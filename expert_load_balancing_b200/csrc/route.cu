@@ -297,6 +297,8 @@ __global__ void __launch_bounds__(kThreads) sample_keys_kernel(
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t s0 = static_cast<int64_t>(blockIdx.x) * kSampleRows;
+  pdl_wait();       // Z and alpha come from the kernels before this one
+  pdl_trigger();
   if constexpr (kBias) {
     for (int e = threadIdx.x; e < E; e += kThreads) beta_s[e] = beta[e];
   }
@@ -453,8 +455,7 @@ cudaError_t launch_sample_q(const float* z, const float* alpha, const float* bia
   cudaError_t err =
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  k<<<grid, block, smem, s>>>(z, alpha, bias, N, E, K, S, stride, S_ld, sample);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, block, smem, s, dim3(0, 0, 0), z, alpha, bias, N, E, K, S, stride, S_ld, sample);
 }
 
 }  // namespace
