@@ -17,19 +17,19 @@
 //
 // The projections are one grouped GEMM kernel: a persistent kernel on SM
 // pairs (tcgen05.mma.cta_group::2, bf16 in, fp32 accumulate in TMEM, two
-// accumulators so the epilogue of one tile runs under the MMAs of the
-// next).  The weights are the MMA's M side (256 features per pair) and the
+// accumulator buffers so the epilogue of one tile runs under the MMAs of
+// the next).  The weights are the MMA's M side (256 rows per pair) and the
 // tokens its N side, so the last token block of an expert is an MMA of just
 // its rows rounded up to 32 (with balanced loads of about 256 rows an
 // expert, 256-row blocks of tokens on the M side would spend up to half of
 // the tensor time on empty rows).  Tiles are (expert, token block, feature
-// block)
-// from the offsets, so no host round trip is needed between the
-// permutation and the GEMMs.  In the gate/up projection a CTA stages the
-// gate rows and the up rows of the same 128 units and issues one MMA for
-// each into its own columns, so a thread holds both sums of its unit and
-// the epilogue forms SiLU(gate) * up in registers.  Stores are one token
-// row segment per warp instruction.  No load uses cluster multicast.
+// block); every CTA maps a tile index to them on the device from the
+// offsets, so no host round trip is needed between the permutation and the
+// GEMMs.  In the gate/up projection a CTA stages the gate rows and the up
+// rows of the same 128 units and issues one MMA for each into its own
+// columns, so a thread holds both sums of its unit and the epilogue forms
+// SiLU(gate) * up in registers.  Stores are one token row segment per warp
+// instruction.  No load uses cluster multicast.
 #include <cuda_bf16.h>
 
 #include "launch.h"
@@ -120,10 +120,23 @@ struct TileMap {
 
 // All threads: mt[0..G] from the offsets (a block-wide exclusive scan), and
 // a shared-memory copy of the offsets (off[0..G]; without offsets: 0, rows).
+// Offsets that do not start at 0, decrease, or pass the row count are
+// flagged (device status) and give no tiles at all, so nothing is stored.
 __device__ void build_tile_prefix(const GroupedParams& p, int tok, int32_t* mt, int64_t* off,
                                   int32_t* warp_tot) {
-  for (int g = threadIdx.x; g <= p.G; g += kThreads)
-    off[g] = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.rows);
+  __shared__ int bad_s;
+  if (threadIdx.x == 0) bad_s = 0;
+  __syncthreads();
+  for (int g = threadIdx.x; g <= p.G; g += kThreads) {
+    const int64_t o = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.rows);
+    off[g] = o;
+    const bool ok = (g == 0 ? o == 0 : true) && o <= p.rows &&
+                    (g == 0 || !p.offsets || p.offsets[g - 1] <= o);
+    if (!ok) bad_s = 1;
+  }
+  __syncthreads();
+  const bool bad = bad_s != 0;
+  if (bad && threadIdx.x == 0 && blockIdx.x == 0) raise_status(kStatusBadInput);
   constexpr int kPer = (kMaxGroups + kThreads - 1) / kThreads;   // 3
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t v[kPer];
@@ -132,8 +145,8 @@ __device__ void build_tile_prefix(const GroupedParams& p, int tok, int32_t* mt, 
   for (int i = 0; i < kPer; ++i) {
     const int g = tid * kPer + i;
     int32_t c = 0;
-    if (g < p.G) {
-      const int64_t len = p.offsets ? (p.offsets[g + 1] - p.offsets[g]) : p.rows;
+    if (g < p.G && !bad) {
+      const int64_t len = off[g + 1] - off[g];
       c = static_cast<int32_t>((len + tok - 1) / tok);
     }
     v[i] = c;

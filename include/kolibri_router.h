@@ -395,7 +395,9 @@ KOLIBRI_API kolibri_status kolibri_intervention_rate(const float *z, const int32
  * ws: kolibri_expert_ffn_workspace_size(N, d, F, K, shared) bytes of device
  * memory (the gathered rows, h and the routed outputs; about
  * N K (6 d + 2 F) bytes), owned by the caller.  Out-of-range entries of perm
- * or inv are skipped and set KOLIBRI_ERR_DEVICE in kolibri_device_status.
+ * or inv are skipped and set KOLIBRI_ERR_DEVICE in kolibri_device_status;
+ * offsets that do not start at 0, decrease, or pass N*K make the projections
+ * store nothing and set the same status.
  */
 KOLIBRI_API size_t kolibri_expert_ffn_workspace_size(int64_t N, int32_t d, int32_t F, int32_t K,
                                                      int32_t shared);

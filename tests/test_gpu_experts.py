@@ -317,6 +317,20 @@ def test_expert_bad_perm_sets_device_status():
     assert B.kolibri_device_status() == B.KOLIBRI_OK
 
 
+@pytest.mark.parametrize("offsets", [[0, 300, 100, 400], [0, 100, 200, 999], [5, 100, 200, 400]])
+def test_expert_bad_offsets_flagged_and_nothing_written(offsets):
+    # decreasing, past the rows, not starting at 0: the projection schedules
+    # no tile, sets the device status, and leaves the output as it was
+    rows, d, F, G = 400, 256, 256, 3
+    a = torch.zeros(rows, d, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(G, 2 * F, d, dtype=torch.bfloat16, device="cuda")
+    h = torch.full((rows, F), 7.0, dtype=torch.bfloat16, device="cuda")
+    B.kolibri_expert_gate_up(a, dev(np.array(offsets, np.int64)), w, h)
+    assert B.kolibri_device_status() == B.KOLIBRI_ERR_DEVICE
+    assert bool((h == 7.0).all())
+    assert B.kolibri_device_status() == B.KOLIBRI_OK
+
+
 def test_expert_unsupported_shapes_rejected():
     a = torch.zeros(4, 192, dtype=torch.bfloat16, device="cuda")        # d not a multiple of 256
     w = torch.zeros(1, 256, 192, dtype=torch.bfloat16, device="cuda")
