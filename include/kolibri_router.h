@@ -37,6 +37,10 @@
  *   - Calls on different streams may run concurrently if they use separate
  *     workspaces; one workspace must not be shared by calls that can
  *     overlap on the GPU.
+ *   - The first call of an entry point in a process looks up launch limits
+ *     (occupancy, kernel attributes) and keeps them in process-wide
+ *     variables.  Make the first call of each entry point before calling it
+ *     from several host threads at once.
  */
 #ifndef KOLIBRI_ROUTER_H
 #define KOLIBRI_ROUTER_H
