@@ -9,7 +9,14 @@ inputs; ``build`` compiles the library in-tree.
 from . import binding  # noqa: F401  (loads the library lazily, on first call)
 from .binding import (  # noqa: F401
     KolibriError,
+    expert_ffn_workspace,
     kolibri_device_status,
+    kolibri_eqb_bf16_bias,
+    kolibri_eqb_bf16_digit,
+    kolibri_eqb_bf16_histogram,
+    kolibri_eqb_key_bias,
+    kolibri_eqb_key_digit,
+    kolibri_eqb_key_histogram,
     kolibri_eqb_update,
     kolibri_eqb_update_bf16,
     kolibri_expert_combine,
@@ -19,13 +26,16 @@ from .binding import (  # noqa: F401
     kolibri_expert_gate_up,
     kolibri_expert_permute,
     kolibri_expert_permute_noalloc,
+    kolibri_intervention_rate,
+    kolibri_lei_inject,
     kolibri_route_and_balance,
     kolibri_router_forward,
     kolibri_router_forward_eqb,
+    kolibri_router_forward_permute,
     kolibri_router_logits,
-    kolibri_intervention_rate,
-    kolibri_lei_inject,
     kolibri_router_topk,
     kolibri_score_grad_to_logits,
+    kolibri_selftest_bounded_wait,
     kolibri_workspace_bytes,
+    workspace,
 )

@@ -62,6 +62,7 @@ SIGNATURES = {
     "kolibri_expert_down": (ctypes.c_int, [_P, _I64, _P, _I32, _P, _P, _I32, _I32, _P]),
     "kolibri_expert_combine": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I32, _I32, _P, _P]),
     "kolibri_device_status": (ctypes.c_int, [_P]),
+    "kolibri_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, _P]),
 }
 
 
@@ -361,6 +362,12 @@ def kolibri_route_and_balance(z: torch.Tensor, bias: torch.Tensor, K: int,
 def kolibri_device_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status word."""
     return int(load().kolibri_device_status(_stream(stream)))
+
+
+def kolibri_selftest_bounded_wait(limit_ns: int = 1_000_000, stream=None) -> None:
+    """Enqueue a wait that runs out after about limit_ns; the next
+    kolibri_device_status on that stream reports KOLIBRI_ERR_TIMEOUT."""
+    _check("kolibri_selftest_bounded_wait", load().kolibri_selftest_bounded_wait(int(limit_ns), _stream(stream)))
 
 
 # ------------------------------------------------ bf16-key EQB, LEI, intervention

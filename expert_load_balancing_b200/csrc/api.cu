@@ -33,6 +33,17 @@ kolibri_status check_ek(int64_t N, int32_t E, int32_t K) {
 
 kolibri_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KOLIBRI_OK : KOLIBRI_ERR_CUDA; }
 
+// One warp waits, through the kernels' bounded wait, on a shared-memory
+// barrier that nothing arrives at: the wait gives up after about limit_ns,
+// records the timeout in the status word and the kernel returns.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) mbar_init(b, 1);
+  __syncthreads();
+  mbar_wait(b, 0u, limit_ns);
+}
+
 }  // namespace
 }  // namespace kolibri
 
@@ -338,6 +349,12 @@ kolibri_status kolibri_expert_combine(const float* y_perm, const float* y_shared
   if (d % 4 != 0 || N * K >= kExpertRowLimit) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
   return from_cuda(launch_expert_combine(y_perm, y_shared, inv, gates, N, d, K, y,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull) return KOLIBRI_ERR_INVALID_ARG;
+  bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return from_cuda(cudaGetLastError());
 }
 
 kolibri_status kolibri_device_status(void* stream) {

@@ -440,6 +440,17 @@ KOLIBRI_API kolibri_status kolibri_expert_combine(const float *y_perm, const flo
                                                   void *stream);
 
 /*
+ * Diagnostic of the device-side failure path: launches one warp that waits,
+ * through the same bounded wait the kernels use, on a shared-memory barrier
+ * that nothing arrives at.  After about limit_ns nanoseconds (1e3 to 1e9,
+ * else KOLIBRI_ERR_INVALID_ARG) the wait gives up, records
+ * KOLIBRI_ERR_TIMEOUT in the device status word and the kernel returns, so
+ * kolibri_device_status(stream) then reports the timeout and the context
+ * stays usable.  Touches no caller memory.
+ */
+KOLIBRI_API kolibri_status kolibri_selftest_bounded_wait(uint64_t limit_ns, void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device: KOLIBRI_OK, KOLIBRI_ERR_TIMEOUT or KOLIBRI_ERR_DEVICE
  * (the first recorded), or KOLIBRI_ERR_CUDA if the synchronisation failed.

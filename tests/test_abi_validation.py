@@ -135,3 +135,10 @@ def test_expert_layer_checks(lib):
     assert cb(F, None, F, F, n, d, 40, F, None) == INVALID
     assert cb(F, ODD, F, F, n, d, K, F, None) == INVALID
     assert cb(None, None, F, F, n, d, K, F, None) == INVALID
+
+
+def test_selftest_limits(lib):
+    # the diagnostic wait takes 1 us to 1 s; anything else is refused on the host
+    assert lib.kolibri_selftest_bounded_wait(0, None) == INVALID
+    assert lib.kolibri_selftest_bounded_wait(999, None) == INVALID
+    assert lib.kolibri_selftest_bounded_wait(1_000_000_001, None) == INVALID
