@@ -5,6 +5,11 @@ library's CUDA kernels.  PyTorch supplies device memory and the current
 stream.  The library must have been built (``python -m
 expert_load_balancing_b200.build``); loading fails loudly otherwise, and
 there is no CPU fallback.
+
+The library launches on the current CUDA device: the tensors of a call must
+live on it (inside ``torch.cuda.device(t.device)`` when several GPUs are in
+use).  The wrappers check dtype, shape, contiguity and that tensors are on a
+GPU, not which one, to keep the per-call host cost of small batches low.
 """
 from __future__ import annotations
 
