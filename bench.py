@@ -464,8 +464,6 @@ def run_reference(args, rank, world):
     }
 
 
-# ---------------------------------------------------------------- main
-
 # ---------------------------------------------------------------- the balancing pieces
 
 PARTS = {
@@ -827,6 +825,8 @@ def run_decode(args):
                          "kind": "oracle", "sample": "one whole step at N=8 (50 layers)"},
     }
 
+
+# ---------------------------------------------------------------- main
 
 def main():
     ap = argparse.ArgumentParser()
