@@ -219,6 +219,24 @@ class RouterStep:
             events[5].record(stream)
 
 
+def maxvio(counts, wl):
+    """MaxVio of one routing ("Kolibri Pre-Training from Scratch" 6.2): the
+    largest expert load over the mean load N K / E, minus one."""
+    return float(counts.max().item()) / (wl.N * wl.K / wl.E) - 1.0
+
+
+def rerouted_maxvio(step, stream):
+    """MaxVio of the batch routed again with the bias the last timed step's
+    EQB update produced (outside the timed region)."""
+    wl = step.wl
+    B.kolibri_router_forward(step.x, step.w, step.beta, wl.K, z=step.z, ids=step.ids,
+                             gates=step.gates, alpha=step.alpha, stream=stream)
+    B.kolibri_expert_permute(step.ids, wl.E, step.ws_perm, step.counts, step.offsets, step.perm,
+                             step.inv, stream=stream)
+    stream.synchronize()
+    return maxvio(step.counts, wl)
+
+
 def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
@@ -230,9 +248,14 @@ def run_ours(args, rank, world, local_rank):
     N, d, E, K = wl.N, wl.d, wl.E, wl.K
     step = RouterStep(wl, device, seed=rank)
     stream = torch.cuda.Stream(device)
+    balance = {}
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
+        for i in range(args.warmup):
             step.run(stream)
+            if i == 0:
+                # the loads of the first routing, with the workload's initial bias
+                torch.cuda.synchronize()
+                balance["maxvio_initial_bias"] = maxvio(step.counts, wl)
     stream.synchronize()
     st = B.kolibri_device_status(stream)
     if st != B.KOLIBRI_OK:
@@ -268,6 +291,11 @@ def run_ours(args, rank, world, local_rank):
 
     total_ms = reduce_max_over_ranks(total_ms, device)
     ms_per_step = total_ms / args.steps
+    # balance of the routing, outside the timed region: the last timed step's
+    # loads (bias before its update) and a re-route with the updated bias
+    balance["maxvio_last_step"] = maxvio(step.counts, wl)
+    with torch.cuda.stream(stream):
+        balance["maxvio_rerouted"] = rerouted_maxvio(step, stream)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -314,6 +342,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step(N, E, K) * args.steps,
         "clocks": clocks,
         "e2e": e2e,
+        "balance": balance,
+        "gpu_name": torch.cuda.get_device_name(device),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
