@@ -6,7 +6,9 @@ two and three gloo ranks on the CPU; the three library calls are replaced by
 CPU stand-ins built from the oracle's bf16 rounding and key (the GPU kernels
 behind them are checked against the oracle in test_gpu_balance.py).  Every
 rank must end with the exact quantile of the union and the same bias; the
-pages' counter-example shows that averaging per-rank quantiles would not."""
+pages' counter-example shows that averaging per-rank quantiles would not.
+A rank that exits or stalls between steps makes the survivor's next
+all-reduce end with an error, not wait for good."""
 import os
 import socket
 
@@ -218,3 +220,64 @@ def test_fp32_keys_three_ranks_equal_the_union(oracle_mod):
     for q, b in res:
         np.testing.assert_array_equal(q, v)
         np.testing.assert_array_equal(b, oracle_mod.eqb_bias(v))
+
+
+
+def _worker_peer_lost(rank, world, port, out, mode):
+    """Rank 1 fails right after joining: it exits ("exit") or stays alive
+    without entering any collective ("stall").  Rank 0 then runs the update,
+    whose first histogram all-reduce must end in an error, not wait for good."""
+    import sys
+    import time
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        out[1] = "left"
+        if mode == "stall":
+            time.sleep(15)
+        os._exit(0)            # no destroy, no collective: the peer is gone
+    import oracle
+    from expert_load_balancing_b200 import distributed as D
+    rng = np.random.default_rng(5)
+    z = torch.from_numpy((rng.standard_normal((12, 4)) * 2).astype(np.float32))
+    a = torch.zeros(12)
+    bias = torch.zeros(4)
+    t = time.time()
+    try:
+        D.eqb_update_distributed(z, a, bias, 2, 24, ops=_CpuKeyOps(oracle))
+        out[0] = ("finished", time.time() - t)
+    except Exception as e:          # the collective reports the lost peer
+        out[0] = ("error", time.time() - t, type(e).__name__)
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+@pytest.mark.parametrize("mode", ["exit", "stall"])
+def test_lost_rank_ends_the_update_with_an_error(mode):
+    # host-side failure between steps: a rank that exits, or one that never
+    # joins the next collective; the survivor's all-reduce fails (at once, or
+    # after the process group's 5 s timeout) instead of hanging
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_peer_lost, args=(r, 2, port, out, mode)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+            pytest.fail("a rank did not end")
+    assert out[1] == "left"
+    res = out[0]
+    assert res[0] == "error", res
+    assert res[1] < 14.0, res          # ended by the error, before the stalled rank left
