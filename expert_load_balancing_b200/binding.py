@@ -31,6 +31,8 @@ KOLIBRI_ERR_DEVICE = 6
 KOLIBRI_OP_PERMUTE = 1
 KOLIBRI_OP_EQB = 2
 KOLIBRI_OP_EQB_BF16 = 3
+# size of the library-held scratch of kolibri_expert_permute_noalloc (the header's macro)
+KOLIBRI_NOALLOC_SCRATCH_BYTES = 2 << 20
 
 # every symbol the header declares, with (restype, argtypes)
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t

@@ -26,11 +26,18 @@ void* g_scratch_ptr[kMaxDevices] = {};
 // first call for that device).  Returns nullptr if the lookup fails.
 void* scratch_on_current_device() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
   if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();   // clear it, so no later launch check reports it as its own
+      return nullptr;
+    }
     g_scratch_ptr[dev] = p;
   }
   return g_scratch_ptr[dev];

@@ -205,7 +205,7 @@ KOLIBRI_API kolibri_status kolibri_expert_permute(const int32_t *ids, int64_t N,
  *   Arguments and results are those of kolibri_expert_permute, without ws.
  *   Sizes whose scratch (kolibri_workspace_bytes(KOLIBRI_OP_PERMUTE, N, E,
  *   K)) exceeds the array return KOLIBRI_ERR_WORKSPACE_TOO_SMALL and
- *   enqueue nothing (at E = 384, up to 11,182,080 routed slots N*K fit).
+ *   enqueue nothing (at E = 384, up to 11,173,888 routed slots N*K fit).
  *   The first call on each device looks up the array's device address with
  *   that device current; make that first call before any stream capture.
  *   Every call shares the one array: calls that can overlap on the GPU (on

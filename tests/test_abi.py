@@ -111,3 +111,38 @@ def test_library_refuses_to_run_without_extension(tmp_path):
             binding.load(str(tmp_path / "missing.so"))
         finally:
             binding._lib = None
+
+
+def _noalloc_header_limit():
+    src = open(HEADER).read()
+    m = re.search(r"up to ([\d,]+) routed slots N\*K fit", src)
+    assert m, "the header states the no-allocation limit"
+    return int(m.group(1).replace(",", ""))
+
+
+def test_noalloc_limit_is_the_largest_size_that_fits(kolibri_lib):
+    """The figure the header gives for E = 384 is exactly the boundary of the
+    fixed scratch array: that many slots fit, one more does not (host-side
+    layout sizes only; K = 1 so that every slot count can be formed)."""
+    from expert_load_balancing_b200 import binding as B
+    limit = _noalloc_header_limit()
+    cap = B.KOLIBRI_NOALLOC_SCRATCH_BYTES
+    assert B.kolibri_workspace_bytes(B.KOLIBRI_OP_PERMUTE, limit, 384, 1) <= cap
+    assert B.kolibri_workspace_bytes(B.KOLIBRI_OP_PERMUTE, limit + 1, 384, 1) > cap
+    # the figure does not depend on how the slots split into tokens and ranks
+    assert B.kolibri_workspace_bytes(B.KOLIBRI_OP_PERMUTE, limit // 8, 384, 8) <= cap
+
+
+def test_noalloc_refuses_oversized_on_the_host(kolibri_lib):
+    """The size check runs before any CUDA call, so with placeholder pointers
+    an oversized call is refused without a device.  Skipped where a GPU is
+    present: there the GPU test checks the refusal with real buffers."""
+    from conftest import gpu_available
+    if gpu_available():
+        pytest.skip("covered with real buffers by the GPU test")
+    from expert_load_balancing_b200 import binding as B
+    limit = _noalloc_header_limit()
+    fake = ctypes.c_void_p(0x1000)
+    st = kolibri_lib.kolibri_expert_permute_noalloc(fake, limit + 1, 384, 1, fake, fake, fake,
+                                                    None, None)
+    assert st == B.KOLIBRI_ERR_WORKSPACE_TOO_SMALL

@@ -39,13 +39,22 @@ def test_noalloc_matches_workspace_version_twice(N, E, K):
 
 
 def test_noalloc_refuses_oversized():
-    E, K = 384, 6
-    N = 11_182_080 // K + 8192                    # scratch beyond the fixed array
-    ids = torch.zeros((1, K), dtype=torch.int32, device="cuda")
-    lib = B.load()
+    """One slot beyond the fixed array is refused before anything is enqueued.
+    Every buffer has the size the arguments imply (ids, perm and inv of N*K
+    entries), so even a call that got past the size check would stay inside
+    the caller's buffers."""
     import ctypes
-    st = lib.kolibri_expert_permute_noalloc(ctypes.c_void_p(ids.data_ptr()), N, E, K,
-                                            ctypes.c_void_p(ids.data_ptr()),
-                                            ctypes.c_void_p(ids.data_ptr()),
-                                            ctypes.c_void_p(ids.data_ptr()), None, None)
+    E, K = 384, 1
+    N = 11_173_888 + 1                            # the header's limit, plus one slot
+    ids = torch.zeros((N, K), dtype=torch.int32, device="cuda")
+    counts = torch.empty((E,), dtype=torch.int32, device="cuda")
+    offsets = torch.empty((E + 1,), dtype=torch.int64, device="cuda")
+    perm = torch.empty((N * K,), dtype=torch.int32, device="cuda")
+    inv = torch.empty((N * K,), dtype=torch.int32, device="cuda")
+    st = B.load().kolibri_expert_permute_noalloc(
+        ctypes.c_void_p(ids.data_ptr()), N, E, K, ctypes.c_void_p(counts.data_ptr()),
+        ctypes.c_void_p(offsets.data_ptr()), ctypes.c_void_p(perm.data_ptr()),
+        ctypes.c_void_p(inv.data_ptr()), None)
     assert st == B.KOLIBRI_ERR_WORKSPACE_TOO_SMALL
+    torch.cuda.synchronize()
+    assert B.kolibri_device_status() == B.KOLIBRI_OK
