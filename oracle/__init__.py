@@ -66,6 +66,8 @@ def _load():
     lib.oracle_maxvio.restype = f64
     lib.oracle_intervention_rate.argtypes = [P, P, i64, i32]
     lib.oracle_intervention_rate.restype = f64
+    lib.oracle_intervention_overlap.argtypes = [P, P, i64, i32]
+    lib.oracle_intervention_overlap.restype = i64
     lib.oracle_num_threads.restype = ctypes.c_int
     lib.oracle_bf16_round.argtypes = [f32]
     lib.oracle_bf16_round.restype = ctypes.c_uint16
@@ -213,6 +215,15 @@ def intervention_rate(ids_routed, ids_unbiased) -> float:
     b = _c(ids_unbiased, np.int32)
     N, K = a.shape
     return float(_load().oracle_intervention_rate(_ptr(a), _ptr(b), N, K))
+
+
+def intervention_overlap(ids_routed, ids_unbiased) -> int:
+    """Sum over tokens of |I^u_t and I_t| (section 9): the exact count behind
+    the intervention rate, 1 - overlap / (N K)."""
+    a = _c(ids_routed, np.int32)
+    b = _c(ids_unbiased, np.int32)
+    N, K = a.shape
+    return int(_load().oracle_intervention_overlap(_ptr(a), _ptr(b), N, K))
 
 
 def eqb_target_rank(N: int, K: int, E: int) -> int:

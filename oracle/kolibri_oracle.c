@@ -559,6 +559,21 @@ double oracle_intervention_rate(const int32_t *ids_routed, const int32_t *ids_un
     return acc / (double)N;
 }
 
+/* The integer at the heart of the intervention rate of [KPT] 9: the total,
+ * over tokens, of |I^u_t and I_t|, the routed experts that are also among
+ * the router's own top-K.  The ids of one token are distinct, so counting
+ * equal pairs counts the intersection.  rate = 1 - overlap / (N K). */
+int64_t oracle_intervention_overlap(const int32_t *ids_routed, const int32_t *ids_unbiased,
+                                    int64_t N, int32_t K)
+{
+    int64_t total = 0;
+    for (int64_t t = 0; t < N; ++t)
+        for (int32_t a = 0; a < K; ++a)
+            for (int32_t b = 0; b < K; ++b)
+                total += ids_routed[t * K + a] == ids_unbiased[t * K + b];
+    return total;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -144,10 +144,6 @@ def test_score_grad_to_logits_matches_oracle(oracle_mod):
     assert abs(float(host(one)[0]) - 0.105) < 5e-4                    # section 8
 
 
-def _overlaps(ids_a, ids_b):
-    return int(sum(len(set(a) & set(b)) for a, b in zip(ids_a.tolist(), ids_b.tolist())))
-
-
 @pytest.mark.parametrize("N,E,K", [(1, 4, 2), (5000, 384, 6), (4099, 128, 8), (777, 400, 6)])
 def test_intervention_rate_matches_oracle(oracle_mod, N, E, K):
     wl = workloads.Workload("t", N, 64, E, K, beta="normal0.1")
@@ -158,8 +154,8 @@ def test_intervention_rate_matches_oracle(oracle_mod, N, E, K):
     rate, ovl = B.kolibri_intervention_rate(dev(z), dev(ids_routed))
     torch.cuda.synchronize()
     check_status()
-    n_ovl = _overlaps(ids_routed, ids_unb)
-    assert int(host(ovl)[0]) == n_ovl                       # the exact quantity
+    n_ovl = oracle_mod.intervention_overlap(ids_routed, ids_unb)
+    assert int(host(ovl)[0]) == n_ovl                       # the exact quantity, bit for bit
     # the rate is that count in one division; the oracle's mean of N terms
     # carries up to N roundings of its running sum
     assert float(host(rate)[0]) == 1.0 - n_ovl / (N * K)
@@ -178,4 +174,6 @@ def test_intervention_rate_pages_toy(oracle_mod):
     ids_routed, _, _ = oracle_mod.select(z, beta, 2)
     rate, ovl = B.kolibri_intervention_rate(dev(z), dev(ids_routed))
     torch.cuda.synchronize()
-    assert float(host(rate)[0]) == 0.5 and int(host(ovl)[0]) == 4
+    ids_unb, _, _ = oracle_mod.select(z, None, 2)
+    assert int(host(ovl)[0]) == oracle_mod.intervention_overlap(ids_routed, ids_unb) == 4
+    assert float(host(rate)[0]) == 0.5

@@ -419,3 +419,54 @@ def test_eqb_balances_collapsed_router(oracle_mod):
 def test_maxvio_closed_form(oracle_mod):
     assert oracle_mod.maxvio(np.full(8, 5, np.int32), 20, 2) == 0.0
     assert oracle_mod.maxvio(np.array([10, 0, 0, 0], np.int32), 5, 2) == 3.0
+
+
+# ------------------------------- intervention overlap count (section 9)
+
+def test_intervention_overlap_pages_toy(oracle_mod, toy):
+    """The toy re-routed after one EQB step keeps one of its own top-2 per
+    token: 4 tokens x 1 shared expert, which is the rate 0.5 the pages give."""
+    z = np.array(toy["logits_Z"], np.float32)
+    beta = np.array(toy["beta_centred"], np.float32)
+    ids, _, _ = oracle_mod.select(z, beta, toy["K"])
+    ids_u, _, _ = oracle_mod.select(z, None, toy["K"])
+    ovl = oracle_mod.intervention_overlap(ids, ids_u)
+    assert ovl == 4
+    assert 1.0 - ovl / (toy["T"] * toy["K"]) == toy["intervention_rate_after"]
+    # before the update the router routes exactly its own choice
+    assert oracle_mod.intervention_overlap(ids_u, ids_u) == toy["T"] * toy["K"]
+
+
+def test_intervention_overlap_bruteforce(oracle_mod):
+    rng = np.random.default_rng(5)
+    for N, E, K in ((1, 4, 2), (50, 8, 3), (300, 64, 6), (200, 16, 8)):
+        a = np.stack([rng.choice(E, K, replace=False) for _ in range(N)]).astype(np.int32)
+        b = np.stack([rng.choice(E, K, replace=False) for _ in range(N)]).astype(np.int32)
+        want = sum(len(set(x) & set(y)) for x, y in zip(a.tolist(), b.tolist()))
+        assert oracle_mod.intervention_overlap(a, b) == want
+        # order inside a token does not matter, the routed side and the
+        # router's own side may be swapped
+        assert oracle_mod.intervention_overlap(a[:, ::-1].copy(), b) == want
+        assert oracle_mod.intervention_overlap(b, a) == want
+        # disjoint halves of the experts share nothing
+        lo = np.tile(np.arange(K, dtype=np.int32), (N, 1))
+        assert oracle_mod.intervention_overlap(lo, lo + K) == 0
+        # the rate is that count in one division, up to the rounding of the
+        # rate's running mean
+        r = oracle_mod.intervention_rate(a, b)
+        assert abs(r - (1.0 - want / (N * K))) <= N * 2.0 ** -52
+
+
+def test_intervention_overlap_random_routing_mean(oracle_mod):
+    """Random routing against a fixed own choice: each token's overlap is
+    hypergeometric with mean K^2 / E, so the total is N K^2 / E (section 9's
+    closed form 1 - K/E for the rate)."""
+    rng = np.random.default_rng(17)
+    for K, E in ((2, 4), (6, 384), (8, 128)):
+        N = 20000
+        unb = np.tile(np.arange(K, dtype=np.int32), (N, 1))
+        rnd = np.stack([rng.choice(E, size=K, replace=False) for _ in range(N)]).astype(np.int32)
+        ovl = oracle_mod.intervention_overlap(rnd, unb)
+        mean = K * K / E
+        var = K * (K / E) * (1 - K / E) * (E - K) / max(E - 1, 1)
+        assert abs(ovl - N * mean) < 5 * math.sqrt(N * var)
