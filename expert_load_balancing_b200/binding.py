@@ -61,6 +61,11 @@ SIGNATURES = {
     "kolibri_eqb_key_histogram": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P]),
     "kolibri_eqb_key_digit": (ctypes.c_int, [_P, _I32, _I32, _P, _P, _P]),
     "kolibri_eqb_key_bias": (ctypes.c_int, [_P, _I32, _P, _P, _P]),
+    "kolibri_eqb_split_sample": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I64, _P, _P]),
+    "kolibri_eqb_split_brackets": (ctypes.c_int, [_P, _I32, _I64, _I32, _I64, _I32, _P, _P, _P, _P]),
+    "kolibri_eqb_split_count": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P, _P, _I64, _P]),
+    "kolibri_eqb_split_rank": (ctypes.c_int, [_P, _I32, _I64, _I32, _P, _P, _P]),
+    "kolibri_eqb_split_histogram": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _P, _P, _P]),
     "kolibri_expert_ffn_workspace_size": (_SZ, [_I64, _I32, _I32, _I32, _I32]),
     "kolibri_expert_ffn": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32, _I32,
                                           _I32, _I32, _P, _SZ, _P]),
@@ -446,6 +451,55 @@ def kolibri_eqb_key_bias(key, bias, quantiles, stream=None):
     _check("kolibri_eqb_key_bias",
            load().kolibri_eqb_key_bias(_ptr(key), E, _ptr(bias), _ptr(quantiles), _stream(stream)))
     return bias, quantiles
+
+
+def kolibri_eqb_split_sample(z, alpha, K, S, sample, stream=None):
+    """Keys of this rank's z + alpha at S strided rows into sample [E, S] uint32."""
+    N, E = z.shape
+    _check("kolibri_eqb_split_sample",
+           load().kolibri_eqb_split_sample(_ptr(z), _ptr(alpha), N, E, int(K), int(S), _ptr(sample),
+                                           _stream(stream)))
+    return sample
+
+
+def kolibri_eqb_split_brackets(sample, n_total, K, scratch, lo, hi, stream=None):
+    """Brackets lo, hi [E] uint32 from the gathered samples [R, E, S];
+    scratch [E, ld] uint32 with ld = R S rounded up to a multiple of 4."""
+    R, E, S = sample.shape
+    ld = (R * S + 3) // 4 * 4
+    _need(scratch, scratch.dtype, (E, ld), "scratch")
+    _check("kolibri_eqb_split_brackets",
+           load().kolibri_eqb_split_brackets(_ptr(sample), R, S, E, int(n_total), int(K),
+                                             _ptr(scratch), _ptr(lo), _ptr(hi), _stream(stream)))
+    return lo, hi
+
+
+def kolibri_eqb_split_count(z, alpha, K, lo, hi, counts, cand, stream=None):
+    """One pass over this rank's z + alpha: counts [3, E] uint32, cand [E, cap] uint32."""
+    N, E = z.shape
+    cap = cand.shape[1]
+    _check("kolibri_eqb_split_count",
+           load().kolibri_eqb_split_count(_ptr(z), _ptr(alpha), N, E, int(K), _ptr(lo), _ptr(hi),
+                                          _ptr(counts), _ptr(cand), cap, _stream(stream)))
+    return counts, cand
+
+
+def kolibri_eqb_split_rank(counts_sum, n_total, K, rank, flag, stream=None):
+    """rank [E] int64 and flag [E] uint32 from the counts summed over ranks."""
+    E = counts_sum.shape[1]
+    _check("kolibri_eqb_split_rank",
+           load().kolibri_eqb_split_rank(_ptr(counts_sum), E, int(n_total), int(K), _ptr(rank),
+                                         _ptr(flag), _stream(stream)))
+    return rank, flag
+
+
+def kolibri_eqb_split_histogram(cand, counts, pass_, prefix, hist, stream=None):
+    """Add this rank's histogram of its bracketed keys, digit pass pass_, into hist [E, 256]."""
+    E, cap = cand.shape
+    _check("kolibri_eqb_split_histogram",
+           load().kolibri_eqb_split_histogram(_ptr(cand), _ptr(counts), cap, E, int(pass_),
+                                              _ptr(prefix), _ptr(hist), _stream(stream)))
+    return hist
 
 
 def kolibri_lei_inject(counts: torch.Tensor, g: torch.Tensor, K: int, lam: float = 1e-5,

@@ -256,6 +256,63 @@ kolibri_status kolibri_eqb_key_bias(const uint32_t* key, int32_t E, float* bias,
   return from_cuda(launch_bias_update(quantiles, E, bias, quantiles, s));
 }
 
+kolibri_status kolibri_eqb_split_sample(const float* z, const float* alpha, int64_t N, int32_t E,
+                                       int32_t K, int64_t S, uint32_t* sample, void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (S < 1 || S > N) return KOLIBRI_ERR_INVALID_ARG;
+  if (!z || !alpha || !sample || !aligned16(z)) return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_eqb_sample(z, alpha, nullptr, N, E, K, S, N / S, S, sample,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_split_brackets(const uint32_t* sample, int32_t R, int64_t S, int32_t E,
+                                          int64_t N_total, int32_t K, uint32_t* scratch,
+                                          uint32_t* lo, uint32_t* hi, void* stream) {
+  kolibri_status st = check_ek(N_total, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (R < 1 || S < 1 || static_cast<int64_t>(R) * S > N_total) return KOLIBRI_ERR_INVALID_ARG;
+  if (!sample || !scratch || !lo || !hi || !aligned16(scratch)) return KOLIBRI_ERR_INVALID_ARG;
+  const int64_t m = (N_total * static_cast<int64_t>(K)) / E;
+  const int64_t n = static_cast<int64_t>(R) * S;
+  const int64_t ld = (n + 3) & ~static_cast<int64_t>(3);
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t err = launch_dist_sample_transpose(sample, R, S, E, ld, scratch, s);
+  if (err != cudaSuccess) return KOLIBRI_ERR_CUDA;
+  return from_cuda(launch_dist_brackets(scratch, n, ld, E, m, N_total, lo, hi, s));
+}
+
+kolibri_status kolibri_eqb_split_count(const float* z, const float* alpha, int64_t N, int32_t E,
+                                       int32_t K, const uint32_t* lo, const uint32_t* hi,
+                                       uint32_t* counts, uint32_t* cand, int64_t cap,
+                                       void* stream) {
+  kolibri_status st = check_ek(N, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (cap < 1 || !z || !alpha || !lo || !hi || !counts || !cand || !aligned16(z))
+    return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_dist_count(z, alpha, N, E, K, lo, hi, counts, cand, cap,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_split_rank(const uint32_t* counts, int32_t E, int64_t N_total, int32_t K,
+                                      int64_t* rank, uint32_t* flag, void* stream) {
+  kolibri_status st = check_ek(N_total, E, K);
+  if (st != KOLIBRI_OK) return st;
+  if (!counts || !rank || !flag) return KOLIBRI_ERR_INVALID_ARG;
+  const int64_t m = (N_total * static_cast<int64_t>(K)) / E;
+  return from_cuda(launch_dist_rank(counts, E, m, rank, flag, static_cast<cudaStream_t>(stream)));
+}
+
+kolibri_status kolibri_eqb_split_histogram(const uint32_t* cand, const uint32_t* counts,
+                                           int64_t cap, int32_t E, int32_t pass,
+                                           const uint32_t* prefix, uint32_t* hist, void* stream) {
+  if (E < 1 || E > KOLIBRI_MAX_EXPERTS) return KOLIBRI_ERR_UNSUPPORTED_SHAPE;
+  if (cap < 1 || pass < 0 || pass > 3 || !cand || !counts || !hist || (pass > 0 && !prefix))
+    return KOLIBRI_ERR_INVALID_ARG;
+  return from_cuda(launch_dist_cand_hist(cand, counts, cap, E, pass, prefix, hist,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 kolibri_status kolibri_lei_inject(const int32_t* counts, int64_t N, int32_t E, int32_t K,
                                   double lambda, double tau, float* g, void* stream) {
   kolibri_status st = check_ek(N, E, K);

@@ -248,6 +248,66 @@ __global__ void key_value_kernel(const uint32_t* __restrict__ key, int E, float*
   if (e < E) v[e] = key_to_float(key[e]);
 }
 
+// The sampled-bracket update over a split batch.  After this rank's full
+// pass, counts = [above | inside | overflow] per expert: overflow marks an
+// expert whose bracketed keys did not all fit this rank's gather buffer.
+__global__ void dist_count_finish_kernel(uint32_t* __restrict__ counts, int E, int64_t cap) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e < E) counts[2 * E + e] = static_cast<int64_t>(counts[E + e]) > cap ? 1u : 0u;
+}
+
+// The ranks' gathered samples, rank-major [R][E][S], laid out expert-major
+// [E][ld] (rank r's keys of expert e at e ld + r S) for the sample selection.
+__global__ void dist_sample_transpose_kernel(const uint32_t* __restrict__ in, int R, int64_t S,
+                                             int E, int64_t ld, uint32_t* __restrict__ out) {
+  const int64_t total = static_cast<int64_t>(R) * E * S;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t s = i % S, re = i / S;
+    const int64_t e = re % E, r = re / E;
+    out[e * ld + r * S + s] = in[i];
+  }
+}
+
+// From the counts summed over ranks: the target's rank among the bracketed
+// keys, rank[e] = m - above[e], and flag[e] = 1 unless the target lies in
+// the bracket (above <= m < above + inside) and no rank overflowed.
+__global__ void dist_rank_kernel(const uint32_t* __restrict__ counts, int E, int64_t m,
+                                 int64_t* __restrict__ rank, uint32_t* __restrict__ flag) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  const int64_t above = counts[e], inside = counts[E + e];
+  const bool ok = counts[2 * E + e] == 0u && above <= m && m < above + inside;
+  rank[e] = ok ? m - above : 0;
+  flag[e] = ok ? 0u : 1u;
+}
+
+// One radix pass over this rank's bracketed keys of expert e (one block per
+// expert): adds to hist[e] the count per byte 3 - pass among the keys whose
+// top 8 pass bits equal prefix[e], as key_hist_kernel does over Z.
+constexpr int kCandHistThreads = 256;
+__global__ void __launch_bounds__(kCandHistThreads) dist_cand_hist_kernel(
+    const uint32_t* __restrict__ cand, const uint32_t* __restrict__ counts, int64_t cap, int E,
+    int pass, const uint32_t* __restrict__ prefix, uint32_t* __restrict__ hist) {
+  __shared__ uint32_t h[kBins];
+  const int e = blockIdx.x;
+  for (int b = threadIdx.x; b < kBins; b += kCandHistThreads) h[b] = 0u;
+  __syncthreads();
+  const int shift = 24 - 8 * pass;
+  const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
+  const uint32_t pre = pass == 0 ? 0u : (prefix[e] & hi_mask);
+  int64_t n = counts[E + e];
+  if (n > cap) n = cap;   // flagged: the result is discarded
+  const uint32_t* keys = cand + static_cast<int64_t>(e) * cap;
+  for (int64_t i = threadIdx.x; i < n; i += kCandHistThreads) {
+    const uint32_t k = __ldg(keys + i);
+    if ((k & hi_mask) == pre) atomicAdd(&h[(k >> shift) & 0xffu], 1u);
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < kBins; b += kCandHistThreads)
+    if (h[b]) hist[static_cast<int64_t>(e) * kBins + b] += h[b];
+}
+
 // rho_e = c_e / (K N / E) - 1, xi = max |rho| / tau, delta_e = lambda *
 // (tanh(xi)/xi) * rho_e in fp64 (the factor is 1 at xi = 0), rounded once
 // to fp32.  tanh(x) = (1 - e^(-2x)) / (1 + e^(-2x)) with the gate's exp.
@@ -431,6 +491,38 @@ cudaError_t launch_key_digit(const uint32_t* hist, int32_t E, int32_t pass, int6
 
 cudaError_t launch_key_value(const uint32_t* key, int32_t E, float* v, cudaStream_t s) {
   key_value_kernel<<<(E + 255) / 256, 256, 0, s>>>(key, E, v);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dist_count(const float* z, const float* alpha, int64_t N, int32_t E, int32_t K,
+                              const uint32_t* lo, const uint32_t* hi, uint32_t* counts,
+                              uint32_t* cand, int64_t cap, cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(counts, 0, sizeof(uint32_t) * 3 * static_cast<size_t>(E), s);
+  if (err != cudaSuccess) return err;
+  err = launch_route_window_pass(z, nullptr, alpha, N, E, K, nullptr, nullptr, nullptr, lo, hi,
+                                 counts, counts + E, cand, cap, s);
+  if (err != cudaSuccess) return err;
+  dist_count_finish_kernel<<<(E + 255) / 256, 256, 0, s>>>(counts, E, cap);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dist_sample_transpose(const uint32_t* gathered, int32_t R, int64_t S, int32_t E,
+                                         int64_t ld, uint32_t* sample_em, cudaStream_t s) {
+  const int64_t total = static_cast<int64_t>(R) * E * S;
+  dist_sample_transpose_kernel<<<grid_for(total, 256), 256, 0, s>>>(gathered, R, S, E, ld, sample_em);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dist_rank(const uint32_t* counts, int32_t E, int64_t m, int64_t* rank,
+                             uint32_t* flag, cudaStream_t s) {
+  dist_rank_kernel<<<(E + 255) / 256, 256, 0, s>>>(counts, E, m, rank, flag);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dist_cand_hist(const uint32_t* cand, const uint32_t* counts, int64_t cap,
+                                  int32_t E, int32_t pass, const uint32_t* prefix, uint32_t* hist,
+                                  cudaStream_t s) {
+  dist_cand_hist_kernel<<<E, kCandHistThreads, 0, s>>>(cand, counts, cap, E, pass, prefix, hist);
   return cudaGetLastError();
 }
 

@@ -35,30 +35,30 @@ namespace {
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 constexpr int kSelThreads = 512;
-constexpr int kDigitBits = 11;
-constexpr int kBins = 1 << kDigitBits;
+constexpr int kSelWarps = kSelThreads / kWarp;
+constexpr int kMaxRanks = 2;
+constexpr int kHistWords = 2048;   // one 11-bit histogram, or two 10-bit ones
 
-struct SelectSmem {
-  uint32_t hist[kBins];
-  uint32_t red_min[kSelThreads / kWarp];
-  uint32_t red_max[kSelThreads / kWarp];
-  uint32_t bcast[4];
+// Digit width of a selection of R ranks: the R histograms share kHistWords.
+template <int R>
+struct Digits {
+  static constexpr int kBits = R == 1 ? 11 : 10;
+  static constexpr int kBins = 1 << kBits;
+  static_assert(R * kBins <= kHistWords, "histograms exceed their shared region");
+  static_assert(kBins % kSelThreads == 0, "whole bins per thread");
 };
 
-// Exact (rank+1)-th largest key of {key_at(i) : i < n}, rank < n.
-// Skips the bits common to the minimum and maximum key, then resolves the
-// remaining bits most significant first, kDigitBits per pass.  Every thread
-// of the block must call it; the result is returned to all of them.
-template <class KeyAt>
-__device__ uint32_t block_select_desc(KeyAt key_at, int64_t n, int64_t rank, SelectSmem& sm) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nwarps = blockDim.x >> 5;
-  uint32_t mn = 0xffffffffu, mx = 0u;
-  for (int64_t i = tid; i < n; i += blockDim.x) {
-    uint32_t k = key_at(i);
-    mn = k < mn ? k : mn;
-    mx = k > mx ? k : mx;
-  }
+struct SelectSmem {
+  uint32_t hist[kHistWords];
+  uint32_t wsum[kMaxRanks][kSelWarps];
+  uint32_t red_min[kSelWarps];
+  uint32_t red_max[kSelWarps];
+  uint32_t bcast[2 + 2 * kMaxRanks];
+};
+
+// Block-wide minimum and maximum of the per-thread values (all threads).
+__device__ __forceinline__ void block_minmax(uint32_t& mn, uint32_t& mx, SelectSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   mn = __reduce_min_sync(0xffffffffu, mn);
   mx = __reduce_max_sync(0xffffffffu, mx);
   if (lane == 0) {
@@ -67,8 +67,8 @@ __device__ uint32_t block_select_desc(KeyAt key_at, int64_t n, int64_t rank, Sel
   }
   __syncthreads();
   if (warp == 0) {
-    uint32_t a = lane < nwarps ? sm.red_min[lane] : 0xffffffffu;
-    uint32_t b = lane < nwarps ? sm.red_max[lane] : 0u;
+    uint32_t a = lane < kSelWarps ? sm.red_min[lane] : 0xffffffffu;
+    uint32_t b = lane < kSelWarps ? sm.red_max[lane] : 0u;
     a = __reduce_min_sync(0xffffffffu, a);
     b = __reduce_max_sync(0xffffffffu, b);
     if (lane == 0) {
@@ -80,77 +80,145 @@ __device__ uint32_t block_select_desc(KeyAt key_at, int64_t n, int64_t rank, Sel
   mn = sm.bcast[0];
   mx = sm.bcast[1];
   __syncthreads();
-  if (mn == mx) return mn;
+}
+
+// Exact (rank[i]+1)-th largest keys of {key_at(j) : j < n}, rank[i] < n, for
+// R ranks at once, given the block-wide minimum and maximum key.  Bits
+// common to the minimum and maximum are skipped; the rest are resolved most
+// significant first, one digit per pass over the keys.  Each rank follows
+// its own prefix: ranks whose prefixes still agree share one histogram, so
+// the passes serve all ranks.  Per pass: a shared-memory histogram of the
+// digit of the keys that match the prefix, then a block-wide scan of the
+// bins from the top (largest keys first) finds the bin holding the rank.
+// Every thread of the block (kSelThreads) must call it; out[] is returned
+// to all of them.
+template <int R, class KeyAt>
+__device__ void block_select_ranks(KeyAt key_at, int64_t n, const int64_t (&rank)[R],
+                                   uint32_t mn, uint32_t mx, uint32_t (&out)[R], SelectSmem& sm) {
+  using D = Digits<R>;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (mn == mx) {
+#pragma unroll
+    for (int i = 0; i < R; ++i) out[i] = mn;
+    return;
+  }
   int bits_left = 32 - __clz(static_cast<int>(mn ^ mx));  // lowest bits that still differ
-  uint32_t prefix = (bits_left == 32) ? 0u : (mx & ~((1u << bits_left) - 1u));
-  int64_t r = rank;
+  uint32_t prefix[R];
+  int64_t r[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    prefix[i] = (bits_left == 32) ? 0u : (mx & ~((1u << bits_left) - 1u));
+    r[i] = rank[i];
+  }
   while (bits_left > 0) {
-    const int nb = bits_left < kDigitBits ? bits_left : kDigitBits;
+    const int nb = bits_left < D::kBits ? bits_left : D::kBits;
     const int shift = bits_left - nb;
     const int nbins = 1 << nb;
     const uint32_t hi_mask = (shift + nb >= 32) ? 0u : (0xffffffffu << (shift + nb));
-    for (int b = tid; b < nbins; b += blockDim.x) sm.hist[b] = 0u;
+    // histogram h serves rank h; rank 1 reuses histogram 0 while the
+    // prefixes agree
+    const bool split = R > 1 && (prefix[R - 1] & hi_mask) != (prefix[0] & hi_mask);
+    const int nh = split ? R : 1;
+    for (int b = tid; b < nh * D::kBins; b += kSelThreads) sm.hist[b] = 0u;
     __syncthreads();
-    for (int64_t i = tid; i < n; i += blockDim.x) {
-      uint32_t k = key_at(i);
-      if ((k & hi_mask) == (prefix & hi_mask)) atomicAdd(&sm.hist[(k >> shift) & (nbins - 1)], 1u);
+    const uint32_t p0 = prefix[0] & hi_mask, p1 = prefix[R - 1] & hi_mask;
+    for (int64_t j = tid; j < n; j += kSelThreads) {
+      const uint32_t k = key_at(j);
+      const uint32_t kh = k & hi_mask, bin = (k >> shift) & static_cast<uint32_t>(nbins - 1);
+      if (kh == p0) atomicAdd(&sm.hist[bin], 1u);
+      else if (split && kh == p1) atomicAdd(&sm.hist[D::kBins + bin], 1u);
     }
     __syncthreads();
-    if (warp == 0) {
-      // bins are scanned from the top (largest keys first)
-      const int per = (nbins + 31) / 32;
-      // lane 0 owns the top `per` bins, lane 1 the next, ...
-      const int top = nbins - 1 - lane * per;
-      uint32_t part = 0;
-      for (int q = 0; q < per; ++q) {
-        int b = top - q;
-        if (b >= 0) part += sm.hist[b];
-      }
-      // exclusive prefix over lanes (in scan order)
-      uint32_t incl = part;
+    // scan from the top: thread t owns bins top - t*per - q, q < per
+    const int per = nbins >= kSelThreads ? nbins / kSelThreads : 1;
+    const int top = nbins - 1 - tid * per;
+    uint32_t part[R], incl[R];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
+    for (int h = 0; h < R; ++h) {
+      part[h] = 0u;
+      if (h < nh) {
+        for (int q = 0; q < per; ++q)
+          if (top - q >= 0) part[h] += sm.hist[h * D::kBins + top - q];
       }
-      uint32_t excl = incl - part;
-      bool mine = static_cast<int64_t>(excl) <= r && r < static_cast<int64_t>(incl);
-      if (mine) {
-        int64_t rr = r - excl;
-        int b = top;
-        for (int q = 0; q < per; ++q, --b) {
-          uint32_t c = sm.hist[b];
-          if (rr < static_cast<int64_t>(c)) break;
-          rr -= c;
+      incl[h] = part[h];
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+      for (int h = 0; h < R; ++h) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl[h], o);
+        if (lane >= o) incl[h] += t;
+      }
+    }
+    if (lane == 31) {
+#pragma unroll
+      for (int h = 0; h < R; ++h) sm.wsum[h][warp] = incl[h];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < R; ++h) {
+      uint32_t wb = 0u;
+      for (int w = 0; w < warp; ++w) wb += sm.wsum[h][w];
+      const uint32_t ex = wb + incl[h] - part[h];
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int hi = split ? i : 0;
+        if (hi != h) continue;
+        if (part[h] != 0u && static_cast<int64_t>(ex) <= r[i] &&
+            r[i] < static_cast<int64_t>(ex) + part[h]) {
+          int64_t rr = r[i] - ex;
+          int b = top;
+          for (int q = 0; q < per; ++q, --b) {
+            const uint32_t c = sm.hist[h * D::kBins + b];
+            if (rr < static_cast<int64_t>(c)) break;
+            rr -= c;
+          }
+          sm.bcast[2 + 2 * i] = static_cast<uint32_t>(b);
+          sm.bcast[3 + 2 * i] = static_cast<uint32_t>(rr);
         }
-        sm.bcast[2] = static_cast<uint32_t>(b);
-        sm.bcast[3] = static_cast<uint32_t>(rr);
       }
     }
     __syncthreads();
-    prefix |= sm.bcast[2] << shift;
-    r = sm.bcast[3];
+    // (unsplit prefixes are equal: both hold only bits above this digit)
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      prefix[i] |= sm.bcast[2 + 2 * i] << shift;
+      r[i] = sm.bcast[3 + 2 * i];
+    }
     bits_left = shift;
     __syncthreads();
   }
-  return prefix;
+#pragma unroll
+  for (int i = 0; i < R; ++i) out[i] = prefix[i];
 }
 
 // Keys of one expert staged in shared memory when they fit (kSmemKeys),
-// otherwise read from global memory (L2) on every pass.
+// otherwise read from global memory (L2) on every pass.  Either way the
+// block-wide minimum and maximum key come back in mn / mx.
 constexpr int kSmemKeys = 16384;
 
-__device__ __forceinline__ int64_t stage_keys(const uint32_t* __restrict__ keys, int64_t n,
-                                              uint32_t* keys_s) {
-  if (n > kSmemKeys) return n;
+__device__ __forceinline__ void stage_keys(const uint32_t* __restrict__ keys, int64_t n,
+                                           uint32_t* keys_s, uint32_t& mn, uint32_t& mx,
+                                           SelectSmem& sm) {
+  mn = 0xffffffffu;
+  mx = 0u;
+  const bool to_smem = n <= kSmemKeys;
   // 16-byte vector loads only from a 16-byte aligned source
   const bool vec = (reinterpret_cast<uintptr_t>(keys) & 15u) == 0u;
   const int64_t n4 = vec ? (n & ~static_cast<int64_t>(3)) : 0;
-  for (int64_t i = 4 * threadIdx.x; i < n4; i += 4 * blockDim.x)
-    *reinterpret_cast<uint4*>(keys_s + i) = __ldg(reinterpret_cast<const uint4*>(keys + i));
-  for (int64_t i = n4 + threadIdx.x; i < n; i += blockDim.x) keys_s[i] = __ldg(keys + i);
-  __syncthreads();
-  return n;
+  for (int64_t i = 4 * threadIdx.x; i < n4; i += 4 * kSelThreads) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(keys + i));
+    if (to_smem) *reinterpret_cast<uint4*>(keys_s + i) = v;
+    mn = min(min(mn, v.x), min(v.y, min(v.z, v.w)));
+    mx = max(max(mx, v.x), max(v.y, max(v.z, v.w)));
+  }
+  for (int64_t i = n4 + threadIdx.x; i < n; i += kSelThreads) {
+    const uint32_t v = __ldg(keys + i);
+    if (to_smem) keys_s[i] = v;
+    mn = min(mn, v);
+    mx = max(mx, v);
+  }
+  block_minmax(mn, mx, sm);   // its barriers also publish keys_s
 }
 
 // Step 2 (or the whole selection when the sample is the column).
@@ -172,21 +240,26 @@ __global__ void __launch_bounds__(kSelThreads) sample_select_kernel(
     clear_flag[e] = 0u;
   }
   const uint32_t* keys = sample + static_cast<int64_t>(e) * S_ld;
-  stage_keys(keys, S, keys_s);
+  uint32_t mn, mx;
+  stage_keys(keys, S, keys_s, mn, mx, sm);
   const bool in_smem = S <= kSmemKeys;
   auto at = [keys, in_smem](int64_t i) {
     extern __shared__ __align__(16) uint32_t ks[];
     return in_smem ? ks[i] : __ldg(keys + i);
   };
   if (exact) {
-    uint32_t k = block_select_desc(at, S, m_exact, sm);
-    if (threadIdx.x == 0) v[e] = key_to_float(k);
+    const int64_t rk[1] = {m_exact};
+    uint32_t k[1];
+    block_select_ranks<1>(at, S, rk, mn, mx, k, sm);
+    if (threadIdx.x == 0) v[e] = key_to_float(k[0]);
   } else {
-    uint32_t kh = block_select_desc(at, S, r_hi, sm);
-    uint32_t kl = block_select_desc(at, S, r_lo, sm);
+    // both bracket ranks in the same passes (r_hi <= r_lo)
+    const int64_t rk[2] = {r_hi, r_lo};
+    uint32_t k[2];
+    block_select_ranks<2>(at, S, rk, mn, mx, k, sm);
     if (threadIdx.x == 0) {
-      hi[e] = kh;
-      lo[e] = kl;
+      hi[e] = k[0];
+      lo[e] = k[1];
     }
   }
 }
@@ -208,15 +281,18 @@ __global__ void __launch_bounds__(kSelThreads) bracket_select_kernel(
     return;
   }
   const uint32_t* keys = cand + static_cast<int64_t>(e) * cap;
-  stage_keys(keys, c, keys_s);
+  uint32_t mn, mx;
+  stage_keys(keys, c, keys_s, mn, mx, sm);
   const bool in_smem = c <= kSmemKeys;
   auto at = [keys, in_smem](int64_t i) {
     extern __shared__ __align__(16) uint32_t ks[];
     return in_smem ? ks[i] : __ldg(keys + i);
   };
-  uint32_t k = block_select_desc(at, c, m - ab, sm);
+  const int64_t rk[1] = {m - ab};
+  uint32_t k[1];
+  block_select_ranks<1>(at, c, rk, mn, mx, k, sm);
   if (threadIdx.x == 0) {
-    v[e] = key_to_float(k);
+    v[e] = key_to_float(k[0]);
     flag[e] = 0u;
   }
 }
@@ -233,8 +309,17 @@ __global__ void __launch_bounds__(kSelThreads) column_fallback_kernel(
   auto at = [z, alpha, E, e](int64_t t) {
     return order_key(__fadd_rn(__ldg(z + t * E + e), __ldg(alpha + t)));
   };
-  uint32_t k = block_select_desc(at, N, m, sm);
-  if (threadIdx.x == 0) v[e] = key_to_float(k);
+  uint32_t mn = 0xffffffffu, mx = 0u;
+  for (int64_t t = threadIdx.x; t < N; t += kSelThreads) {
+    const uint32_t k = at(t);
+    mn = min(mn, k);
+    mx = max(mx, k);
+  }
+  block_minmax(mn, mx, sm);
+  const int64_t rk[1] = {m};
+  uint32_t k[1];
+  block_select_ranks<1>(at, N, rk, mn, mx, k, sm);
+  if (threadIdx.x == 0) v[e] = key_to_float(k[0]);
 }
 
 // a5: beta = -v, centred.  fp64 sum in ascending expert order (one thread),
@@ -456,5 +541,34 @@ cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t
 }
 
 KOLIBRI_DEFINE_STATUS_TAKE(status_take_eqb)
+
+}  // namespace kolibri
+
+namespace kolibri {
+
+// Brackets of the EQB update over a batch split across ranks: the same
+// sample selection as the one-GPU update, over the ranks' gathered samples
+// laid out expert-major ([E][ld], n keys per expert, ld a multiple of 4).
+cudaError_t launch_dist_brackets(const uint32_t* sample_em, int64_t n, int64_t ld, int32_t E,
+                                 int64_t m, int64_t N_total, uint32_t* lo, uint32_t* hi,
+                                 cudaStream_t s) {
+  // sample ranks about q n with q = (m+1)/N_total, six binomial standard
+  // deviations (plus a few keys) either side, as for one GPU
+  const double q = static_cast<double>(m + 1) / static_cast<double>(N_total);
+  const double center = q * static_cast<double>(n);
+  const double sd = std::sqrt(center * (1.0 - q));
+  const int64_t margin = static_cast<int64_t>(std::ceil(6.0 * sd)) + 8;
+  int64_t r_hi = static_cast<int64_t>(std::floor(center)) - margin;
+  int64_t r_lo = static_cast<int64_t>(std::ceil(center)) + margin;
+  if (r_hi < 0) r_hi = 0;
+  if (r_lo > n - 1) r_lo = n - 1;
+  if (r_hi > r_lo) r_hi = r_lo;
+  cudaError_t err = set_select_smem();
+  if (err != cudaSuccess) return err;
+  return launch_pdl(sample_select_kernel, dim3(E), dim3(kSelThreads), select_smem(n), s,
+                    dim3(0, 0, 0), sample_em, n, static_cast<int64_t>(0), r_hi, r_lo, ld, false,
+                    static_cast<float*>(nullptr), lo, hi, static_cast<uint32_t*>(nullptr),
+                    static_cast<uint32_t*>(nullptr), static_cast<uint32_t*>(nullptr));
+}
 
 }  // namespace kolibri

@@ -175,6 +175,21 @@ cudaError_t launch_key_digit(const uint32_t* hist, int32_t E, int32_t pass, int6
                              uint32_t* prefix, cudaStream_t s);
 cudaError_t launch_key_value(const uint32_t* key, int32_t E, float* v, cudaStream_t s);
 
+// The sampled-bracket EQB update over a split batch (eqb.cu, balance.cu).
+cudaError_t launch_dist_brackets(const uint32_t* sample_em, int64_t n, int64_t ld, int32_t E,
+                                 int64_t m, int64_t N_total, uint32_t* lo, uint32_t* hi,
+                                 cudaStream_t s);
+cudaError_t launch_dist_sample_transpose(const uint32_t* gathered, int32_t R, int64_t S, int32_t E,
+                                         int64_t ld, uint32_t* sample_em, cudaStream_t s);
+cudaError_t launch_dist_count(const float* z, const float* alpha, int64_t N, int32_t E, int32_t K,
+                              const uint32_t* lo, const uint32_t* hi, uint32_t* counts,
+                              uint32_t* cand, int64_t cap, cudaStream_t s);
+cudaError_t launch_dist_rank(const uint32_t* counts, int32_t E, int64_t m, int64_t* rank,
+                             uint32_t* flag, cudaStream_t s);
+cudaError_t launch_dist_cand_hist(const uint32_t* cand, const uint32_t* counts, int64_t cap,
+                                  int32_t E, int32_t pass, const uint32_t* prefix, uint32_t* hist,
+                                  cudaStream_t s);
+
 unsigned status_take_api();
 unsigned status_take_eqb();
 unsigned status_take_noalloc();

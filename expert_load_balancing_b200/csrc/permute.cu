@@ -12,9 +12,9 @@
 //      exclusive prefix; the last block to finish (ticket) scans the totals
 //      into offsets/counts;
 //   C  each block re-sorts its tile in shared memory with a stable counting
-//      sort (__match_any_sync groups a warp's lanes by expert, per-warp
-//      running counters keep slot order), writes inv in slot order and perm
-//      as one contiguous run per expert.
+//      sort (one ballot per bit of the expert id groups a warp's lanes by
+//      expert, per-warp running counters keep slot order), writes inv in
+//      slot order and perm as one contiguous run per expert.
 // Small inputs (decode) run the same steps inside one block.
 #include "launch.h"
 #include "common.cuh"
@@ -31,6 +31,29 @@ constexpr int64_t kTile = static_cast<int64_t>(kPermThreads) * kSlotsPerThread; 
 constexpr int64_t kSingleMax = 4096;    // N*K handled by one block
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Bits that index the experts and a spare value for "no expert": E < 2^bits.
+__host__ __device__ inline int expert_bits(int E) {
+  int b = 1;
+  while ((1 << b) <= E) ++b;
+  return b;
+}
+
+// The lanes of this warp holding the same value v < 2^nbits: the AND, over
+// v's bits, of the ballot of the lanes that agree with it on that bit.  The
+// same mask as __match_any_sync, from vote instructions only.
+__device__ __forceinline__ unsigned lanes_with_value(uint32_t v, int nbits) {
+  unsigned peers = 0xffffffffu;
+#pragma unroll
+  for (int b = 0; b < 10; ++b) {
+    if (b < nbits) {
+      const bool bit = (v >> b) & 1u;
+      const unsigned ones = __ballot_sync(0xffffffffu, bit);
+      peers &= bit ? ones : ~ones;
+    }
+  }
+  return peers;
+}
 
 __global__ void __launch_bounds__(kPermThreads) tile_count_kernel(
     const int32_t* __restrict__ ids, int64_t NK, int E, uint32_t* __restrict__ tile_counts) {
@@ -175,6 +198,7 @@ __global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
   int32_t ex[kSlotsPerThread];
   uint32_t rk[kSlotsPerThread];
   const int64_t w0 = t0 + static_cast<int64_t>(warp) * (kSlotsPerThread * 32);
+  const int nbits = expert_bits(E);   // "no expert" is the value E
 #pragma unroll
   for (int r = 0; r < kSlotsPerThread; ++r) {
     const int64_t j = w0 + r * 32 + lane;
@@ -184,7 +208,7 @@ __global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
 #pragma unroll
   for (int r = 0; r < kSlotsPerThread; ++r) {
     const int32_t e = ex[r];
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const unsigned peers = lanes_with_value(e >= 0 ? static_cast<uint32_t>(e) : static_cast<uint32_t>(E), nbits);
     const uint32_t below = __popc(peers & lt);
     rk[r] = (e >= 0) ? my_cnt[e] + below : 0u;
     __syncwarp();
@@ -241,7 +265,7 @@ __global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
 
 // All three steps in one block (small N*K, decode batches).  Each of the 16
 // warps ranks a contiguous segment of slots (stable inside the segment: the
-// lanes of a round are grouped by expert with __match_any_sync and a per-warp
+// lanes of a round are grouped by expert with one ballot per id bit and a per-warp
 // counter per expert carries the rounds); one thread per expert turns the
 // per-warp counts into starts; a block scan gives the offsets.  Slot order is
 // segment order, then round order, then lane order, which is j order.
@@ -262,6 +286,7 @@ __global__ void __launch_bounds__(kSingleThreads) permute_single_kernel(
   uint32_t* my_cnt = cnt_w[warp];
   for (int e = lane; e < E; e += 32) my_cnt[e] = 0u;
   __syncwarp();
+  const int nbits = expert_bits(E);   // "no expert" is the value E
   pdl_wait();       // ids come from the kernel before this one
   pdl_trigger();
   // ---- segment ranks: this warp's slots [w0, w0 + 32 * rounds)
@@ -278,7 +303,7 @@ __global__ void __launch_bounds__(kSingleThreads) permute_single_kernel(
     if (in && !(x >= 0 && x < E)) bad = true;
     x = (x >= 0 && x < E) ? x : -1;
     ex[r] = x;
-    const unsigned peers = __match_any_sync(0xffffffffu, x);
+    const unsigned peers = lanes_with_value(x >= 0 ? static_cast<uint32_t>(x) : static_cast<uint32_t>(E), nbits);
     const uint32_t below = __popc(peers & lt);
     rk[r] = (x >= 0) ? my_cnt[x] + below : 0u;
     __syncwarp();

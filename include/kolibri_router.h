@@ -342,6 +342,65 @@ KOLIBRI_API kolibri_status kolibri_eqb_key_bias(const uint32_t *key, int32_t E, 
                                                 float *quantiles, void *stream);
 
 /*
+ * kolibri_eqb_update's sampled-bracket design over a batch split across R
+ * ranks ("Kolibri Pre-Training from Scratch" 7.3: each rank holds its own
+ * tokens, only counts cross ranks, every rank ends with the same exact
+ * quantile of the union and the same bias).  Z is read once per rank; the
+ * exchange is one all-gather of the samples, one all-reduce of 3 E counts
+ * and four all-reduces of 256 E counts.  The result equals the four-pass
+ * form above and, on one rank, kolibri_eqb_update, bit for bit.
+ *   kolibri_eqb_split_sample: keys of z + alpha at the S rows t = s (N / S),
+ *     s < S, of this rank's N tokens, written expert-major to sample [E][S]
+ *     (uint32 order keys; 1 <= S <= N).  The caller gathers every rank's
+ *     sample rank-major into [R][E][S] (all-gather; the same S everywhere).
+ *   kolibri_eqb_split_brackets: per expert, two order statistics of the R S
+ *     gathered keys bracket the target (m+1)-th largest of the union, m =
+ *     floor(N_total K / E) (sample ranks about (m+1) R S / N_total, six
+ *     binomial standard deviations apart): keys lo[E] <= hi[E].  The same on
+ *     every rank.  scratch: caller-owned [E][ld] uint32, ld = R S rounded up
+ *     to a multiple of 4, 16-byte aligned (the samples laid out expert-major).
+ *   kolibri_eqb_split_count: one pass over this rank's z + alpha: counts
+ *     [3][E] uint32 = keys above hi, keys in [lo, hi], and 1 where the latter
+ *     exceeded cap; the keys in [lo, hi] go to cand [E][cap].  The caller
+ *     keeps these counts and sums a copy over ranks (all-reduce).
+ *   kolibri_eqb_split_rank: from the summed counts, rank[e] = m - above[e]
+ *     (int64, the target's rank among the bracketed keys of the union) and
+ *     flag[e] = 1 where the target lies outside [lo, hi] or a rank's gather
+ *     overflowed.  If any flag is set (the caller reads flag), the update is
+ *     finished with the four-pass form (kolibri_eqb_key_histogram over z)
+ *     instead; this happens only when the sample misleads.
+ *   kolibri_eqb_split_histogram: pass p (0..3) adds to hist [E][256] the
+ *     counts per byte 3 - p of this rank's bracketed keys (cand, with this
+ *     rank's own counts) whose top 8p bits equal prefix[e]: the gathered keys'
+ *     form of kolibri_eqb_key_histogram.  Then kolibri_eqb_key_digit with
+ *     rank, and after four passes kolibri_eqb_key_bias, as in that form.
+ * Sequence per update: sample; all-gather; brackets; count; all-reduce a
+ * copy of counts; rank; read flag; for p = 0..3 { zero hist; histogram(p);
+ * all-reduce hist; key_digit(p) }; key_bias.  On one rank the exchange
+ * steps are skipped (R = 1).  alpha is required: the token bias of the
+ * routing, as kolibri_router_topk writes it.
+ */
+KOLIBRI_API kolibri_status kolibri_eqb_split_sample(const float *z, const float *alpha, int64_t N,
+                                                    int32_t E, int32_t K, int64_t S,
+                                                    uint32_t *sample, void *stream);
+KOLIBRI_API kolibri_status kolibri_eqb_split_brackets(const uint32_t *sample, int32_t R, int64_t S,
+                                                      int32_t E, int64_t N_total, int32_t K,
+                                                      uint32_t *scratch, uint32_t *lo, uint32_t *hi,
+                                                      void *stream);
+KOLIBRI_API kolibri_status kolibri_eqb_split_count(const float *z, const float *alpha, int64_t N,
+                                                   int32_t E, int32_t K, const uint32_t *lo,
+                                                   const uint32_t *hi, uint32_t *counts,
+                                                   uint32_t *cand, int64_t cap, void *stream);
+KOLIBRI_API kolibri_status kolibri_eqb_split_rank(const uint32_t *counts, int32_t E,
+                                                  int64_t N_total, int32_t K, int64_t *rank,
+                                                  uint32_t *flag, void *stream);
+KOLIBRI_API kolibri_status kolibri_eqb_split_histogram(const uint32_t *cand,
+                                                       const uint32_t *counts, int64_t cap,
+                                                       int32_t E, int32_t pass,
+                                                       const uint32_t *prefix, uint32_t *hist,
+                                                       void *stream);
+
+/*
  * Load-Error Injection ("Kolibri Pre-Training from Scratch" 8) on the score
  * gradient of one microbatch of N tokens:
  *   f_e = counts[e] / (K N / E), rho_e = f_e - 1, xi = max_e |rho_e| / tau,

@@ -81,6 +81,40 @@ def test_fp32_key_passes_checks(lib):
     assert lib.kolibri_eqb_key_bias(F, 0, F, F, None) == SHAPE
 
 
+def test_split_eqb_checks(lib):
+    # the sampled-bracket form over a split batch: every argument error is
+    # refused on the host before anything is enqueued
+    smp = lib.kolibri_eqb_split_sample
+    #            z  alpha N    E    K  S     sample stream
+    assert smp(F, F, 1000, 384, 6, 0, F, None) == INVALID
+    assert smp(F, F, 1000, 384, 6, 1001, F, None) == INVALID       # S > N
+    assert smp(F, None, 1000, 384, 6, 100, F, None) == INVALID     # alpha is required
+    assert smp(ODD, F, 1000, 384, 6, 100, F, None) == INVALID
+    assert smp(F, F, 1000, 386, 6, 100, F, None) == SHAPE          # E % 4
+    br = lib.kolibri_eqb_split_brackets
+    #           sample R  S    E    N_total K scratch lo hi stream
+    assert br(F, 0, 100, 384, 1000, 6, F, F, F, None) == INVALID
+    assert br(F, 4, 300, 384, 1000, 6, F, F, F, None) == INVALID      # R S > N_total
+    assert br(F, 2, 100, 384, 1000, 6, F, F, None, None) == INVALID
+    assert br(F, 2, 100, 384, 1000, 6, ODD, F, F, None) == INVALID    # scratch 16-byte aligned
+    assert br(F, 2, 100, 384, 1000, 400, F, F, F, None) == INVALID    # K >= E
+    cnt = lib.kolibri_eqb_split_count
+    #            z  alpha N    E    K  lo hi counts cand cap stream
+    assert cnt(F, F, 1000, 384, 6, F, F, F, F, 0, None) == INVALID
+    assert cnt(F, F, 1000, 384, 6, F, None, F, F, 64, None) == INVALID
+    assert cnt(ODD, F, 1000, 384, 6, F, F, F, F, 64, None) == INVALID
+    rk = lib.kolibri_eqb_split_rank
+    #           counts E    N_total K rank flag stream
+    assert rk(F, 384, 0, 6, F, F, None) == INVALID
+    assert rk(F, 384, 1000, 6, None, F, None) == INVALID
+    h = lib.kolibri_eqb_split_histogram
+    #          cand counts cap E    pass prefix hist stream
+    assert h(F, F, 64, 384, 4, F, F, None) == INVALID               # pass 0..3
+    assert h(F, F, 64, 384, 1, None, F, None) == INVALID            # prefix from pass 1 on
+    assert h(F, F, 0, 384, 0, None, F, None) == INVALID
+    assert h(F, F, 64, 600, 0, None, F, None) == SHAPE
+
+
 def test_balance_metric_checks(lib):
     lei = lib.kolibri_lei_inject
     #              counts N   E    K  lambda tau  g    stream

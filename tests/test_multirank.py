@@ -1,6 +1,9 @@
-"""The multi-GPU path of bench.py is N independent replicas; its only
-cross-rank steps are the barrier and the max-over-ranks reduction of device
-times.  Checked here with two gloo ranks on the CPU."""
+"""The cross-rank plumbing of bench.py's multi-GPU path: the barrier, the
+max-over-ranks reduction of device times, and the reference arm that runs on
+rank 0 only.  (Its data-path exchange, the EQB update over the union of the
+ranks' tokens, is distributed.eqb_update_split: tests/test_multirank_eqb.py
+on gloo ranks, tests/test_gpu_multirank_eqb.py with the library's kernels.)
+Checked here with two gloo ranks on the CPU."""
 import os
 import socket
 
