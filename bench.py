@@ -8,10 +8,14 @@ Zipf(1.1) expert offsets), inputs resident in HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU (torchrun, one rank per GPU): the path has no exchange step on one
-node, so each rank runs an independent replica of the batch ("replicas
-only", weak scaling); the reported value is all ranks' tokens over the
-slowest rank's device time.
+Multi-GPU (torchrun, one rank per GPU): data parallel, weak scaling.  Each
+rank routes its own batch of N tokens (logits, selection, permutation stay
+local) and the EQB update is the exact quantile of the union of all ranks'
+tokens ("Kolibri Pre-Training from Scratch" 7.3), by the sampled-bracket
+form over NCCL (distributed.eqb_update_split: an all-gather of the samples,
+an all-reduce of 3 E counts, four all-reduces of [E, 256] histograms).  The
+reported value is all ranks' tokens over the slowest rank's device time.
+``--eqb split`` runs that form on one GPU too (no exchange), to time it.
 
 ``--impl reference`` times the CPU oracle on the host cores (bounded sample
 of the same workload per step); it is the slow baseline, not a target.
@@ -55,14 +59,17 @@ def _peaks():
 
 # ---------------------------------------------------------------- algorithmic work
 
-def algorithmic_work(N, d, E, K):
+def algorithmic_work(N, d, E, K, updates=1):
     """FLOPs and bytes a perfect implementation must spend per step.
 
-    GEMM 2 N d E FLOP.  Bytes: x read (2Nd), Z written once and read once
-    (8NE), ids+gates written (8NK), perm+inv written (8NK), alpha (4N), W
-    once (2Ed); counts/offsets/beta are negligible."""
+    GEMM 2 N d E FLOP.  Bytes: x read (2Nd), Z written once (4NE), W once
+    (2Ed); then per routing + EQB update: Z read once (4NE), ids+gates
+    written (8NK), perm+inv written (8NK), alpha (4N).  counts/offsets/beta
+    are negligible.  `updates` > 1 re-routes the same Z with each new bias
+    (the collapsed-router loop)."""
     flops = 2.0 * N * d * E
-    bytes_ = 2.0 * N * d + 8.0 * N * E + 16.0 * N * K + 4.0 * N + 2.0 * E * d
+    bytes_ = (2.0 * N * d + 4.0 * N * E + 2.0 * E * d
+              + updates * (4.0 * N * E + 16.0 * N * K + 4.0 * N))
     return flops, bytes_
 
 
@@ -71,14 +78,27 @@ def gemm_bytes(N, d, E):
     return 2.0 * N * d + 4.0 * N * E + 2.0 * E * d
 
 
-def launches_per_step(N, E, K):
+def launches_per_step(N, E, K, updates=1, split=False):
     """Kernels of ours per step: logits + selection 2 (the fused GEMM and the
-    check for rows it left to the row kernel); EQB update 3 (N <= 16384:
-    sample, exact select, bias) or 6 (sample, bracket, bracketed pass,
-    select, fallback check, bias); permutation 1 or 3."""
-    eqb = 3 if N <= 16384 else 6
+    check for rows it left to the row kernel, or the small-batch logits and
+    the row kernel); EQB update 3 (N <= 16384: sample, exact select, bias)
+    or 6 (sample, bracket, bracketed pass, select, fallback check, bias), or
+    over a split batch 15 (sample, brackets, bracketed pass and its finish,
+    rank, four histogram + digit passes, key value, bias); permutation 1 or
+    3.  Each further update re-routes (1) first."""
+    eqb = 15 if split else (3 if N <= 16384 else 6)
     permute = 1 if N * K <= 4096 else 3
-    return 2 + eqb + permute
+    return 2 + eqb + permute + (updates - 1) * (1 + eqb + permute)
+
+
+def choose_bf16_peak(peaks, clocks, timed_s):
+    """The bf16 peak a tensor-bound fraction is taken against: the burst
+    figure when the timed region is short (under 0.5 s) or the clock record
+    shows no sw_power_cap under load, the sustained one otherwise."""
+    capped = "sw_power_cap" in ((clocks or {}).get("reasons") or [])
+    if timed_s < 0.5 or not capped:
+        return peaks["bf16_tflops"], "burst"
+    return peaks["bf16_tflops_sustained"], "sustained"
 
 
 def reduce_max_over_ranks(value: float, device) -> float:
@@ -159,8 +179,12 @@ class ClockSampler:
 class RouterStep:
     """Buffers and the four calls of one step, all on one stream."""
 
-    def __init__(self, wl, device, seed=0):
+    def __init__(self, wl, device, seed=0, split_eqb=False, world=1):
         self.wl = wl
+        # the EQB update over the union of all ranks' tokens (sampled-bracket form)
+        self.split_eqb = split_eqb
+        self.n_total = wl.N * world
+        self.split_bufs = None
         N, d, E, K = wl.N, wl.d, wl.E, wl.K
         g = torch.Generator(device=device)
         g.manual_seed(1234 + seed)
@@ -197,6 +221,9 @@ class RouterStep:
         of Z) and the permutation.  events (6, optional): start, forward
         done, EQB done, permutation start and end (second stream), step end."""
         wl = self.wl
+        if wl.eqb_updates > 1:
+            self._run_loop(stream, events)
+            return
         if events:
             events[0].record(stream)
         B.kolibri_router_forward(self.x, self.w, self.beta, wl.K, z=self.z, ids=self.ids,
@@ -210,13 +237,66 @@ class RouterStep:
                                  self.perm, self.inv, stream=self.side)
         join = events[4] if events else self.join
         join.record(self.side)
-        B.kolibri_eqb_update(self.z, self.alpha, self.beta, wl.K, self.ws_eqb, self.q,
-                             stream=stream)
+        if self.split_eqb:
+            self._split_update(stream)
+        else:
+            B.kolibri_eqb_update(self.z, self.alpha, self.beta, wl.K, self.ws_eqb, self.q,
+                                 stream=stream)
         if events:
             events[2].record(stream)
         stream.wait_event(join)
         if events:
             events[5].record(stream)
+
+
+    def _split_update(self, stream):
+        """The EQB update over every rank's tokens, sampled-bracket form."""
+        from expert_load_balancing_b200 import distributed as D
+        wl = self.wl
+        if self.split_bufs is None:
+            R = D.DeviceComm().world()
+            S = D.split_sample_rows(wl.N, R)
+            self.split_bufs = D.SplitBuffers(wl.E, S, R, D.CAND_CAP, self.z.device)
+        with torch.cuda.stream(stream):
+            D.eqb_update_split(self.z, self.alpha, self.beta, wl.K, self.n_total,
+                               quantiles=self.q, bufs=self.split_bufs, n_local_min=wl.N)
+
+    def _run_loop(self, stream, events=None):
+        """The collapsed-router loop: the same batch re-routed after every
+        update ("Kolibri Pre-Training from Scratch" 7.2 repairs a collapsed
+        router in one update; this configuration applies ten).  Logits +
+        routing with the initial bias, its permutation and the first update;
+        then per further update the routing with the new bias together with
+        the update (kolibri_route_and_balance) and its permutation.  One
+        stream: each routing's ids feed its permutation.  events as in run();
+        EQB done marks the end of the loop, the permutation events bracket
+        the first permutation."""
+        wl = self.wl
+        ev = events
+        if ev:
+            ev[0].record(stream)
+        with torch.cuda.stream(stream):
+            self.beta.copy_(self.beta0, non_blocking=True)   # every step repairs the collapse anew
+        B.kolibri_router_forward(self.x, self.w, self.beta, wl.K, z=self.z, ids=self.ids,
+                                 gates=self.gates, alpha=self.alpha, stream=stream)
+        if ev:
+            ev[1].record(stream)
+            ev[3].record(stream)
+        B.kolibri_expert_permute(self.ids, wl.E, self.ws_perm, self.counts, self.offsets,
+                                 self.perm, self.inv, stream=stream)
+        if ev:
+            ev[4].record(stream)
+        B.kolibri_eqb_update(self.z, self.alpha, self.beta, wl.K, self.ws_eqb, self.q,
+                             stream=stream)
+        for _ in range(wl.eqb_updates - 1):
+            B.kolibri_route_and_balance(self.z, self.beta, wl.K, self.ws_eqb, ids=self.ids,
+                                        gates=self.gates, alpha=self.alpha, quantiles=self.q,
+                                        stream=stream)
+            B.kolibri_expert_permute(self.ids, wl.E, self.ws_perm, self.counts, self.offsets,
+                                     self.perm, self.inv, stream=stream)
+        if ev:
+            ev[2].record(stream)
+            ev[5].record(stream)
 
 
 def maxvio(counts, wl):
@@ -246,16 +326,22 @@ def run_ours(args, rank, world, local_rank):
         import dataclasses
         wl = dataclasses.replace(wl, N=args.tokens)
     N, d, E, K = wl.N, wl.d, wl.E, wl.K
-    step = RouterStep(wl, device, seed=rank)
+    split_eqb = world > 1 or args.eqb == "split"
+    if split_eqb and wl.eqb_updates > 1:
+        raise SystemExit("the split-batch EQB update runs the one-update step only")
+    step = RouterStep(wl, device, seed=rank, split_eqb=split_eqb, world=world)
     stream = torch.cuda.Stream(device)
     balance = {}
     with torch.cuda.stream(stream):
+        # the loads of the first routing, with the workload's initial bias
+        B.kolibri_router_forward(step.x, step.w, step.beta, wl.K, z=step.z, ids=step.ids,
+                                 gates=step.gates, alpha=step.alpha, stream=stream)
+        B.kolibri_expert_permute(step.ids, wl.E, step.ws_perm, step.counts, step.offsets,
+                                 step.perm, step.inv, stream=stream)
+        stream.synchronize()
+        balance["maxvio_initial_bias"] = maxvio(step.counts, wl)
         for i in range(args.warmup):
             step.run(stream)
-            if i == 0:
-                # the loads of the first routing, with the workload's initial bias
-                torch.cuda.synchronize()
-                balance["maxvio_initial_bias"] = maxvio(step.counts, wl)
     stream.synchronize()
     st = B.kolibri_device_status(stream)
     if st != B.KOLIBRI_OK:
@@ -304,18 +390,35 @@ def run_ours(args, rank, world, local_rank):
 
     if rank != 0:
         return None
+    timed_s = total_ms * 1e-3
+    line = result_line(wl, world, args, ms_per_step, stage_ms, clocks, timed_s, split_eqb)
+    if split_eqb:
+        line["config"]["parallelism"] = (f"dp{world}: tokens split by rank, EQB over the union "
+                                         f"({world * N} tokens), sampled-bracket form")
+    line["e2e"] = e2e
+    line["balance"] = balance
+    line["gpu_name"] = torch.cuda.get_device_name(device)
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    return line
+
+
+def result_line(wl, world, args, ms_per_step, stage_ms, clocks, timed_s, split=False):
+    """The JSON line of one routing-step run: throughput, the fused
+    kernel's roofline (tensor-bound), the EQB update's (HBM-bound), the
+    whole step's against max(FLOP / bf16 peak, bytes / HBM peak)."""
+    N, d, E, K, U = wl.N, wl.d, wl.E, wl.K, wl.eqb_updates
     peaks = _peaks()
-    flops, bytes_ = algorithmic_work(N, d, E, K)
-    roof_ms = max(flops / (peaks["bf16_tflops_sustained"] * 1e12),
-                  bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
+    peak_t, peak_kind = choose_bf16_peak(peaks, clocks, timed_s)
+    flops, bytes_ = algorithmic_work(N, d, E, K, U)
+    roof_ms = max(flops / (peak_t * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
     gemm_ms = float(stage_ms[0])   # the fused GEMM + selection, and the row check after it
     gemm_tflops = 2.0 * N * d * E / (gemm_ms * 1e-3) / 1e12
-    # the timed region runs ~1 s under the 1 kW power cap: the sustained peak
-    peak_t = peaks["bf16_tflops_sustained"]
-    traffic = _traffic_from_profile(N)
+    traffic = _traffic_from_profile(N) if (d, E) == (2560, 384) and N > 1024 else None
+    routed = N * U
     line = {
         "metric": METRIC,
-        "value": world * N / (ms_per_step * 1e-3),
+        "value": world * routed / (ms_per_step * 1e-3),
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
@@ -327,26 +430,40 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "bf16/fp32",
         "data": "synthetic",
         "config": {"workload": wl.name, "N": N, "d": d, "E": E, "K": K, "offsets": wl.offsets,
+                   "beta0": wl.beta, "eqb_updates": U,
                    "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (x %.2f GB, Z %.2f GB)" % (2 * N * d / 1e9, 4 * N * E / 1e9)},
-        "roofline": {"bound": "tensor", "kernel": "router_forward_kernel",
+                   "l2": ("inputs larger than L2 (x %.2f GB, Z %.2f GB)" if 2 * N * d > 126e6 else
+                          "inputs fit in L2 (x %.3f GB, Z %.3f GB); warm, stated so")
+                         % (2 * N * d / 1e9, 4 * N * E / 1e9)},
+        "roofline": {"bound": "tensor", "kernel": "router_forward_kernel" if N > 1024 else
+                     "small_logits_kernel + route_rows_kernel",
                      "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
                      "frac": gemm_tflops / peak_t, "traffic": traffic,
-                     "peak_kind": f"bf16 sustained (cuBLAS, seconds-long loop under the power cap), of {peaks['source']}",
-                     "burst_frac": gemm_tflops / peaks["bf16_tflops"]},
+                     "peak_kind": f"bf16 {peak_kind} (cuBLAS), of {peaks['source']}: "
+                                  f"timed region {timed_s:.3f} s",
+                     "burst_frac": gemm_tflops / peaks["bf16_tflops"],
+                     "sustained_frac": gemm_tflops / peaks["bf16_tflops_sustained"]},
         "path_roofline": {"roofline_ms": roof_ms, "frac": roof_ms / ms_per_step,
                           "flops": flops, "bytes": bytes_,
-                          "peaks": f"bf16 sustained {peaks['bf16_tflops_sustained']} TF/s, HBM {peaks['hbm_gbs']} GB/s, of {peaks['source']}"},
-        "stages_ms": {"logits_and_routing": gemm_ms, "eqb_update": float(stage_ms[1]),
-                      "permute_concurrent": float(stage_ms[2])},
-        "gpu_launches": launches_per_step(N, E, K) * args.steps,
+                          "peaks": f"bf16 {peak_kind} {peak_t} TF/s, HBM {peaks['hbm_gbs']} GB/s, "
+                                   f"of {peaks['source']}"},
+        "stages_ms": {"logits_and_routing": gemm_ms},
+        "gpu_launches": launches_per_step(N, E, K, U, split) * args.steps,
         "clocks": clocks,
-        "e2e": e2e,
-        "balance": balance,
-        "gpu_name": torch.cuda.get_device_name(device),
     }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    if U == 1:
+        eqb_ms = float(stage_ms[1])
+        eqb_bytes = 4.0 * N * E + 4.0 * N        # Z and alpha read once
+        line["stages_ms"]["eqb_update"] = eqb_ms
+        line["stages_ms"]["permute_concurrent"] = float(stage_ms[2])
+        line["eqb_roofline"] = {"bound": "hbm", "achieved": eqb_bytes / (eqb_ms * 1e-3) / 1e9,
+                                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": eqb_bytes / (eqb_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                "algorithmic": "4E + 4 B per token (Z and alpha read once)"}
+    else:
+        line["stages_ms"]["update_loop"] = float(stage_ms[1])
+        line["stages_ms"]["first_permute"] = float(stage_ms[2])
+        line["config"]["routed"] = f"{U} routings of the same N tokens per step (value counts each)"
     return line
 
 
@@ -442,10 +559,12 @@ def _oracle_step(oracle, wl, n_rows, beta):
     w = workloads.bf16_bits(workloads.make_w(wl))
     t = time.perf_counter()
     z = oracle.router_logits(x, w)
-    ids, gates, alpha = oracle.select(z, beta, wl.K)
-    oracle.permute(ids, wl.E)
-    v = oracle.column_quantiles(z, alpha, oracle.eqb_target_rank(n_rows, wl.K, wl.E))
-    oracle.eqb_bias(v)
+    b = beta
+    for _ in range(wl.eqb_updates):      # re-routing with each new bias (collapsed loop)
+        ids, gates, alpha = oracle.select(z, b, wl.K)
+        oracle.permute(ids, wl.E)
+        v = oracle.column_quantiles(z, alpha, oracle.eqb_target_rank(n_rows, wl.K, wl.E))
+        b = oracle.eqb_bias(v)
     return time.perf_counter() - t
 
 
@@ -457,9 +576,10 @@ def cpu_baseline(wl, seconds):
     n_rows = int(max(256, min(wl.N, 256 * seconds / max(t_cal, 1e-3))))
     n_rows = (n_rows // 256) * 256
     t = _oracle_step(oracle, wl, n_rows, beta)
-    return {"value": n_rows / t, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"first {n_rows} tokens of {wl.name} (full d, E, K), one pass of logits, "
-                      f"top-K, permutation and the EQB update over that sample; {t:.1f} s"}
+    return {"value": n_rows * wl.eqb_updates / t, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"first {n_rows} tokens of {wl.name} (full d, E, K), one pass of logits, then "
+                      f"{wl.eqb_updates} x (top-K, permutation, EQB update) over that sample; {t:.1f} s"}
 
 
 def run_reference(args, rank, world):
@@ -479,7 +599,7 @@ def run_reference(args, rank, world):
         _oracle_step(oracle, wl, 256, beta)
     times = [_oracle_step(oracle, wl, n_rows, beta) for _ in range(args.steps)]
     ms = 1e3 * sum(times) / len(times)
-    value = n_rows / (ms * 1e-3)
+    value = n_rows * wl.eqb_updates / (ms * 1e-3)
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -750,6 +870,50 @@ def _decode_oracle(oracle, wl, layers, xs, ws, betas):
     return time.perf_counter() - t
 
 
+def _decode_e2e(args, wl, xs, ws, betas, stream, a, b):
+    """The decode step through the public API with host buffers: every
+    layer's tokens copied in from pinned host memory, the forward + grouping
+    call per layer, and every layer's ids and gates read back, each step."""
+    L, N, d, E, K = wl.layers, wl.N, wl.d, wl.E, wl.K
+    dev = xs[0].device
+    x_h = torch.stack([x.cpu() for x in xs]).pin_memory()
+    ids = torch.empty((L, N, K), dtype=torch.int32, device=dev)
+    gates = torch.empty((L, N, K), dtype=torch.float32, device=dev)
+    ids_h = torch.empty((L, N, K), dtype=torch.int32, pin_memory=True)
+    gates_h = torch.empty((L, N, K), dtype=torch.float32, pin_memory=True)
+    z = torch.empty((N, E), dtype=torch.float32, device=dev)
+    alpha = torch.empty((N,), dtype=torch.float32, device=dev)
+    counts = torch.empty((E,), dtype=torch.int32, device=dev)
+    offsets = torch.empty((E + 1,), dtype=torch.int64, device=dev)
+    perm = torch.empty((N * K,), dtype=torch.int32, device=dev)
+    inv = torch.empty((N * K,), dtype=torch.int32, device=dev)
+    wsp = B.workspace(B.KOLIBRI_OP_PERMUTE, N, E, K, dev)
+
+    def one():
+        with torch.cuda.stream(stream):
+            for l in range(L):
+                xs[l].copy_(x_h[l], non_blocking=True)
+                B.kolibri_router_forward_permute(xs[l], ws[l], betas[l], K, z=z, ids=ids[l],
+                                                 gates=gates[l], alpha=alpha, counts=counts,
+                                                 offsets=offsets, perm=perm, inv=inv, ws=wsp,
+                                                 stream=stream)
+            ids_h.copy_(ids, non_blocking=True)
+            gates_h.copy_(gates, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        one()
+    stream.synchronize()
+    a.record(stream)
+    for _ in range(args.steps):
+        one()
+    b.record(stream)
+    b.synchronize()
+    us = a.elapsed_time(b) * 1e3 / args.steps
+    return {"us_per_step": us, "unit": "us/step", "tokens": N, "path": "eager, one call per layer",
+            "h2d_bytes_per_step": int(x_h.numel() * 2),
+            "d2h_bytes_per_step": int(ids_h.numel() * 4 + gates_h.numel() * 4)}
+
+
 def run_decode(args):
     """The decode sweep: per step, 50 layers of logits + top-K + gates + alpha
     + counts + stable permutation (kolibri_router_forward_permute) for N in
@@ -821,6 +985,8 @@ def run_decode(args):
         if st != B.KOLIBRI_OK:
             raise RuntimeError(f"device status: {B.status_string(st)}")
         res["graph_us_per_layer"] = res["graph_us"] / L
+        if n_tok == workloads.DECODE_TOKENS[-1]:
+            e2e = _decode_e2e(args, wl, xs, ws, betas, stream, a, b)
         # per layer: one launch up to 16 tokens (forward and grouping); else the forward (one launch
         # up to 96 tokens, else logits + selection) and the permutation
         res["gpu_launches"] = (1 if N <= 16 else 2 if N <= 96 else 3) * L
@@ -834,6 +1000,7 @@ def run_decode(args):
     bh = [workloads.make_beta(wl, l).numpy() for l in range(wl.layers)]
     cpu_s = _decode_oracle(oracle, wl, range(wl.layers), xs, wh, bh)
     top = per_n[str(workloads.DECODE_TOKENS[-1])]
+    e2e["value"] = e2e.pop("us_per_step")
     w_bytes = top["w_bytes_per_step"]
     achieved = w_bytes / (top["graph_us"] * 1e-6) / 1e9
     return {
@@ -846,6 +1013,7 @@ def run_decode(args):
                    "tokens": list(workloads.DECODE_TOKENS), "d": 2560, "E": 384, "K": 6,
                    "inputs": "distinct x, W, beta per layer (98 MB of W per step, under L2 size)"},
         "per_n": per_n,
+        "e2e": e2e,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                      "algorithmic": "W read once per layer: 2 E d bytes",
@@ -873,6 +1041,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--eqb", choices=["one", "split"], default="one",
+                    help="split: the EQB update by the split-batch form even on one GPU")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode sweep (50 layers, N = 1, 8, 64, 256; one GPU)")
     ap.add_argument("--part", choices=sorted(PARTS) + ["experts"], default=None,

@@ -39,3 +39,32 @@ def test_maxvio_of_loads():
     assert bench.maxvio(torch.tensor([2, 2, 2, 2], dtype=torch.int32), wl) == 0.0
     # the collapsed toy router of section 7.2: two experts take every slot
     assert bench.maxvio(torch.tensor([4, 0, 0, 4], dtype=torch.int32), wl) == 1.0
+
+
+def test_algorithmic_work_of_the_collapsed_loop():
+    # ten routings + updates over one GEMM's Z: x and the Z write once, then
+    # per update Z read once, ids/gates/perm/inv and alpha
+    N, d, E, K = 16384, 2560, 384, 6
+    flops, bytes_ = bench.algorithmic_work(N, d, E, K, updates=10)
+    assert flops == 2.0 * N * d * E
+    assert bytes_ == 2 * N * d + 4 * N * E + 2 * E * d + 10 * (4 * N * E + 16 * N * K + 4 * N)
+    # one update is the step's own accounting
+    assert bench.algorithmic_work(N, d, E, K, updates=1) == bench.algorithmic_work(N, d, E, K)
+
+
+def test_launches_of_the_collapsed_loop():
+    # forward 2, permutation 3, update 3 (the sample is the column), then nine
+    # times re-route 1 + update 3 + permutation 3
+    assert bench.launches_per_step(16384, 384, 6, updates=10) == 2 + 3 + 3 + 9 * 7
+
+
+@pytest.mark.parametrize("timed_s,reasons,kind", [
+    (0.046, ["sw_power_cap"], "burst"),        # short region: the burst figure
+    (1.0, [], "burst"),                        # long, but never capped
+    (1.0, ["sw_power_cap"], "sustained"),      # long and capped
+])
+def test_bf16_peak_follows_the_run(timed_s, reasons, kind):
+    peaks = {"bf16_tflops": 1622.9, "bf16_tflops_sustained": 1354.4}
+    peak, got = bench.choose_bf16_peak(peaks, {"reasons": reasons}, timed_s)
+    assert got == kind
+    assert peak == (1622.9 if kind == "burst" else 1354.4)
