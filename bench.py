@@ -414,7 +414,9 @@ def result_line(wl, world, args, ms_per_step, stage_ms, clocks, timed_s, split=F
     roof_ms = max(flops / (peak_t * 1e12), bytes_ / (peaks["hbm_gbs"] * 1e9)) * 1e3
     gemm_ms = float(stage_ms[0])   # the fused GEMM + selection, and the row check after it
     gemm_tflops = 2.0 * N * d * E / (gemm_ms * 1e-3) / 1e12
-    traffic = _traffic_from_profile(N) if (d, E) == (2560, 384) and N > 1024 else None
+    # the profiled DRAM bytes per token scale with N only where x and Z stream
+    # through HBM (at and above the 131,072-token capture)
+    traffic = _traffic_from_profile(N) if (d, E) == (2560, 384) and N >= 131072 else None
     routed = N * U
     line = {
         "metric": METRIC,

@@ -24,6 +24,7 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / kWarp;
 constexpr int kRowsPerWarp = 32;     // most rows per warp between gather flushes
 constexpr int kStageSlots = 16;      // staged bracket keys per expert per block
+constexpr int kRowPrefetch = 2;      // rows ahead that the EQB pass prefetches into L2
 
 struct RouteParams {
   const float* z;
@@ -173,6 +174,18 @@ __global__ void __launch_bounds__(kThreads, kAlphaIn ? 4 : 3) route_rows_kernel(
       if (row + 1 < r1) {
         load_row<Q, kFull>(p.z + (row + 1) * E, E, lane, znext);
         if constexpr (kAlphaIn) anext = __ldg(p.alpha_in + row + 1);
+      }
+      if constexpr (kWindow && kAlphaIn) {
+        // the EQB pass streams Z once: the row after next goes to L2 now
+        // (one prefetch per 128-byte line), so each warp has three rows in
+        // flight while holding only two in registers
+        if (row + kRowPrefetch < r1 && (lane & 7) == 0) {
+          const float* pr = p.z + (row + kRowPrefetch) * E;
+#pragma unroll
+          for (int q = 0; q < Q; ++q)
+            if (kFull || 128 * q + 4 * lane < E)
+              asm volatile("prefetch.global.L2 [%0];" ::"l"(pr + 128 * q + 4 * lane));
+        }
       }
 
       float alpha;

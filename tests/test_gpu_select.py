@@ -175,7 +175,8 @@ def test_permute_bad_id_sets_device_status():
 # ------------------------------------------------ EQB, bit-exact
 
 @pytest.mark.parametrize("N,E,K", [(4, 4, 2), (256, 384, 6), (999, 384, 6), (16384, 384, 6),
-                                   (16385, 384, 6), (40000, 128, 8), (70001, 384, 6)])
+                                   (16385, 384, 6), (40000, 128, 8), (70001, 384, 6),
+                                   (20011, 512, 16)])
 def test_eqb_random(oracle_mod, N, E, K):
     z = workloads.random_logits(N, E, seed=N)
     z[:, : max(1, E // 48)] += np.float32(3.0)                # a few collapsed experts
