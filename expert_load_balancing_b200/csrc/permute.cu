@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
 
 // All three steps in one block (small N*K, decode batches).  Each of the 16
 // warps ranks a contiguous segment of slots (stable inside the segment: the
-// lanes of a round are grouped by expert with one ballot per id bit and a per-warp
+// lanes of a round are grouped by expert with __match_any_sync and a per-warp
 // counter per expert carries the rounds); one thread per expert turns the
 // per-warp counts into starts; a block scan gives the offsets.  Slot order is
 // segment order, then round order, then lane order, which is j order.
@@ -286,7 +286,6 @@ __global__ void __launch_bounds__(kSingleThreads) permute_single_kernel(
   uint32_t* my_cnt = cnt_w[warp];
   for (int e = lane; e < E; e += 32) my_cnt[e] = 0u;
   __syncwarp();
-  const int nbits = expert_bits(E);   // "no expert" is the value E
   pdl_wait();       // ids come from the kernel before this one
   pdl_trigger();
   // ---- segment ranks: this warp's slots [w0, w0 + 32 * rounds)
@@ -303,7 +302,9 @@ __global__ void __launch_bounds__(kSingleThreads) permute_single_kernel(
     if (in && !(x >= 0 && x < E)) bad = true;
     x = (x >= 0 && x < E) ? x : -1;
     ex[r] = x;
-    const unsigned peers = lanes_with_value(x >= 0 ? static_cast<uint32_t>(x) : static_cast<uint32_t>(E), nbits);
+    // one block, latency-bound: a single match instruction beats the chain of
+    // per-bit ballots that the tiled scatter uses for throughput
+    const unsigned peers = __match_any_sync(0xffffffffu, x);
     const uint32_t below = __popc(peers & lt);
     rk[r] = (x >= 0) ? my_cnt[x] + below : 0u;
     __syncwarp();
