@@ -39,35 +39,49 @@ __host__ __device__ inline int expert_bits(int E) {
   return b;
 }
 
-// The lanes of this warp holding the same value v < 2^nbits: the AND, over
-// v's bits, of the ballot of the lanes that agree with it on that bit.  The
-// same mask as __match_any_sync, from vote instructions only.
-__device__ __forceinline__ unsigned lanes_with_value(uint32_t v, int nbits) {
+// The lanes of this warp holding the same value v < 2^NB: the AND, over v's
+// bits, of the ballot of the lanes that agree with it on that bit.  The same
+// mask as __match_any_sync, from vote instructions only.  NB is a
+// compile-time count so that the NB ballots are independent and issue back
+// to back.
+template <int NB>
+__device__ __forceinline__ unsigned lanes_with_value(uint32_t v) {
+  unsigned ones[NB];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) ones[b] = __ballot_sync(0xffffffffu, (v >> b) & 1u);
   unsigned peers = 0xffffffffu;
 #pragma unroll
-  for (int b = 0; b < 10; ++b) {
-    if (b < nbits) {
-      const bool bit = (v >> b) & 1u;
-      const unsigned ones = __ballot_sync(0xffffffffu, bit);
-      peers &= bit ? ones : ~ones;
-    }
-  }
+  for (int b = 0; b < NB; ++b) peers &= ((v >> b) & 1u) ? ones[b] : ~ones[b];
   return peers;
 }
 
 __global__ void __launch_bounds__(kPermThreads) tile_count_kernel(
-    const int32_t* __restrict__ ids, int64_t NK, int E, uint32_t* __restrict__ tile_counts) {
+    const int32_t* __restrict__ ids, int64_t NK, int E, uint32_t* __restrict__ tile_counts,
+    uint32_t* __restrict__ ticket) {
   __shared__ uint32_t hist[KOLIBRI_MAX_EXPERTS];
   for (int e = threadIdx.x; e < E; e += kPermThreads) hist[e] = 0u;
+  // ids come from the kernel before this one; once it is complete the next
+  // two kernels of the chain may be scheduled (the scatter reads ids before
+  // its own wait)
+  pdl_wait();
+  pdl_trigger();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;   // read by the scan after this grid
   __syncthreads();
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTile;
+  // every load is issued before the first shared-memory add, so the tile
+  // costs one memory round trip rather than one per slot
+  int32_t x[kSlotsPerThread];
+#pragma unroll
+  for (int u = 0; u < kSlotsPerThread; ++u) {
+    const int64_t j = t0 + u * kPermThreads + threadIdx.x;
+    x[u] = j < NK ? __ldg(ids + j) : 0;
+  }
   bool bad = false;
-#pragma unroll 8
+#pragma unroll
   for (int u = 0; u < kSlotsPerThread; ++u) {
     const int64_t j = t0 + u * kPermThreads + threadIdx.x;
     if (j < NK) {
-      const int32_t x = __ldg(ids + j);
-      if (x >= 0 && x < E) atomicAdd(&hist[x], 1u);
+      if (x[u] >= 0 && x[u] < E) atomicAdd(&hist[x[u]], 1u);
       else bad = true;
     }
   }
@@ -87,6 +101,8 @@ __global__ void __launch_bounds__(kPermThreads) chunk_scan_kernel(
   __shared__ bool last_s;
   const int e = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();       // the tile counts and the ticket
+  pdl_trigger();    // the scatter may start ranking its tile meanwhile
   if (threadIdx.x == 0) carry_s = 0u;
   __syncthreads();
   for (int64_t c0 = 0; c0 < nchunks; c0 += kPermThreads) {
@@ -178,15 +194,17 @@ __device__ __forceinline__ uint32_t block_scan_pairs(uint32_t v0, uint32_t v1, u
 }
 
 // Stable counting sort of one tile in shared memory, then coalesced output.
+// NB: bits of an expert id, with the value E meaning "no expert" (E < 2^NB).
+// Each slot lives in one register from load to store: its expert in the low
+// 10 bits, its rank inside the warp's run of that expert above them.
+template <int NB>
 __global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
     const int32_t* __restrict__ ids, int64_t NK, int E, const uint32_t* __restrict__ tile_prefix,
     const int64_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
   extern __shared__ __align__(16) uint32_t sm[];
   uint32_t* cnt_w = sm;                                   // [kPermWarps][E]
-  uint32_t* lo_e = cnt_w + kPermWarps * E;                // [E] tile-local start of expert e
-  uint32_t* base_e = lo_e + E;                            // [E] global start of e's run
-  uint32_t* sorted = base_e + E;                          // [kTile] slot index by local position
-  uint32_t* sorted_e = sorted + kTile;                    // [kTile] its expert
+  uint32_t* delta_e = cnt_w + kPermWarps * E;             // [E] global minus tile-local start of e's run
+  uint32_t* sorted = delta_e + E;                         // [kTile] (tile slot << 10) | expert
   __shared__ uint32_t warp_sums[kPermWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
@@ -195,28 +213,34 @@ __global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
   for (int e = lane; e < E; e += 32) my_cnt[e] = 0u;
   __syncwarp();
   // ---- phase 1: per-warp stable ranks, 32 consecutive slots per round
-  int32_t ex[kSlotsPerThread];
-  uint32_t rk[kSlotsPerThread];
+  uint32_t xr[kSlotsPerThread];
   const int64_t w0 = t0 + static_cast<int64_t>(warp) * (kSlotsPerThread * 32);
-  const int nbits = expert_bits(E);   // "no expert" is the value E
+  const uint32_t none = static_cast<uint32_t>(E);
 #pragma unroll
   for (int r = 0; r < kSlotsPerThread; ++r) {
+    // ids are complete before the scan this kernel follows was scheduled;
+    // they are read through L2 (.cg), the point of coherence
     const int64_t j = w0 + r * 32 + lane;
-    const int32_t x = j < NK ? __ldg(ids + j) : -1;
-    ex[r] = (x >= 0 && x < E) ? x : -1;
+    const int32_t x = j < NK ? __ldcg(ids + j) : -1;
+    xr[r] = (x >= 0 && x < E) ? static_cast<uint32_t>(x) : none;
   }
 #pragma unroll
   for (int r = 0; r < kSlotsPerThread; ++r) {
-    const int32_t e = ex[r];
-    const unsigned peers = lanes_with_value(e >= 0 ? static_cast<uint32_t>(e) : static_cast<uint32_t>(E), nbits);
+    const uint32_t e = xr[r];
+    const unsigned peers = lanes_with_value<NB>(e);
     const uint32_t below = __popc(peers & lt);
-    rk[r] = (e >= 0) ? my_cnt[e] + below : 0u;
+    const uint32_t rk = (e != none) ? my_cnt[e] + below : 0u;
     __syncwarp();
-    if (e >= 0 && below == 0u) my_cnt[e] += __popc(peers);
+    if (e != none && below == 0u) my_cnt[e] += __popc(peers);
     __syncwarp();
+    xr[r] = e | (rk << 10);
   }
+  // the scan's tile prefixes and offsets; perm and inv are written only
+  // after this wait, so every earlier user of them has finished
+  pdl_wait();
   __syncthreads();
-  // ---- phase 2: warp prefixes per expert, tile-local and global starts
+  // ---- phase 2: per expert, the warps' runs one after another; the
+  // expert's run in the tile after the lower experts' runs
   const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
   uint32_t tot0 = 0u, tot1 = 0u;
   for (int w = 0; w < kPermWarps; ++w) {
@@ -233,33 +257,35 @@ __global__ void __launch_bounds__(kPermThreads, 2) tile_scatter_kernel(
   }
   uint32_t tile_total;
   const uint32_t start0 = block_scan_pairs(tot0, tot1, warp_sums, &tile_total);
-  if (e0 < E) {
-    lo_e[e0] = start0;
-    base_e[e0] = static_cast<uint32_t>(offsets[e0]) + tile_prefix[static_cast<int64_t>(blockIdx.x) * E + e0];
+  const uint32_t start1 = start0 + tot0;
+  // warp starts become tile-local positions
+  for (int w = 0; w < kPermWarps; ++w) {
+    if (e0 < E) cnt_w[w * E + e0] += start0;
+    if (e1 < E) cnt_w[w * E + e1] += start1;
   }
-  if (e1 < E) {
-    lo_e[e1] = start0 + tot0;
-    base_e[e1] = static_cast<uint32_t>(offsets[e1]) + tile_prefix[static_cast<int64_t>(blockIdx.x) * E + e1];
-  }
+  if (e0 < E)
+    delta_e[e0] = static_cast<uint32_t>(offsets[e0]) +
+                  tile_prefix[static_cast<int64_t>(blockIdx.x) * E + e0] - start0;
+  if (e1 < E)
+    delta_e[e1] = static_cast<uint32_t>(offsets[e1]) +
+                  tile_prefix[static_cast<int64_t>(blockIdx.x) * E + e1] - start1;
   __syncthreads();
-  // ---- phase 3: local positions; inv in slot order
+  // ---- phase 3: tile-local positions; inv in slot order
 #pragma unroll
   for (int r = 0; r < kSlotsPerThread; ++r) {
-    const int32_t e = ex[r];
-    if (e >= 0) {
-      const uint32_t within = my_cnt[e] + rk[r];           // position inside e's tile run
-      const uint32_t lpos = lo_e[e] + within;
-      const int64_t j = w0 + r * 32 + lane;
-      sorted[lpos] = static_cast<uint32_t>(j);
-      sorted_e[lpos] = static_cast<uint32_t>(e);
-      if (inv) inv[j] = static_cast<int32_t>(base_e[e] + within);
+    const uint32_t e = xr[r] & 1023u;
+    if (e != none) {
+      const uint32_t lpos = my_cnt[e] + (xr[r] >> 10);
+      const uint32_t jl = static_cast<uint32_t>(warp * (kSlotsPerThread * 32) + r * 32 + lane);
+      sorted[lpos] = (jl << 10) | e;
+      if (inv) inv[t0 + jl] = static_cast<int32_t>(delta_e[e] + lpos);
     }
   }
   __syncthreads();
   // ---- phase 4: perm as one contiguous run per expert
   for (uint32_t pidx = threadIdx.x; pidx < tile_total; pidx += kPermThreads) {
-    const uint32_t e = sorted_e[pidx];
-    perm[base_e[e] + (pidx - lo_e[e])] = static_cast<int32_t>(sorted[pidx]);
+    const uint32_t v = sorted[pidx];
+    perm[delta_e[v & 1023u] + pidx] = static_cast<int32_t>(t0 + (v >> 10));
   }
 }
 
@@ -357,8 +383,8 @@ __global__ void __launch_bounds__(kSingleThreads) permute_single_kernel(
 }  // namespace
 
 size_t tile_scatter_smem(int E) {
-  return sizeof(uint32_t) * (static_cast<size_t>(kPermWarps) * E + 2 * static_cast<size_t>(E) +
-                             2 * static_cast<size_t>(kTile));
+  return sizeof(uint32_t) * (static_cast<size_t>(kPermWarps) * E + static_cast<size_t>(E) +
+                             static_cast<size_t>(kTile));
 }
 
 PermuteLayout permute_layout(int64_t N, int32_t E, int32_t K) {
@@ -391,20 +417,22 @@ cudaError_t launch_permute(const int32_t* ids, int64_t N, int32_t E, int32_t K, 
   uint32_t* tile_counts = reinterpret_cast<uint32_t*>(base + L.off_chunk_counts);
   uint32_t* totals = reinterpret_cast<uint32_t*>(base + L.off_counts);
   uint32_t* ticket = reinterpret_cast<uint32_t*>(base + L.off_ticket);
-  cudaError_t err = cudaMemsetAsync(ticket, 0, sizeof(uint32_t), s);
-  if (err != cudaSuccess) return err;
   const unsigned tiles = static_cast<unsigned>(L.nchunks);
-  tile_count_kernel<<<tiles, kPermThreads, 0, s>>>(ids, NK, E, tile_counts);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  chunk_scan_kernel<<<E, kPermThreads, 0, s>>>(tile_counts, L.nchunks, E, totals, ticket, counts,
-                                               offsets);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const size_t smem = tile_scatter_smem(E);
-  err = cudaFuncSetAttribute(tile_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+  const int nb = expert_bits(E);   // E itself stands for "no expert"
+  auto kern = nb <= 8 ? tile_scatter_kernel<8> : nb <= 9 ? tile_scatter_kernel<9> : tile_scatter_kernel<10>;
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  tile_scatter_kernel<<<tiles, kPermThreads, smem, s>>>(ids, NK, E, tile_counts, offsets, perm, inv);
-  return cudaGetLastError();
+  // a chain of programmatic dependent launches: see each kernel's waits
+  err = launch_pdl(tile_count_kernel, dim3(tiles), dim3(kPermThreads), 0, s, dim3(0, 0, 0), ids, NK, E,
+                   tile_counts, ticket);
+  if (err != cudaSuccess) return err;
+  err = launch_pdl(chunk_scan_kernel, dim3(static_cast<unsigned>(E)), dim3(kPermThreads), 0, s,
+                   dim3(0, 0, 0), tile_counts, L.nchunks, E, totals, ticket, counts, offsets);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(kern, dim3(tiles), dim3(kPermThreads), smem, s, dim3(0, 0, 0), ids, NK, E,
+                    static_cast<const uint32_t*>(tile_counts), static_cast<const int64_t*>(offsets), perm, inv);
 }
 
 KOLIBRI_DEFINE_STATUS_TAKE(status_take_permute)

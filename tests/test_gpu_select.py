@@ -135,7 +135,11 @@ def test_gates_unchanged_by_bias():
                                    (40000, 128, 8), (12345, 16, 3),
                                    # one block up to N*K = 4096: its edges
                                    (512, 512, 8), (4096, 16, 1), (1, 512, 16), (13, 48, 5),
-                                   (4097, 16, 1)])
+                                   (4097, 16, 1),
+                                   # tiled path at each width of the expert-id grouping
+                                   # (E itself marks an empty slot: 8 bits up to E = 252,
+                                   # 9 bits up to 511, 10 bits at 512)
+                                   (9001, 252, 3), (7000, 256, 4), (3000, 512, 8)])
 def test_permute(oracle_mod, N, E, K):
     rng = np.random.default_rng(N)
     ids = np.stack([rng.choice(E, size=K, replace=False) for _ in range(N)]).astype(np.int32)
