@@ -221,6 +221,41 @@ __device__ __forceinline__ void stage_keys(const uint32_t* __restrict__ keys, in
   block_minmax(mn, mx, sm);   // its barriers also publish keys_s
 }
 
+// a5 by the last block of an update's final grid: beta = -v, centred, with
+// the arithmetic of bias_update_kernel (fp64 sum in ascending expert order by
+// one thread, mean rounded once to fp32, subtraction in fp32).  Every block
+// calls it after thread 0 wrote its v[e]; each makes that write visible
+// (fence) and takes a ticket; the block drawing the last ticket reads all E
+// values and updates the bias, then puts the ticket back to zero.  No block
+// waits for another.  The ticket must be zero when the grid starts.
+__device__ void bias_by_last_block(const float* v, int E, uint32_t* ticket, float* bias,
+                                   float* quantiles, SelectSmem& sm) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    sm.bcast[0] = (atomicAdd(ticket, 1u) == gridDim.x - 1u) ? 1u : 0u;
+  }
+  __syncthreads();
+  if (sm.bcast[0] == 0u) return;
+  __threadfence();
+  float* v_s = reinterpret_cast<float*>(sm.hist);       // E <= 512 < kHistWords
+  for (int e = threadIdx.x; e < E; e += kSelThreads) v_s[e] = __ldcg(v + e);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double sum = 0.0;
+    for (int e = 0; e < E; ++e) sum = __dadd_rn(sum, static_cast<double>(-v_s[e]));
+    sm.red_min[0] = __float_as_uint(__double2float_rn(__ddiv_rn(sum, static_cast<double>(E))));
+    *ticket = 0u;
+  }
+  __syncthreads();
+  const float mean = __uint_as_float(sm.red_min[0]);
+  for (int e = threadIdx.x; e < E; e += kSelThreads) {
+    const float ve = v_s[e];
+    bias[e] = __fsub_rn(-ve, mean);
+    if (quantiles) quantiles[e] = ve;
+  }
+}
+
 // Step 2 (or the whole selection when the sample is the column).
 // The bracket path also clears this expert's counters of the full pass
 // (clear non-null: above, cnt, flag).
@@ -228,7 +263,8 @@ __global__ void __launch_bounds__(kSelThreads) sample_select_kernel(
     const uint32_t* __restrict__ sample, int64_t S, int64_t m_exact, int64_t r_hi, int64_t r_lo,
     int64_t S_ld, bool exact, float* __restrict__ v, uint32_t* __restrict__ lo,
     uint32_t* __restrict__ hi, uint32_t* __restrict__ clear_above, uint32_t* __restrict__ clear_cnt,
-    uint32_t* __restrict__ clear_flag) {
+    uint32_t* __restrict__ clear_flag, uint32_t* __restrict__ ticket, float* __restrict__ bias,
+    float* __restrict__ quantiles) {
   __shared__ SelectSmem sm;
   extern __shared__ __align__(16) uint32_t keys_s[];
   const int e = blockIdx.x;
@@ -252,6 +288,8 @@ __global__ void __launch_bounds__(kSelThreads) sample_select_kernel(
     uint32_t k[1];
     block_select_ranks<1>(at, S, rk, mn, mx, k, sm);
     if (threadIdx.x == 0) v[e] = key_to_float(k[0]);
+    // ticket given: this grid also ends the update (bias from all v)
+    if (ticket != nullptr) bias_by_last_block(v, static_cast<int>(gridDim.x), ticket, bias, quantiles, sm);
   } else {
     // both bracket ranks in the same passes (r_hi <= r_lo)
     const int64_t rk[2] = {r_hi, r_lo};
@@ -264,62 +302,53 @@ __global__ void __launch_bounds__(kSelThreads) sample_select_kernel(
   }
 }
 
-// Step 4.
-__global__ void __launch_bounds__(kSelThreads) bracket_select_kernel(
+// Steps 4-5 and a5 in one grid, one block per expert.  If the target lies
+// inside the expert's bracket (above <= m < above + inside, and the gather
+// did not overflow), v is the (m - above)-th largest gathered key; otherwise
+// the block selects over the whole column of Z + alpha.  The block drawing
+// the last ticket then updates the bias.
+__global__ void __launch_bounds__(kSelThreads) bracket_finish_kernel(
     const uint32_t* __restrict__ cand, const uint32_t* __restrict__ cnt,
-    const uint32_t* __restrict__ above, int64_t cap, int64_t m, float* __restrict__ v,
-    uint32_t* __restrict__ flag) {
+    const uint32_t* __restrict__ above, int64_t cap, int64_t m, const float* __restrict__ z,
+    const float* __restrict__ alpha, int64_t N, float* __restrict__ v, uint32_t* __restrict__ ticket,
+    float* __restrict__ bias, float* __restrict__ quantiles) {
   __shared__ SelectSmem sm;
   extern __shared__ __align__(16) uint32_t keys_s[];
   const int e = blockIdx.x;
+  const int E = static_cast<int>(gridDim.x);
   pdl_wait();       // counts and gathered keys come from the full pass
   pdl_trigger();
   const int64_t c = cnt[e], ab = above[e];
   const bool ok = c <= cap && ab <= m && m < ab + c;
-  if (!ok) {
-    if (threadIdx.x == 0) flag[e] = 1u;
-    return;
-  }
-  const uint32_t* keys = cand + static_cast<int64_t>(e) * cap;
-  uint32_t mn, mx;
-  stage_keys(keys, c, keys_s, mn, mx, sm);
-  const bool in_smem = c <= kSmemKeys;
-  auto at = [keys, in_smem](int64_t i) {
-    extern __shared__ __align__(16) uint32_t ks[];
-    return in_smem ? ks[i] : __ldg(keys + i);
-  };
-  const int64_t rk[1] = {m - ab};
   uint32_t k[1];
-  block_select_ranks<1>(at, c, rk, mn, mx, k, sm);
-  if (threadIdx.x == 0) {
-    v[e] = key_to_float(k[0]);
-    flag[e] = 0u;
+  if (ok) {
+    const uint32_t* keys = cand + static_cast<int64_t>(e) * cap;
+    uint32_t mn, mx;
+    stage_keys(keys, c, keys_s, mn, mx, sm);
+    const bool in_smem = c <= kSmemKeys;
+    auto at = [keys, in_smem](int64_t i) {
+      extern __shared__ __align__(16) uint32_t ks[];
+      return in_smem ? ks[i] : __ldg(keys + i);
+    };
+    const int64_t rk[1] = {m - ab};
+    block_select_ranks<1>(at, c, rk, mn, mx, k, sm);
+  } else {
+    // the bracket missed (or its gather overflowed): the whole column
+    auto at = [z, alpha, E, e](int64_t t) {
+      return order_key(__fadd_rn(__ldg(z + t * E + e), __ldg(alpha + t)));
+    };
+    uint32_t mn = 0xffffffffu, mx = 0u;
+    for (int64_t t = threadIdx.x; t < N; t += kSelThreads) {
+      const uint32_t kk = at(t);
+      mn = min(mn, kk);
+      mx = max(mx, kk);
+    }
+    block_minmax(mn, mx, sm);
+    const int64_t rk[1] = {m};
+    block_select_ranks<1>(at, N, rk, mn, mx, k, sm);
   }
-}
-
-// Step 5: radix selection over the whole column of the flagged experts.
-__global__ void __launch_bounds__(kSelThreads) column_fallback_kernel(
-    const float* __restrict__ z, const float* __restrict__ alpha, int64_t N, int E, int64_t m,
-    const uint32_t* __restrict__ flag, float* __restrict__ v) {
-  __shared__ SelectSmem sm;
-  const int e = blockIdx.x;
-  pdl_wait();
-  pdl_trigger();
-  if (flag[e] == 0u) return;
-  auto at = [z, alpha, E, e](int64_t t) {
-    return order_key(__fadd_rn(__ldg(z + t * E + e), __ldg(alpha + t)));
-  };
-  uint32_t mn = 0xffffffffu, mx = 0u;
-  for (int64_t t = threadIdx.x; t < N; t += kSelThreads) {
-    const uint32_t k = at(t);
-    mn = min(mn, k);
-    mx = max(mx, k);
-  }
-  block_minmax(mn, mx, sm);
-  const int64_t rk[1] = {m};
-  uint32_t k[1];
-  block_select_ranks<1>(at, N, rk, mn, mx, k, sm);
   if (threadIdx.x == 0) v[e] = key_to_float(k[0]);
+  bias_by_last_block(v, E, ticket, bias, quantiles, sm);
 }
 
 // a5: beta = -v, centred.  fp64 sum in ascending expert order (one thread),
@@ -385,7 +414,7 @@ cudaError_t set_select_smem() {
   cudaError_t err = cudaFuncSetAttribute(sample_select_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (err != cudaSuccess) return err;
-  return cudaFuncSetAttribute(bracket_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(bracket_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               bytes);
 }
 
@@ -413,9 +442,11 @@ EqbBuffers eqb_buffers(int64_t N, int32_t E, int32_t K, void* ws) {
   return b;
 }
 
-// Step 2 from the sample keys: either the exact quantile (small N) or the
-// per-expert bracket, with the full-pass counters cleared.
-cudaError_t eqb_brackets(int64_t N, int32_t E, int32_t K, const EqbBuffers& b, cudaStream_t s) {
+// Step 2 from the sample keys: either the exact quantile and the bias update
+// (small N: the sample is the column), or the per-expert bracket, with the
+// full-pass counters cleared.
+cudaError_t eqb_brackets(int64_t N, int32_t E, int32_t K, const EqbBuffers& b, float* bias,
+                         float* quantiles, cudaStream_t s) {
   const EqbLayout& L = b.L;
   const int64_t m = (N * static_cast<int64_t>(K)) / E;
   cudaError_t err;
@@ -425,7 +456,7 @@ cudaError_t eqb_brackets(int64_t N, int32_t E, int32_t K, const EqbBuffers& b, c
     return launch_pdl(sample_select_kernel, dim3(E), dim3(kSelThreads), select_smem(L.S), s, dim3(0, 0, 0),
                       b.sample, L.S, m, static_cast<int64_t>(0), static_cast<int64_t>(0), L.S_ld, true, b.v,
                       b.lo, b.hi, static_cast<uint32_t*>(nullptr), static_cast<uint32_t*>(nullptr),
-                      static_cast<uint32_t*>(nullptr));
+                      static_cast<uint32_t*>(nullptr), b.flag, bias, quantiles);
   }
   // bracket ranks in the sample, descending order: the target sits at
   // about q*S with q = (m+1)/N; margin 6 binomial standard deviations
@@ -442,36 +473,34 @@ cudaError_t eqb_brackets(int64_t N, int32_t E, int32_t K, const EqbBuffers& b, c
   // the select also clears the full pass's counters (above, cnt, flag)
   return launch_pdl(sample_select_kernel, dim3(E), dim3(kSelThreads), select_smem(L.S), s, dim3(0, 0, 0),
                     b.sample, L.S, static_cast<int64_t>(0), r_hi, r_lo, L.S_ld, false, b.v, b.lo, b.hi,
-                    b.above, b.cnt, b.flag);
+                    b.above, b.cnt, b.flag, static_cast<uint32_t*>(nullptr), static_cast<float*>(nullptr),
+                    static_cast<float*>(nullptr));
 }
 
-// Steps 1-2: sample keys (token bias given, or computed from bias_in), then
-// the brackets (or the exact quantile for small N).
-cudaError_t eqb_begin(const float* z, const float* alpha, const float* bias, int64_t N, int32_t E,
-                      int32_t K, const EqbBuffers& b, cudaStream_t s) {
+// Steps 1-2: sample keys (token bias given, or computed from the bias), then
+// the brackets, or for small N the exact quantile and the bias update.  The
+// word b.flag[0] is the ticket of the grid that ends the update: cleared
+// by the sample kernel (small N) or by the sample select (the bracket path).
+cudaError_t eqb_begin(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
+                      int32_t K, float* quantiles, const EqbBuffers& b, cudaStream_t s) {
   const EqbLayout& L = b.L;
   cudaError_t err = launch_eqb_sample(z, alpha, alpha ? nullptr : bias, N, E, K, L.S, L.stride,
-                                      L.S_ld, b.sample, s);
+                                      L.S_ld, b.sample, s, L.exact_small ? b.flag : nullptr);
   if (err != cudaSuccess) return err;
-  return eqb_brackets(N, E, K, b, s);
+  return eqb_brackets(N, E, K, b, bias, quantiles, s);
 }
 
-// Steps 4-5 and the bias update.
+// Steps 4-5 and the bias update, in one grid (the bracket path; for small N
+// eqb_begin already finished the update).
 cudaError_t eqb_end(const float* z, const float* alpha_used, float* bias, int64_t N, int32_t E,
                     int32_t K, float* quantiles, const EqbBuffers& b, cudaStream_t s) {
+  if (b.L.exact_small) return cudaSuccess;
   const int64_t m = (N * static_cast<int64_t>(K)) / E;
-  cudaError_t err;
-  if (!b.L.exact_small) {
-    err = set_select_smem();
-    if (err != cudaSuccess) return err;
-    err = launch_pdl(bracket_select_kernel, dim3(E), dim3(kSelThreads), select_smem(kSmemKeys), s,
-                     dim3(0, 0, 0), b.cand, b.cnt, b.above, static_cast<int64_t>(kCandCap), m, b.v, b.flag);
-    if (err != cudaSuccess) return err;
-    err = launch_pdl(column_fallback_kernel, dim3(E), dim3(kSelThreads), 0, s, dim3(0, 0, 0), z, alpha_used, N,
-                     E, m, b.flag, b.v);
-    if (err != cudaSuccess) return err;
-  }
-  return launch_pdl(bias_update_kernel, dim3(1), dim3(512), 0, s, dim3(0, 0, 0), b.v, E, bias, quantiles);
+  const cudaError_t err = set_select_smem();
+  if (err != cudaSuccess) return err;
+  return launch_pdl(bracket_finish_kernel, dim3(E), dim3(kSelThreads), select_smem(kSmemKeys), s,
+                    dim3(0, 0, 0), b.cand, b.cnt, b.above, static_cast<int64_t>(kCandCap), m, z, alpha_used, N,
+                    b.v, b.flag, bias, quantiles);
 }
 
 }  // namespace
@@ -484,7 +513,7 @@ cudaError_t launch_bias_update(const float* v, int32_t E, float* bias, float* qu
 cudaError_t launch_eqb(const float* z, const float* alpha, float* bias, int64_t N, int32_t E,
                        int32_t K, float* quantiles, void* ws, cudaStream_t s) {
   const EqbBuffers b = eqb_buffers(N, E, K, ws);
-  cudaError_t err = eqb_begin(z, alpha, bias, N, E, K, b, s);
+  cudaError_t err = eqb_begin(z, alpha, bias, N, E, K, quantiles, b, s);
   if (err != cudaSuccess) return err;
   const float* alpha_used = alpha;
   if (!b.L.exact_small) {
@@ -523,7 +552,7 @@ cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t
     // the sample is the whole column: route first, then select from its alpha
     err = launch_topk(z, bias, N, E, K, ids, gates, alpha_out, s);
     if (err != cudaSuccess) return err;
-    err = eqb_begin(z, alpha_out, bias, N, E, K, b, s);
+    err = eqb_begin(z, alpha_out, bias, N, E, K, quantiles, b, s);
     if (err != cudaSuccess) return err;
   } else {
     // Routing first (writes alpha), then the bracketed pass with alpha given.
@@ -531,7 +560,7 @@ cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t
     // per-row dependency chain is longer than 24 warps per SM can hide).
     err = launch_topk(z, bias, N, E, K, ids, gates, alpha_out, s);
     if (err != cudaSuccess) return err;
-    err = eqb_begin(z, alpha_out, bias, N, E, K, b, s);
+    err = eqb_begin(z, alpha_out, bias, N, E, K, quantiles, b, s);
     if (err != cudaSuccess) return err;
     err = launch_route_window_pass(z, bias, alpha_out, N, E, K, nullptr, nullptr, nullptr, b.lo,
                                    b.hi, b.above, b.cnt, b.cand, kCandCap, s);
@@ -568,7 +597,8 @@ cudaError_t launch_dist_brackets(const uint32_t* sample_em, int64_t n, int64_t l
   return launch_pdl(sample_select_kernel, dim3(E), dim3(kSelThreads), select_smem(n), s,
                     dim3(0, 0, 0), sample_em, n, static_cast<int64_t>(0), r_hi, r_lo, ld, false,
                     static_cast<float*>(nullptr), lo, hi, static_cast<uint32_t*>(nullptr),
-                    static_cast<uint32_t*>(nullptr), static_cast<uint32_t*>(nullptr));
+                    static_cast<uint32_t*>(nullptr), static_cast<uint32_t*>(nullptr),
+                    static_cast<uint32_t*>(nullptr), static_cast<float*>(nullptr), static_cast<float*>(nullptr));
 }
 
 }  // namespace kolibri

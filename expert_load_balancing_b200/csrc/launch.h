@@ -133,9 +133,11 @@ cudaError_t launch_route_balance(const float* z, float* bias, int64_t N, int32_t
                                  void* ws, cudaStream_t s);
 
 // pieces of the EQB update living in route.cu (they walk rows of Z)
+// zero_word (nullable): a word the sampling kernel sets to zero for the
+// kernels after it.
 cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* bias, int64_t N,
                               int32_t E, int32_t K, int64_t S, int64_t stride, int64_t S_ld,
-                              uint32_t* sample, cudaStream_t s);
+                              uint32_t* sample, cudaStream_t s, uint32_t* zero_word = nullptr);
 // Bracketed full pass.  alpha_in given: use it.  Otherwise alpha is derived
 // from bias (and written to alpha_out); with ids/gates non-null the same
 // pass also writes the routing.

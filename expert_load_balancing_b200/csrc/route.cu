@@ -293,13 +293,14 @@ __global__ void __launch_bounds__(kThreads, kAlphaIn ? 4 : 3) route_rows_kernel(
 // Keys of Z + alpha at sampled rows t = s * stride, written expert-major:
 // sample[e * S + s].  A block handles 32 consecutive samples and transposes
 // them through shared memory so every expert row is written in 128-byte runs.
+// zero_word (nullable) is cleared by block 0 for the kernels after this one.
 constexpr int kSampleRows = 32;
 
 template <int Q, bool kAlphaIn, bool kBias>
 __global__ void __launch_bounds__(kThreads) sample_keys_kernel(
     const float* __restrict__ z, const float* __restrict__ alpha_in, const float* __restrict__ beta,
     int64_t N, int E, int K, int64_t S, int64_t stride, int64_t S_ld,
-    uint32_t* __restrict__ sample) {
+    uint32_t* __restrict__ sample, uint32_t* __restrict__ zero_word) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int V = 4 * Q;
   const int ld = E + 1;
@@ -312,6 +313,7 @@ __global__ void __launch_bounds__(kThreads) sample_keys_kernel(
   const int64_t s0 = static_cast<int64_t>(blockIdx.x) * kSampleRows;
   pdl_wait();       // Z and alpha come from the kernels before this one
   pdl_trigger();
+  if (zero_word != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0u;
   if constexpr (kBias) {
     for (int e = threadIdx.x; e < E; e += kThreads) beta_s[e] = beta[e];
   }
@@ -320,6 +322,33 @@ __global__ void __launch_bounds__(kThreads) sample_keys_kernel(
 #pragma unroll
   for (int j = 0; j < V; ++j) valid |= (static_cast<int>(slot_expert(lane, j)) < E) ? (1u << j) : 0u;
 
+  if constexpr (kAlphaIn) {
+    // the warp's rows r = warp + kWarps i: every load issued before the first
+    // use, one memory round trip
+    constexpr int kPerWarp = kSampleRows / kWarps;
+    float zv[kPerWarp][V];
+    float al[kPerWarp];
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+      const int64_t s = s0 + warp + kWarps * i;
+      al[i] = 0.f;
+      if (s < S) {
+        const int64_t row = s * stride;
+        load_row<Q, false>(z + row * E, E, lane, zv[i]);
+        al[i] = __ldg(alpha_in + row);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kPerWarp; ++i) {
+      const int r = warp + kWarps * i;
+      if (s0 + r >= S) break;
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const int e = static_cast<int>(slot_expert(lane, j));
+        if (e < E) tile[r * ld + e] = order_key(__fadd_rn(zv[i][j], al[i]));
+      }
+    }
+  } else
   for (int r = warp; r < kSampleRows; r += kWarps) {
     const int64_t s = s0 + r;
     if (s >= S) break;
@@ -459,7 +488,8 @@ cudaError_t dispatch(const RouteParams& p, bool route, bool alpha_out, bool alph
 template <int Q>
 cudaError_t launch_sample_q(const float* z, const float* alpha, const float* bias, int64_t N,
                             int E, int K, int64_t S, int64_t stride, int64_t S_ld,
-                            uint32_t* sample, cudaStream_t s) {
+                            uint32_t* sample, cudaStream_t s, uint32_t* zero_word) {
+  static_assert(kSampleRows % kWarps == 0, "whole rows per warp");
   const size_t smem = ((4 * kSampleRows * (E + 1) + 15) & ~15) + ((4 * E + 15) & ~15) +
                       sizeof(RowScratch<Q>) * kWarps;
   dim3 grid(static_cast<unsigned>((S + kSampleRows - 1) / kSampleRows)), block(kThreads);
@@ -468,7 +498,8 @@ cudaError_t launch_sample_q(const float* z, const float* alpha, const float* bia
   cudaError_t err =
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  return launch_pdl(k, grid, block, smem, s, dim3(0, 0, 0), z, alpha, bias, N, E, K, S, stride, S_ld, sample);
+  return launch_pdl(k, grid, block, smem, s, dim3(0, 0, 0), z, alpha, bias, N, E, K, S, stride, S_ld, sample,
+                    zero_word);
 }
 
 }  // namespace
@@ -515,12 +546,12 @@ cudaError_t launch_select_fixup(const float* z, const float* bias, int64_t N, in
 
 cudaError_t launch_eqb_sample(const float* z, const float* alpha, const float* bias, int64_t N,
                               int32_t E, int32_t K, int64_t S, int64_t stride, int64_t S_ld,
-                              uint32_t* sample, cudaStream_t s) {
+                              uint32_t* sample, cudaStream_t s, uint32_t* zero_word) {
   switch ((E + 127) / 128) {
-    case 1: return launch_sample_q<1>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s);
-    case 2: return launch_sample_q<2>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s);
-    case 3: return launch_sample_q<3>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s);
-    case 4: return launch_sample_q<4>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s);
+    case 1: return launch_sample_q<1>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s, zero_word);
+    case 2: return launch_sample_q<2>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s, zero_word);
+    case 3: return launch_sample_q<3>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s, zero_word);
+    case 4: return launch_sample_q<4>(z, alpha, bias, N, E, K, S, stride, S_ld, sample, s, zero_word);
     default: return cudaErrorInvalidValue;
   }
 }
