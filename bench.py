@@ -81,12 +81,13 @@ def gemm_bytes(N, d, E):
 def launches_per_step(N, E, K, updates=1, split=False):
     """Kernels of ours per step: logits + selection 2 (the fused GEMM and the
     check for rows it left to the row kernel, or the small-batch logits and
-    the row kernel); EQB update 3 (N <= 16384: sample, exact select, bias)
-    or 6 (sample, bracket, bracketed pass, select, fallback check, bias), or
-    over a split batch 15 (sample, brackets, bracketed pass and its finish,
-    rank, four histogram + digit passes, key value, bias); permutation 1 or
-    3.  Each further update re-routes (1) first."""
-    eqb = 15 if split else (3 if N <= 16384 else 6)
+    the row kernel); EQB update 2 (N <= 16384: sample, exact select ending
+    in the bias update) or 4 (sample, bracket, bracketed pass, and one grid
+    for the select, any column fallback and the bias update), or over a
+    split batch 15 (sample, brackets, bracketed pass and its finish, rank,
+    four histogram + digit passes, key value, bias); permutation 1 or 3.
+    Each further update re-routes (1) first."""
+    eqb = 15 if split else (2 if N <= 16384 else 4)
     permute = 1 if N * K <= 4096 else 3
     return 2 + eqb + permute + (updates - 1) * (1 + eqb + permute)
 

@@ -26,9 +26,9 @@ def test_gemm_bytes():
 
 
 @pytest.mark.parametrize("N,K,want", [
-    (1 << 20, 6, 2 + 6 + 3),      # bracketed EQB chain, tiled permutation
-    (16384, 6, 2 + 3 + 3),        # the sample is the column
-    (256, 6, 2 + 3 + 1),          # one-block permutation (N K <= 4096)
+    (1 << 20, 6, 2 + 4 + 3),      # bracketed EQB chain, tiled permutation
+    (16384, 6, 2 + 2 + 3),        # the sample is the column
+    (256, 6, 2 + 2 + 1),          # one-block permutation (N K <= 4096)
 ])
 def test_launches_per_step(N, K, want):
     assert bench.launches_per_step(N, 384, K) == want
@@ -53,9 +53,9 @@ def test_algorithmic_work_of_the_collapsed_loop():
 
 
 def test_launches_of_the_collapsed_loop():
-    # forward 2, permutation 3, update 3 (the sample is the column), then nine
-    # times re-route 1 + update 3 + permutation 3
-    assert bench.launches_per_step(16384, 384, 6, updates=10) == 2 + 3 + 3 + 9 * 7
+    # forward 2, permutation 3, update 2 (the sample is the column), then nine
+    # times re-route 1 + update 2 + permutation 3
+    assert bench.launches_per_step(16384, 384, 6, updates=10) == 2 + 2 + 3 + 9 * 6
 
 
 @pytest.mark.parametrize("timed_s,reasons,kind", [
