@@ -419,6 +419,269 @@ __global__ void __launch_bounds__(kThreads) select_fixup_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Selection alone over large batches: eight lanes per row, four rows per warp.
+//
+// The same exact rule as warp_select_row (top K + 1 of B = Z + beta by order
+// key, ties to the lower expert id), laid out so that the warp-wide steps
+// serve four rows at once.  Lane s of a row's segment holds the C = E / 32
+// chunks c = 8 i + s (columns 32 i + 4 s .. + 3), loaded as float4.
+//  1. threshold: the lanes cut their chunks into GPL groups (24 or 32
+//     groups per row); K + 1 rounds of a segment-wide maximum over the lanes'
+//     sorted group maxima, each round removing the maximum from every lane
+//     that holds it.  After the last round at least K + 1 distinct elements
+//     (group maxima) are >= its value T, so T is at most the (K+1)-th
+//     largest score, and only a few scores per row reach it;
+//  2. candidates (scores >= T, a few per row) go to a 32-slot row buffer in
+//     shared memory, in any order, as 64-bit composites (order key, then
+//     511 - id) with their raw logit;
+//  3. each candidate's rank is the number of the row's candidates with a
+//     larger composite (a larger key, or the same key and a lower id); the
+//     candidates of rank 0..K are the K selected experts and alpha.
+// A row with more than 32 candidates (heavy ties), or fewer than K + 1
+// (non-finite values), is finished by the whole warp with warp_select_row.
+constexpr int kSegRows = 4;                   // rows per warp
+constexpr int kSegSlots = 32;                 // candidates per row
+
+template <int C>
+struct SegScratch {
+  float z[kSegRows][32 * C];                  // the rows' raw logits (lane-chunk order)
+  uint64_t comp[kSegRows][kSegSlots + 1];     // (key, 511 - id); one pad word pair per row
+  float zc[kSegRows][kSegSlots + 2];          // the candidates' raw logits
+  uint32_t win[kSegRows][24];                 // slot of rank r (r <= K)
+};
+
+// Groups per lane: 3 of four chunks at C = 12, else 4 (8 GPL >= 24 >= K + 1).
+template <int C>
+struct SegGroups {
+  static constexpr int kGPL = C == 12 ? 3 : 4;
+  static constexpr int kGS = C / kGPL;             // chunks per group
+  static_assert(C % kGPL == 0, "whole groups");
+};
+
+template <int C, bool kBias>
+__global__ void __launch_bounds__(kThreads) seg_select_kernel(
+    const float* __restrict__ z, const float* __restrict__ beta, int64_t N, int E, int K,
+    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int V = 4 * C;
+  float* beta_s = reinterpret_cast<float*>(smem);
+  SegScratch<C>& sc = reinterpret_cast<SegScratch<C>*>(smem + 4 * 32 * C)[threadIdx.x >> 5];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int seg = lane >> 3, sl = lane & 7;
+  pdl_wait();       // Z comes from the kernel before this one
+  pdl_trigger();
+  for (int e = threadIdx.x; e < E; e += kThreads) beta_s[e] = kBias ? beta[e] : 0.f;
+  __syncthreads();
+  const int64_t step = static_cast<int64_t>(gridDim.x) * kWarps * kSegRows;
+  for (int64_t base = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * kSegRows; base < N; base += step) {
+    const int64_t row = base + seg;
+    const bool live = row < N;
+    float zv[V];
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (live) v = __ldg(reinterpret_cast<const float4*>(z + row * E + 32 * i + 4 * sl));
+      zv[4 * i] = v.x;
+      zv[4 * i + 1] = v.y;
+      zv[4 * i + 2] = v.z;
+      zv[4 * i + 3] = v.w;
+    }
+    // scores, chunk maxima, group maxima
+    constexpr int GPL = SegGroups<C>::kGPL, GS = SegGroups<C>::kGS;
+    float cmax[C];
+    float g[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const float4 bq = *reinterpret_cast<const float4*>(&beta_s[32 * i + 4 * sl]);
+      const float b0 = kBias ? __fadd_rn(zv[4 * i], bq.x) : zv[4 * i];
+      const float b1 = kBias ? __fadd_rn(zv[4 * i + 1], bq.y) : zv[4 * i + 1];
+      const float b2 = kBias ? __fadd_rn(zv[4 * i + 2], bq.z) : zv[4 * i + 2];
+      const float b3 = kBias ? __fadd_rn(zv[4 * i + 3], bq.w) : zv[4 * i + 3];
+      const float m = fmaxf(fmaxf(b0, b1), fmaxf(b2, b3));
+      cmax[i] = m;
+      g[i / GS] = fmaxf(g[i / GS], m);
+    }
+    // this lane's group maxima sorted descending (GPL = 3 leaves g[3] at -inf)
+#define KOLIBRI_FCE(a, b)                    \
+  {                                          \
+    const float hi_ = fmaxf(g[a], g[b]);     \
+    g[b] = fminf(g[a], g[b]);                \
+    g[a] = hi_;                              \
+  }
+    KOLIBRI_FCE(0, 1) KOLIBRI_FCE(2, 3) KOLIBRI_FCE(0, 2) KOLIBRI_FCE(1, 3) KOLIBRI_FCE(1, 2)
+#undef KOLIBRI_FCE
+    (void)GPL;
+    float T = -INFINITY;
+    for (int r = 0; r <= K; ++r) {
+      float m = g[0];
+#pragma unroll
+      for (int d = 1; d < 8; d <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+      T = m;
+      if (g[0] == m) {            // every lane holding the maximum drops it
+        g[0] = g[1];
+        g[1] = g[2];
+        g[2] = g[3];
+        g[3] = -INFINITY;
+      }
+    }
+    // the row in shared memory (candidates are read back by chunk index)
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < C; ++i)
+      *reinterpret_cast<float4*>(&sc.z[seg][32 * i + 4 * sl]) =
+          make_float4(zv[4 * i], zv[4 * i + 1], zv[4 * i + 2], zv[4 * i + 3]);
+    uint32_t cm = 0u;   // chunks holding a candidate
+#pragma unroll
+    for (int i = 0; i < C; ++i) cm |= (cmax[i] >= T) ? (1u << i) : 0u;
+    // candidates per lane, then their positions in the row buffer
+    uint32_t cnt = 0u;
+    {
+      uint32_t mm = cm;
+      while (mm) {
+        const int i = __ffs(mm) - 1;
+        mm &= mm - 1u;
+        const float4 zq = *reinterpret_cast<const float4*>(&sc.z[seg][32 * i + 4 * sl]);
+        const float4 bq = *reinterpret_cast<const float4*>(&beta_s[32 * i + 4 * sl]);
+        cnt += (kBias ? __fadd_rn(zq.x, bq.x) : zq.x) >= T;
+        cnt += (kBias ? __fadd_rn(zq.y, bq.y) : zq.y) >= T;
+        cnt += (kBias ? __fadd_rn(zq.z, bq.z) : zq.z) >= T;
+        cnt += (kBias ? __fadd_rn(zq.w, bq.w) : zq.w) >= T;
+      }
+    }
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, d, 8);
+      if (sl >= d) incl += t;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 7, 8);
+    // the candidates as 64-bit composites (order key, then 511 - id), with
+    // their logits
+    if (total <= kSegSlots) {
+      uint32_t pos = incl - cnt;
+      while (cm) {
+        const int i = __ffs(cm) - 1;
+        cm &= cm - 1u;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int e = 32 * i + 4 * sl + u;
+          const float zz = sc.z[seg][e];
+          const float bb = kBias ? __fadd_rn(zz, beta_s[e]) : zz;
+          if (bb >= T) {
+            sc.comp[seg][pos] = (static_cast<uint64_t>(order_key(bb)) << 32) | (511u - static_cast<uint32_t>(e));
+            sc.zc[seg][pos] = zz;
+            ++pos;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    const bool fine = live && total >= static_cast<uint32_t>(K + 1) && total <= kSegSlots;
+    // rank of each candidate: how many of the row's candidates come first
+    // (larger key, or the same key and a lower id); ranks 0..K are the result
+    if (fine) {
+      uint64_t c[4];
+      uint32_t rk[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t slot = static_cast<uint32_t>(sl + 8 * q);
+        c[q] = slot < total ? sc.comp[seg][slot] : 0ull;
+        rk[q] = 0u;
+      }
+      for (uint32_t t = 0; t < total; ++t) {
+        const uint64_t o = sc.comp[seg][t];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) rk[q] += (o > c[q]) ? 1u : 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t slot = static_cast<uint32_t>(sl + 8 * q);
+        if (slot < total && rk[q] <= static_cast<uint32_t>(K)) sc.win[seg][rk[q]] = slot;
+      }
+    }
+    __syncwarp();
+    if (live && fine) {
+      {
+        // lane s writes ranks s, s + 8, s + 16
+        for (int r = sl; r <= K; r += 8) {
+          const uint32_t slot = sc.win[seg][r];
+          const uint64_t w = sc.comp[seg][slot];
+          if (r < K) {
+            ids[row * K + r] = static_cast<int32_t>(511u - static_cast<uint32_t>(w & 511u));
+            gates[row * K + r] = gate_sigmoid(sc.zc[seg][slot]);
+          } else if (alpha != nullptr) {
+            alpha[row] = -key_to_float(static_cast<uint32_t>(w >> 32));
+          }
+        }
+      }
+    }
+    __syncwarp();
+    // Rows left open (more than 32 candidates: heavy ties; or fewer than
+    // K + 1: non-finite values) take the exact warp-per-row selection of
+    // route.cuh, the whole warp on each, with the rows' buffer as scratch.
+    constexpr int Q = C / 4;
+    static_assert(sizeof(RowScratch<Q>) <= sizeof(sc.z), "the row scratch fits the rows' buffer");
+    unsigned open = __ballot_sync(0xffffffffu, sl == 0 && live && !fine);
+    while (open) {
+      const int sg = (__ffs(open) - 1) >> 3;
+      open &= open - 1u;
+      const int64_t rr = base + sg;
+      float zr[4 * Q];
+      load_row<Q, true>(z + rr * E, E, lane, zr);
+      RowScratch<Q>& rs = *reinterpret_cast<RowScratch<Q>*>(&sc.z[0][0]);
+      int rank;
+      uint32_t key, id;
+      warp_select_row<Q, true, kBias>(zr, beta_s, 0xffffffffu, K, lane, rs, rank, key, id);
+      if (rank >= 0 && rank < K) {
+        const uint32_t e = id < static_cast<uint32_t>(E) ? id : 0u;
+        ids[rr * K + rank] = static_cast<int32_t>(id);
+        gates[rr * K + rank] = gate_sigmoid(rs.row[buffer_pos<Q>(e)]);
+      }
+      if (rank == K && alpha != nullptr) alpha[rr] = -key_to_float(key);
+      __syncwarp();
+    }
+  }
+}
+
+template <int C>
+cudaError_t launch_seg(const float* z, const float* bias, int64_t N, int E, int K, int32_t* ids,
+                       float* gates, float* alpha, cudaStream_t s) {
+  auto kern = bias ? seg_select_kernel<C, true> : seg_select_kernel<C, false>;
+  const size_t smem = 4 * 32 * C + sizeof(SegScratch<C>) * kWarps;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (err != cudaSuccess) return err;
+  if (per_sm < 1) per_sm = 1;
+  const int64_t rows_per_block = static_cast<int64_t>(kWarps) * kSegRows;
+  int64_t blocks = (N + rows_per_block - 1) / rows_per_block;
+  const int64_t resident = static_cast<int64_t>(device_sm_count()) * per_sm;
+  if (blocks > resident) blocks = resident;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), smem, s, dim3(0, 0, 0), z, bias,
+                    N, E, K, ids, gates, alpha);
+}
+
+// Batches at least this large take the segment kernel; decode-sized ones
+// keep the warp-per-row kernel.
+constexpr int64_t kSegMinRows = 4096;
+
+bool seg_select_applies(int64_t N, int E, int K) {
+  return N >= kSegMinRows && (E == 128 || E == 256 || E == 384 || E == 512) && K + 1 <= 24;
+}
+
+cudaError_t launch_seg_select(const float* z, const float* bias, int64_t N, int E, int K, int32_t* ids,
+                              float* gates, float* alpha, cudaStream_t s) {
+  switch (E / 32) {
+    case 4: return launch_seg<4>(z, bias, N, E, K, ids, gates, alpha, s);
+    case 8: return launch_seg<8>(z, bias, N, E, K, ids, gates, alpha, s);
+    case 12: return launch_seg<12>(z, bias, N, E, K, ids, gates, alpha, s);
+    case 16: return launch_seg<16>(z, bias, N, E, K, ids, gates, alpha, s);
+    default: return cudaErrorNotSupported;
+  }
+}
+
 template <int Q, bool kFull, bool kBias, bool kRoute, bool kAlphaOut, bool kAlphaIn, bool kWindow>
 cudaError_t launch_rows(RouteParams p, cudaStream_t s) {
   auto kern = route_rows_kernel<Q, kFull, kBias, kRoute, kAlphaOut, kAlphaIn, kWindow>;
@@ -506,6 +769,7 @@ cudaError_t launch_sample_q(const float* z, const float* alpha, const float* bia
 
 cudaError_t launch_topk(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
                         int32_t* ids, float* gates, float* alpha, cudaStream_t s) {
+  if (seg_select_applies(N, E, K)) return launch_seg_select(z, bias, N, E, K, ids, gates, alpha, s);
   RouteParams p{};
   p.z = z;
   p.beta = bias;
@@ -538,7 +802,8 @@ cudaError_t launch_select_fixup(const float* z, const float* bias, int64_t N, in
     case 1: KOLIBRI_FIXUP(1) break;
     case 2: KOLIBRI_FIXUP(2) break;
     case 3: KOLIBRI_FIXUP(3) break;
-    default: return cudaErrorInvalidValue;   // the fused kernel covers E <= 384
+    case 4: KOLIBRI_FIXUP(4) break;
+    default: return cudaErrorInvalidValue;
   }
 #undef KOLIBRI_FIXUP
   return cudaGetLastError();

@@ -114,6 +114,27 @@ def test_select_extreme_values(oracle_mod):
     _select_case(oracle_mod, z, workloads.random_logits(1, E, 5)[0], K)
 
 
+@pytest.mark.parametrize("N,E,K", [(16384, 384, 6), (16411, 128, 8), (16400, 256, 1),
+                                   (16390, 512, 16), (20001, 384, 15), (16384, 128, 7)])
+def test_select_large_batch(oracle_mod, N, E, K):
+    # From 16384 rows the selection runs eight lanes per row (E in 128, 256,
+    # 384, 512); rows with heavy ties (more than 32 scores at or above its
+    # threshold) are left to the row kernel through a NaN alpha.  Mixed in:
+    # tied rows, all-equal rows, signed zeros, large and subnormal logits.
+    z = workloads.random_logits(N, E, seed=N + E + K) * np.float32(4.0)
+    t = workloads.tied_logits(N, E, seed=K)
+    z[::97] = t[::97]
+    z[5::211] = np.float32(0.0)
+    z[7::389, ::3] = np.float32(-0.0)
+    z[11::401, :10] = np.float32(900.0)
+    z[13::409] = np.float32(1e-40)
+    z[17::419] = np.float32(-800.0)
+    beta = workloads.random_logits(1, E, seed=8)[0] * np.float32(0.3)
+    _select_case(oracle_mod, z, beta, K)
+    _select_case(oracle_mod, z, None, K)
+    check_status()
+
+
 def test_gates_unchanged_by_bias():
     z = workloads.random_logits(500, 384, seed=21)
     i1, g1, _ = gpu_select(z, workloads.random_logits(1, 384, 22)[0], 6)
