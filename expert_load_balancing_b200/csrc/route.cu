@@ -460,7 +460,7 @@ struct SegGroups {
 };
 
 template <int C, bool kBias>
-__global__ void __launch_bounds__(kThreads) seg_select_kernel(
+__global__ void __launch_bounds__(kThreads, C >= 16 ? 2 : 3) seg_select_kernel(
     const float* __restrict__ z, const float* __restrict__ beta, int64_t N, int E, int K,
     int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -486,6 +486,15 @@ __global__ void __launch_bounds__(kThreads) seg_select_kernel(
       zv[4 * i + 1] = v.y;
       zv[4 * i + 2] = v.z;
       zv[4 * i + 3] = v.w;
+    }
+    {
+      // the warp's next rows go to L2 while these are worked on: the row's
+      // 128-byte lines split over the segment's lanes
+      const int64_t nrow = row + step;
+      if (nrow < N) {
+        const char* pr = reinterpret_cast<const char*>(z + nrow * E);
+        for (int ln = sl; ln < E / 32; ln += 8) asm volatile("prefetch.global.L2 [%0];" ::"l"(pr + 128 * ln));
+      }
     }
     // scores, chunk maxima, group maxima
     constexpr int GPL = SegGroups<C>::kGPL, GS = SegGroups<C>::kGS;
