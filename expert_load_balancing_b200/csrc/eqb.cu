@@ -91,12 +91,16 @@ __device__ __forceinline__ void block_minmax(uint32_t& mn, uint32_t& mx, SelectS
 // digit of the keys that match the prefix, then a block-wide scan of the
 // bins from the top (largest keys first) finds the bin holding the rank.
 // Every thread of the block (kSelThreads) must call it; out[] is returned
-// to all of them.
+// to all of them.  With max_passes, it stops after that many digits: out[i]
+// then holds the resolved high bits with zeros below, and *unresolved the
+// number of low bits left open (the rank's key lies in [out, out | 2^u - 1]).
 template <int R, class KeyAt>
 __device__ void block_select_ranks(KeyAt key_at, int64_t n, const int64_t (&rank)[R],
-                                   uint32_t mn, uint32_t mx, uint32_t (&out)[R], SelectSmem& sm) {
+                                   uint32_t mn, uint32_t mx, uint32_t (&out)[R], SelectSmem& sm,
+                                   int max_passes = 1 << 30, int* unresolved = nullptr) {
   using D = Digits<R>;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (unresolved != nullptr) *unresolved = 0;
   if (mn == mx) {
 #pragma unroll
     for (int i = 0; i < R; ++i) out[i] = mn;
@@ -110,7 +114,7 @@ __device__ void block_select_ranks(KeyAt key_at, int64_t n, const int64_t (&rank
     prefix[i] = (bits_left == 32) ? 0u : (mx & ~((1u << bits_left) - 1u));
     r[i] = rank[i];
   }
-  while (bits_left > 0) {
+  for (int pass = 0; bits_left > 0 && pass < max_passes; ++pass) {
     const int nb = bits_left < D::kBits ? bits_left : D::kBits;
     const int shift = bits_left - nb;
     const int nbins = 1 << nb;
@@ -190,6 +194,7 @@ __device__ void block_select_ranks(KeyAt key_at, int64_t n, const int64_t (&rank
   }
 #pragma unroll
   for (int i = 0; i < R; ++i) out[i] = prefix[i];
+  if (unresolved != nullptr) *unresolved = bits_left;
 }
 
 // Keys of one expert staged in shared memory when they fit (kSmemKeys),
@@ -291,13 +296,24 @@ __global__ void __launch_bounds__(kSelThreads) sample_select_kernel(
     // ticket given: this grid also ends the update (bias from all v)
     if (ticket != nullptr) bias_by_last_block(v, static_cast<int>(gridDim.x), ticket, bias, quantiles, sm);
   } else {
-    // both bracket ranks in the same passes (r_hi <= r_lo)
+    // both bracket ranks in the same passes (r_hi <= r_lo), two digits deep:
+    // the bracket only has to contain the two sample keys, so it takes the
+    // outer edges of their bins (at 20 resolved bits a bin holds a few keys
+    // of the column near the target; the counts decide exactness)
     const int64_t rk[2] = {r_hi, r_lo};
     uint32_t k[2];
-    block_select_ranks<2>(at, S, rk, mn, mx, k, sm);
+    int open_bits = 0;
+    block_select_ranks<2>(at, S, rk, mn, mx, k, sm, 2, &open_bits);
     if (threadIdx.x == 0) {
-      hi[e] = k[0];
-      lo[e] = k[1];
+      // widened bounds stay within [key(-inf), key(+inf)] when the keys were,
+      // so the pass may compare them as floats
+      constexpr uint32_t kKeyNegInf = 0x007fffffu, kKeyPosInf = 0xff800000u;
+      const uint32_t low = open_bits >= 32 ? 0xffffffffu : ((1u << open_bits) - 1u);
+      uint32_t h = k[0] | low, l = k[1];
+      if (k[0] <= kKeyPosInf && h > kKeyPosInf) h = kKeyPosInf;
+      if (l < kKeyNegInf && (k[1] | low) >= kKeyNegInf) l = kKeyNegInf;
+      hi[e] = h;
+      lo[e] = l;
     }
   }
 }
