@@ -633,6 +633,8 @@ PARTS = {
                    lambda E, K: 12 * E, "Z and dS read, dZ written"),
     "intervention": ("intervention rate (own top-K vs routed ids)",
                      lambda E, K: 4 * E + 4 * K, "Z and ids read"),
+    "topk": ("selection alone: bias add, top-K ids, sigmoid gates, alpha (kolibri_router_topk)",
+             lambda E, K: 4 * E + 8 * K + 4, "Z read; ids, gates and alpha written"),
 }
 
 
@@ -645,6 +647,9 @@ def run_part(args):
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens:
+        import dataclasses
+        wl = dataclasses.replace(wl, N=args.tokens)
     N, d, E, K = wl.N, wl.d, wl.E, wl.K
     step = RouterStep(wl, device)
     stream = torch.cuda.Stream(device)
@@ -656,6 +661,9 @@ def run_part(args):
     gs = torch.randn((N, E), generator=g, device=device) * 1e-4 if args.part in ("lei", "score_grad") else None
     gz = torch.empty_like(gs) if gs is not None else None
     ws16 = B.workspace(B.KOLIBRI_OP_EQB_BF16, N, E, K, device)
+    ids_t = torch.empty((N, K), dtype=torch.int32, device=device) if args.part == "topk" else None
+    gates_t = torch.empty((N, K), dtype=torch.float32, device=device) if args.part == "topk" else None
+    alpha_t = torch.empty((N,), dtype=torch.float32, device=device) if args.part == "topk" else None
     beta0 = step.beta.clone()
     q = torch.empty((E,), dtype=torch.float32, device=device)
 
@@ -675,6 +683,8 @@ def run_part(args):
             B.kolibri_lei_inject(step.counts, gs, K, stream=stream)
         elif args.part == "score_grad":
             B.kolibri_score_grad_to_logits(step.z, gs, gz, stream=stream)
+        elif args.part == "topk":
+            B.kolibri_router_topk(step.z, step.beta, K, ids_t, gates_t, alpha_t, stream=stream)
         else:
             B.kolibri_intervention_rate(step.z, step.ids, stream=stream)
 
@@ -713,6 +723,8 @@ def run_part(args):
         oracle.lei_inject(step.counts.cpu().numpy(), gs[:n].cpu().numpy(), K)
     elif args.part == "score_grad":
         oracle.score_grad_to_logits(zh, gs[:n].cpu().numpy())
+    elif args.part == "topk":
+        oracle.select(zh, step.beta.cpu().numpy(), K)
     else:
         ids_u, _, _ = oracle.select(zh, None, K)
         oracle.intervention_rate(step.ids[:n].cpu().numpy(), ids_u)
@@ -728,13 +740,15 @@ def run_part(args):
             oracle.lei_inject(step.counts.cpu().numpy(), gs[:n].cpu().numpy(), K)
         elif args.part == "score_grad":
             oracle.score_grad_to_logits(zh, gs[:n].cpu().numpy())
+        elif args.part == "topk":
+            oracle.select(zh, step.beta.cpu().numpy(), K)
         else:
             ids_u, _, _ = oracle.select(zh, None, K)
             oracle.intervention_rate(step.ids[:n].cpu().numpy(), ids_u)
         cpu_s += time.time() - t
         reps += 1
     return {
-        "metric": f"{what}: tokens/s at N=1M, E=384, K=6", "part": args.part,
+        "metric": f"{what}: tokens/s at N={N}, E={E}, K={K}", "part": args.part,
         "value": N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "fp32/f64",
         "data": "synthetic",
