@@ -574,6 +574,11 @@ cudaError_t launch_intervention(const float* z, const int32_t* ids, int64_t N, i
                                 unsigned long long* total, double* rate, cudaStream_t s) {
   cudaError_t err = cudaMemsetAsync(total, 0, sizeof(unsigned long long), s);
   if (err != cudaSuccess) return err;
+  if (seg_overlap_applies(N, E, K)) {
+    if ((err = launch_seg_overlap(z, ids, N, E, K, total, s)) != cudaSuccess) return err;
+    intervention_finish_kernel<<<1, 1, 0, s>>>(total, N, K, rate);
+    return cudaGetLastError();
+  }
   const bool full = (E % 128) == 0;
   const unsigned grid = static_cast<unsigned>(grid_for((N + 7) / 8, 1));
 #define KOLIBRI_OVL(Q)                                                              \

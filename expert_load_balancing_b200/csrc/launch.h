@@ -81,6 +81,12 @@ cudaError_t launch_router_forward(const void* x, const void* w, const float* bia
 cudaError_t launch_select_fixup(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
                                 int32_t* ids, float* gates, float* alpha, cudaStream_t s);
 
+// The intervention rate's overlap count in the selection's eight-lanes-per-
+// row layout (from 4096 rows, E in 128, 256, 384, 512): adds to *total the
+// number of (row, k) whose own top-K expert on Z alone is among ids[row].
+bool seg_overlap_applies(int64_t N, int32_t E, int32_t K);
+cudaError_t launch_seg_overlap(const float* z, const int32_t* ids, int64_t N, int32_t E, int32_t K,
+                               unsigned long long* total, cudaStream_t s);
 cudaError_t launch_topk(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
                         int32_t* ids, float* gates, float* alpha, cudaStream_t s);
 

@@ -459,10 +459,15 @@ struct SegGroups {
   static_assert(C % kGPL == 0, "whole groups");
 };
 
-template <int C, bool kBias>
+// kOverlap: instead of writing the selection, count how many of each row's
+// K experts (selected on Z alone) are among the K ids given for the row, and
+// add the count over all rows to *overlap (the intervention rate's
+// numerator).
+template <int C, bool kBias, bool kOverlap>
 __global__ void __launch_bounds__(kThreads, C >= 16 ? 2 : 3) seg_select_kernel(
     const float* __restrict__ z, const float* __restrict__ beta, int64_t N, int E, int K,
-    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha) {
+    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha,
+    unsigned long long* __restrict__ overlap) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int V = 4 * C;
   float* beta_s = reinterpret_cast<float*>(smem);
@@ -473,6 +478,13 @@ __global__ void __launch_bounds__(kThreads, C >= 16 ? 2 : 3) seg_select_kernel(
   pdl_trigger();
   for (int e = threadIdx.x; e < E; e += kThreads) beta_s[e] = kBias ? beta[e] : 0.f;
   __syncthreads();
+  // kOverlap: is expert e among row t's given ids
+  auto routed = [&](int64_t t, uint32_t e) {
+    bool hit = false;
+    for (int k = 0; k < K; ++k) hit |= __ldg(ids + t * K + k) == static_cast<int32_t>(e);
+    return hit;
+  };
+  uint32_t hits = 0u;
   const int64_t step = static_cast<int64_t>(gridDim.x) * kWarps * kSegRows;
   for (int64_t base = (static_cast<int64_t>(blockIdx.x) * kWarps + warp) * kSegRows; base < N; base += step) {
     const int64_t row = base + seg;
@@ -616,8 +628,11 @@ __global__ void __launch_bounds__(kThreads, C >= 16 ? 2 : 3) seg_select_kernel(
         for (int r = sl; r <= K; r += 8) {
           const uint32_t slot = sc.win[seg][r];
           const uint64_t w = sc.comp[seg][slot];
-          if (r < K) {
-            ids[row * K + r] = static_cast<int32_t>(511u - static_cast<uint32_t>(w & 511u));
+          const uint32_t id = 511u - static_cast<uint32_t>(w & 511u);
+          if constexpr (kOverlap) {
+            if (r < K) hits += routed(row, id) ? 1u : 0u;
+          } else if (r < K) {
+            ids[row * K + r] = static_cast<int32_t>(id);
             gates[row * K + r] = gate_sigmoid(sc.zc[seg][slot]);
           } else if (alpha != nullptr) {
             alpha[row] = -key_to_float(static_cast<uint32_t>(w >> 32));
@@ -642,21 +657,30 @@ __global__ void __launch_bounds__(kThreads, C >= 16 ? 2 : 3) seg_select_kernel(
       int rank;
       uint32_t key, id;
       warp_select_row<Q, true, kBias>(zr, beta_s, 0xffffffffu, K, lane, rs, rank, key, id);
-      if (rank >= 0 && rank < K) {
-        const uint32_t e = id < static_cast<uint32_t>(E) ? id : 0u;
-        ids[rr * K + rank] = static_cast<int32_t>(id);
-        gates[rr * K + rank] = gate_sigmoid(rs.row[buffer_pos<Q>(e)]);
+      if constexpr (kOverlap) {
+        if (rank >= 0 && rank < K) hits += routed(rr, id) ? 1u : 0u;
+      } else {
+        if (rank >= 0 && rank < K) {
+          const uint32_t e = id < static_cast<uint32_t>(E) ? id : 0u;
+          ids[rr * K + rank] = static_cast<int32_t>(id);
+          gates[rr * K + rank] = gate_sigmoid(rs.row[buffer_pos<Q>(e)]);
+        }
+        if (rank == K && alpha != nullptr) alpha[rr] = -key_to_float(key);
       }
-      if (rank == K && alpha != nullptr) alpha[rr] = -key_to_float(key);
       __syncwarp();
     }
+  }
+  if constexpr (kOverlap) {
+    const uint32_t sum = __reduce_add_sync(0xffffffffu, hits);
+    if (lane == 0 && sum != 0u) atomicAdd(overlap, static_cast<unsigned long long>(sum));
   }
 }
 
 template <int C>
 cudaError_t launch_seg(const float* z, const float* bias, int64_t N, int E, int K, int32_t* ids,
-                       float* gates, float* alpha, cudaStream_t s) {
-  auto kern = bias ? seg_select_kernel<C, true> : seg_select_kernel<C, false>;
+                       float* gates, float* alpha, cudaStream_t s, unsigned long long* overlap = nullptr) {
+  auto kern = overlap ? seg_select_kernel<C, false, true>
+                      : (bias ? seg_select_kernel<C, true, false> : seg_select_kernel<C, false, false>);
   const size_t smem = 4 * 32 * C + sizeof(SegScratch<C>) * kWarps;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (err != cudaSuccess) return err;
@@ -669,7 +693,7 @@ cudaError_t launch_seg(const float* z, const float* bias, int64_t N, int E, int 
   const int64_t resident = static_cast<int64_t>(device_sm_count()) * per_sm;
   if (blocks > resident) blocks = resident;
   return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), smem, s, dim3(0, 0, 0), z, bias,
-                    N, E, K, ids, gates, alpha);
+                    N, E, K, ids, gates, alpha, overlap);
 }
 
 // Batches at least this large take the segment kernel; decode-sized ones
@@ -775,6 +799,20 @@ cudaError_t launch_sample_q(const float* z, const float* alpha, const float* bia
 }
 
 }  // namespace
+
+bool seg_overlap_applies(int64_t N, int32_t E, int32_t K) { return seg_select_applies(N, E, K); }
+
+cudaError_t launch_seg_overlap(const float* z, const int32_t* ids, int64_t N, int32_t E, int32_t K,
+                               unsigned long long* total, cudaStream_t s) {
+  int32_t* idv = const_cast<int32_t*>(ids);   // read only in this mode
+  switch (E / 32) {
+    case 4: return launch_seg<4>(z, nullptr, N, E, K, idv, nullptr, nullptr, s, total);
+    case 8: return launch_seg<8>(z, nullptr, N, E, K, idv, nullptr, nullptr, s, total);
+    case 12: return launch_seg<12>(z, nullptr, N, E, K, idv, nullptr, nullptr, s, total);
+    case 16: return launch_seg<16>(z, nullptr, N, E, K, idv, nullptr, nullptr, s, total);
+    default: return cudaErrorNotSupported;
+  }
+}
 
 cudaError_t launch_topk(const float* z, const float* bias, int64_t N, int32_t E, int32_t K,
                         int32_t* ids, float* gates, float* alpha, cudaStream_t s) {

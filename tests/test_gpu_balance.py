@@ -144,6 +144,20 @@ def test_score_grad_to_logits_matches_oracle(oracle_mod):
     assert abs(float(host(one)[0]) - 0.105) < 5e-4                    # section 8
 
 
+def test_intervention_rate_ties_large(oracle_mod):
+    # from 4096 rows the overlap runs eight lanes per row; rows with heavy
+    # ties are finished by the whole warp in the same kernel
+    N, E, K = 6000, 256, 4
+    z = workloads.random_logits(N, E, seed=41)
+    z[::3] = workloads.tied_logits(N, E, seed=42)[::3]
+    ids_routed, _, _ = oracle_mod.select(z, workloads.random_logits(1, E, seed=43)[0], K)
+    ids_unb, _, _ = oracle_mod.select(z, None, K)
+    rate, ovl = B.kolibri_intervention_rate(dev(z), dev(ids_routed))
+    torch.cuda.synchronize()
+    check_status()
+    assert int(host(ovl)[0]) == oracle_mod.intervention_overlap(ids_routed, ids_unb)
+
+
 @pytest.mark.parametrize("N,E,K", [(1, 4, 2), (5000, 384, 6), (4099, 128, 8), (777, 400, 6)])
 def test_intervention_rate_matches_oracle(oracle_mod, N, E, K):
     wl = workloads.Workload("t", N, 64, E, K, beta="normal0.1")
