@@ -509,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, C >= 16 ? 2 : 3) seg_select_kernel(
       }
     }
     // scores, chunk maxima, group maxima
-    constexpr int GPL = SegGroups<C>::kGPL, GS = SegGroups<C>::kGS;
+    constexpr int GS = SegGroups<C>::kGS;       // chunks per group
     float cmax[C];
     float g[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -532,7 +532,6 @@ __global__ void __launch_bounds__(kThreads, C >= 16 ? 2 : 3) seg_select_kernel(
   }
     KOLIBRI_FCE(0, 1) KOLIBRI_FCE(2, 3) KOLIBRI_FCE(0, 2) KOLIBRI_FCE(1, 3) KOLIBRI_FCE(1, 2)
 #undef KOLIBRI_FCE
-    (void)GPL;
     float T = -INFINITY;
     for (int r = 0; r <= K; ++r) {
       float m = g[0];
