@@ -374,21 +374,38 @@ __global__ void __launch_bounds__(kLeiThreads) lei_inject_kernel(
 // dZ = dS * sigma(Z) (1 - sigma(Z)): sigma in fp64 from the gate's exp
 // (saturating outside |z| <= 700 as the gate does), the product in fp64,
 // rounded once to fp32.
+__device__ __forceinline__ float score_grad_one(float zi, float gi) {
+  double s;
+  if (zi > 700.0f) {
+    s = 1.0;
+  } else if (zi < -700.0f) {
+    s = 0.0;
+  } else {
+    s = __ddiv_rn(1.0, __dadd_rn(1.0, gate_exp(-static_cast<double>(zi))));
+  }
+  return __double2float_rn(__dmul_rn(static_cast<double>(gi), __dmul_rn(s, __dsub_rn(1.0, s))));
+}
+
 __global__ void __launch_bounds__(kLeiThreads) score_grad_kernel(
     const float* __restrict__ z, const float* __restrict__ gs, int64_t n, float* __restrict__ gz) {
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kLeiThreads + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * kLeiThreads)
+    gz[i] = score_grad_one(z[i], gs[i]);
+}
+
+// Four consecutive elements per thread (16-byte aligned arrays): the same
+// arithmetic per element, four independent fp64 chains to interleave.
+__global__ void __launch_bounds__(kLeiThreads) score_grad_vec_kernel(
+    const float4* __restrict__ z, const float4* __restrict__ gs, int64_t n4, float4* __restrict__ gz,
+    const float* __restrict__ z_tail, const float* __restrict__ gs_tail, int tail, float* __restrict__ gz_tail) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kLeiThreads + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * kLeiThreads) {
-    const float zi = z[i];
-    double s;
-    if (zi > 700.0f) {
-      s = 1.0;
-    } else if (zi < -700.0f) {
-      s = 0.0;
-    } else {
-      s = __ddiv_rn(1.0, __dadd_rn(1.0, gate_exp(-static_cast<double>(zi))));
-    }
-    gz[i] = __double2float_rn(__dmul_rn(static_cast<double>(gs[i]), __dmul_rn(s, __dsub_rn(1.0, s))));
+    const float4 zq = __ldg(z + i), gq = __ldg(gs + i);
+    gz[i] = make_float4(score_grad_one(zq.x, gq.x), score_grad_one(zq.y, gq.y), score_grad_one(zq.z, gq.z),
+                        score_grad_one(zq.w, gq.w));
   }
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < tail)
+    gz_tail[threadIdx.x] = score_grad_one(z_tail[threadIdx.x], gs_tail[threadIdx.x]);
 }
 
 // Overlap of the router's own top-K (no bias) with the routed ids, summed
@@ -566,6 +583,16 @@ cudaError_t launch_lei_inject(const int32_t* counts, int64_t N, int32_t E, int32
 }
 
 cudaError_t launch_score_grad(const float* z, const float* gs, int64_t n, float* gz, cudaStream_t s) {
+  const bool vec = ((reinterpret_cast<uintptr_t>(z) | reinterpret_cast<uintptr_t>(gs) |
+                     reinterpret_cast<uintptr_t>(gz)) & 15u) == 0u;
+  if (vec && n >= 4) {
+    const int64_t n4 = n / 4;
+    const int tail = static_cast<int>(n - 4 * n4);
+    score_grad_vec_kernel<<<grid_for(n4, kLeiThreads), kLeiThreads, 0, s>>>(
+        reinterpret_cast<const float4*>(z), reinterpret_cast<const float4*>(gs), n4, reinterpret_cast<float4*>(gz),
+        z + 4 * n4, gs + 4 * n4, tail, gz + 4 * n4);
+    return cudaGetLastError();
+  }
   score_grad_kernel<<<grid_for(n, kLeiThreads), kLeiThreads, 0, s>>>(z, gs, n, gz);
   return cudaGetLastError();
 }

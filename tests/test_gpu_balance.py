@@ -140,6 +140,10 @@ def test_score_grad_to_logits_matches_oracle(oracle_mod):
     gz = B.kolibri_score_grad_to_logits(dev(z), dev(gs))
     torch.cuda.synchronize()
     assert_bit_equal(host(gz), oracle_mod.score_grad_to_logits(z, gs), "gz")
+    # views one element in: not 16-byte aligned, so the one-element-per-thread form runs
+    gz1 = B.kolibri_score_grad_to_logits(dev(z)[1:], dev(gs)[1:])
+    torch.cuda.synchronize()
+    assert_bit_equal(host(gz1), oracle_mod.score_grad_to_logits(z[1:], gs[1:]), "gz misaligned")
     one = B.kolibri_score_grad_to_logits(dev(np.array([2.0], np.float32)), dev(np.array([1.0], np.float32)))
     assert abs(float(host(one)[0]) - 0.105) < 5e-4                    # section 8
 
