@@ -134,9 +134,12 @@ def kolibri_workspace_bytes(op: int, N: int, E: int, K: int) -> int:
 
 
 def workspace(op: int, N: int, E: int, K: int, device=None) -> torch.Tensor:
-    """A device buffer large enough for ``op`` (uint8, 256-byte aligned)."""
+    """A zero-filled device buffer large enough for ``op`` (uint8, 256-byte
+    aligned).  Zero-filled because the decode form of
+    kolibri_router_forward_permute keeps a counter in it that must start at
+    zero; the calls leave it zero, so the buffer can be reused."""
     n = max(kolibri_workspace_bytes(op, N, E, K), 1)
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
 def kolibri_router_logits(x: torch.Tensor, w: torch.Tensor, z: torch.Tensor | None = None,

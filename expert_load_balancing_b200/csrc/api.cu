@@ -115,6 +115,12 @@ kolibri_status kolibri_router_forward_permute(const void* x, const void* w, cons
     if (ws_bytes < L.total) return KOLIBRI_ERR_WORKSPACE_TOO_SMALL;
   }
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ws && aligned16(ws) && ws_bytes >= L.total && router_decode_ticket_supported(N, d, E, K)) {
+    uint32_t* ticket = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + L.off_dec_ticket);
+    const cudaError_t err = launch_router_decode_ticket(x, w, bias, z, N, d, E, K, ids, gates, alpha, counts,
+                                                        offsets, perm, inv, ticket, s);
+    if (err != cudaErrorNotSupported) return from_cuda(err);
+  }
   if (router_decode_permutes(N, d, E, K)) {
     const cudaError_t err = launch_router_decode_permute(x, w, bias, z, N, d, E, K, ids, gates, alpha,
                                                          counts, offsets, perm, inv, s);

@@ -36,6 +36,7 @@ struct PermuteLayout {
   size_t off_chunk_counts = 0;  // u32 [E][nchunks]
   size_t off_counts = 0;        // u32 [E]
   size_t off_ticket = 0;        // u32 [1]
+  size_t off_dec_ticket = 0;    // u32 [1]: the decode forward's counter, zero between calls
   size_t total = 0;
 };
 PermuteLayout permute_layout(int64_t N, int32_t E, int32_t K);
@@ -118,6 +119,13 @@ cudaError_t launch_router_decode_permute(const void* x, const void* w, const flo
                                          float* gates, float* alpha, int32_t* counts,
                                          int64_t* offsets, int32_t* perm, int32_t* inv,
                                          cudaStream_t s);
+// The same outputs from E/8 CTAs without a cluster, the last of which (by the
+// counter `ticket`, zero on entry and left zero) selects and groups.
+bool router_decode_ticket_supported(int64_t N, int32_t d, int32_t E, int32_t K);
+cudaError_t launch_router_decode_ticket(const void* x, const void* w, const float* bias, float* z,
+                                        int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                        float* gates, float* alpha, int32_t* counts, int64_t* offsets,
+                                        int32_t* perm, int32_t* inv, uint32_t* ticket, cudaStream_t s);
 
 // The logits by batch size, with the same choice of kernel as the forward.
 cudaError_t launch_router_logits_by_size(const void* x, const void* w, float* z, int64_t N,

@@ -400,6 +400,8 @@ PermuteLayout permute_layout(int64_t N, int32_t E, int32_t K) {
   off += align256(sizeof(uint32_t) * static_cast<size_t>(E));
   L.off_ticket = off;
   off += align256(sizeof(uint32_t));
+  L.off_dec_ticket = off;
+  off += align256(sizeof(uint32_t));
   L.total = off;
   return L;
 }

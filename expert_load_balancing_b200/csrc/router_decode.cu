@@ -128,6 +128,73 @@ __device__ __forceinline__ void bulk_row(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// Counts, offsets and the stable grouping of a decode batch's nk slots
+// (experts ascending, slot index j = t K + k ascending inside an expert),
+// exactly as kolibri_expert_permute.  pid: every slot's expert (shared),
+// pre-filled with kNoId so that a slot the selection did not fill (a row
+// with NaN scores) is counted under expert 0 and reported, never used as an
+// index; cnt: E words, start: 512 words followed by one word per warp
+// (shared).  Called by all kThreads threads of the block; E <= 512.
+template <int kThreads>
+__device__ void group_slots(const uint32_t* pid, int nk, int E, uint32_t* cnt, uint32_t* start,
+                            const DecPerm& pm) {
+  constexpr int kPer = 512 / kThreads;   // experts per thread in the scan
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* wsum = start + 512;
+  for (int e = tid; e < E; e += kThreads) cnt[e] = 0u;
+  __syncthreads();
+  for (int j = tid; j < nk; j += kThreads) {
+    uint32_t e = pid[j];
+    if (e >= static_cast<uint32_t>(E)) {
+      raise_status(kStatusBadInput);
+      e = 0u;
+    }
+    atomicAdd(&cnt[e], 1u);
+  }
+  __syncthreads();
+  uint32_t v[kPer], sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = kPer * tid + i;
+    v[i] = e < E ? cnt[e] : 0u;
+    sum += v[i];
+  }
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  uint32_t run = incl - sum;
+  for (int w2 = 0; w2 < warp; ++w2) run += wsum[w2];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = kPer * tid + i;
+    if (e < E) {
+      start[e] = run;
+      pm.counts[e] = static_cast<int32_t>(v[i]);
+      pm.offsets[e] = run;
+    }
+    run += v[i];
+  }
+  if (tid == 0) pm.offsets[E] = nk;
+  __syncthreads();
+  const auto expert_of = [&](int j) {
+    const uint32_t e = pid[j];
+    return e < static_cast<uint32_t>(E) ? e : 0u;
+  };
+  for (int j = tid; j < nk; j += kThreads) {
+    const uint32_t e = expert_of(j);
+    uint32_t before = 0;                 // earlier slots of the same expert
+    for (int i = 0; i < j; ++i) before += (expert_of(i) == e) ? 1u : 0u;
+    const uint32_t pos = start[e] + before;
+    pm.perm[pos] = j;
+    if (pm.inv) pm.inv[j] = static_cast<int32_t>(pos);
+  }
+}
+
 template <int Q, bool kBias>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_forward_kernel(
     const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
@@ -152,6 +219,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_forward_kernel(
     mbar_init(bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (rank == 0)                         // the slot list of the grouping (CTA 0), see group_slots
+    for (int j = tid; j < kDecTok * 16; j += kDecThreads) reinterpret_cast<uint32_t*>(sm + L.off_pids)[j] = kNoId;
   // token rows past the batch are zero (their logits are never stored)
   for (int i = tid; i < (kDecTok - nv) * (L.ld / 8); i += kDecThreads) {
     const int r = nv + i / (L.ld / 8), c = i % (L.ld / 8);
@@ -251,58 +320,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_forward_kernel(
                                          // slots' experts are in CTA 0
 
   // ---- the permutation, when the batch is this one cluster: CTA 0 forms
-  // counts, offsets and the stable grouping (experts ascending, slot index
-  // j = t K + k ascending inside an expert)
+  // counts, offsets and the stable grouping
   const bool permute = pm.counts != nullptr && ids != nullptr && gridDim.y == 1 && rank == 0;
-  uint32_t* pid = reinterpret_cast<uint32_t*>(sm + L.off_pids);
-  const int nk = nv * K;
-  if (permute) {
-    uint32_t* cnt = reinterpret_cast<uint32_t*>(sm + L.off_pcnt);
-    uint32_t* start = reinterpret_cast<uint32_t*>(sm + L.off_poff);
-    for (int e = tid; e < E; e += kDecThreads) cnt[e] = 0u;
-    __syncthreads();
-    for (int j = tid; j < nk; j += kDecThreads) atomicAdd(&cnt[pid[j]], 1u);
-    __syncthreads();
-    // exclusive scan over the experts: four per thread (E <= 512)
-    uint32_t v[4], sum = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = 4 * tid + i;
-      v[i] = e < E ? cnt[e] : 0u;
-      sum += v[i];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    uint32_t* wsum = reinterpret_cast<uint32_t*>(sm + L.off_poff) + 512;   // 4 words after the starts
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    uint32_t run = incl - sum;
-    for (int w2 = 0; w2 < warp; ++w2) run += wsum[w2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int e = 4 * tid + i;
-      if (e < E) {
-        start[e] = run;
-        pm.counts[e] = static_cast<int32_t>(v[i]);
-        pm.offsets[e] = run;
-      }
-      run += v[i];
-    }
-    if (tid == 0) pm.offsets[E] = nk;
-    __syncthreads();
-    for (int j = tid; j < nk; j += kDecThreads) {
-      const uint32_t e = pid[j];
-      uint32_t before = 0;                 // earlier slots of the same expert
-      for (int i = 0; i < j; ++i) before += (pid[i] == e) ? 1u : 0u;
-      const uint32_t pos = start[e] + before;
-      pm.perm[pos] = j;
-      if (pm.inv) pm.inv[j] = static_cast<int32_t>(pos);
-    }
-  }
+  if (permute)
+    group_slots<kDecThreads>(reinterpret_cast<const uint32_t*>(sm + L.off_pids), nv * K, E,
+                             reinterpret_cast<uint32_t*>(sm + L.off_pcnt),
+                             reinterpret_cast<uint32_t*>(sm + L.off_poff), pm);
 }
 
 template <int Q, bool kBias>
@@ -341,6 +364,194 @@ cudaError_t launch_dec(const void* x, const void* w, const float* bias, float* z
   return launch_pdl(kern, dim3(kDecCtas, tiles, 1), dim3(kDecThreads), L.total, s, dim3(kDecCtas, 1, 1),
                     static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w), bias, z, N,
                     d, E, K, ids, gates, alpha, pm);
+}
+
+// ---- the ticketed form of a batch of at most 16 tokens (no cluster).  The
+// router rows are spread over E/8 CTAs, so each SM brings in 8 of them
+// instead of E/16: CTA b forms the logits of experts [8b, 8b + 8) with the
+// same four quarter sums as the clustered form (the same Z bit for bit) and
+// writes them to z.  Each CTA then takes a ticket (an atomic counter in the
+// caller's workspace, zero between calls); the last one to arrive reads the
+// batch's full rows of Z back from L2 and forms the selection and the
+// grouping, then sets the counter back to zero.  No CTA waits on another.
+constexpr int kTkExperts = 8;            // experts per CTA: one n8 tile
+constexpr int kTkWarps = 8;              // selection: one token per warp at a time
+constexpr int kTkThreads = 32 * kTkWarps;
+constexpr int kTkMmaWarps = 4;           // d in quarters, as the clustered form
+
+struct TkLayout {
+  int ld;
+  uint32_t off_x, off_w, off_zp, off_beta, off_sc, sc_bytes, off_pids, off_pcnt, off_poff, off_bar, total;
+};
+
+template <int Q>
+__host__ __device__ inline TkLayout tk_layout(int d) {
+  TkLayout L;
+  L.ld = d + 8;
+  uint32_t o = 0;
+  L.off_x = o;
+  o += static_cast<uint32_t>(kDecTok * L.ld * 2);
+  L.off_w = o;
+  o += static_cast<uint32_t>(kTkExperts * L.ld * 2);
+  L.off_zp = o;
+  o += static_cast<uint32_t>(kTkMmaWarps * kDecTok * kTkExperts * 4);
+  L.off_beta = o;
+  o += static_cast<uint32_t>(128 * Q * 4);
+  L.sc_bytes = static_cast<uint32_t>((sizeof(RowScratch<Q>) + 15) & ~static_cast<size_t>(15));
+  L.off_sc = o;
+  o += kTkWarps * L.sc_bytes;
+  L.off_pids = o;                        // every slot's expert (16 tokens x K <= 16)
+  o += 4 * kDecTok * 16;
+  L.off_pcnt = o;                        // counts per expert
+  o += 4 * 512;
+  L.off_poff = o;                        // starts per expert, then one word per warp
+  o += 4 * (512 + kTkWarps);
+  L.off_bar = o;                         // mbarrier (8 bytes), then the last-CTA flag
+  o += 16;
+  L.total = o;
+  return L;
+}
+
+template <int Q, bool kBias>
+__global__ void __launch_bounds__(kTkThreads, 1) decode_ticket_kernel(
+    const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
+    const float* __restrict__ bias, float* __restrict__ z, int nv, int d, int E, int K,
+    int32_t* __restrict__ ids, float* __restrict__ gates, float* __restrict__ alpha, const DecPerm pm,
+    uint32_t* __restrict__ ticket) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const TkLayout L = tk_layout<Q>(d);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int e0 = static_cast<int>(blockIdx.x) * kTkExperts;
+  const uint32_t base = smem_u32(sm);
+  const uint32_t bar = base + L.off_bar;
+  volatile int* last_flag = reinterpret_cast<volatile int*>(sm + L.off_bar + 8);
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sm + L.off_x);
+  float* zp = reinterpret_cast<float*>(sm + L.off_zp);
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int j = tid; j < kDecTok * 16; j += kTkThreads)   // the slot list, see group_slots
+    reinterpret_cast<uint32_t*>(sm + L.off_pids)[j] = kNoId;
+  // token rows past the batch are zero (their logits are never stored)
+  for (int i = tid; i < (kDecTok - nv) * (L.ld / 8); i += kTkThreads) {
+    const int r = nv + i / (L.ld / 8), c = i % (L.ld / 8);
+    *reinterpret_cast<uint4*>(xs + r * L.ld + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncthreads();
+  pdl_wait();                            // x, the bias and the ticket follow the kernel before
+  pdl_trigger();
+  const uint32_t row_bytes = static_cast<uint32_t>(d) * 2;
+  if (warp == 0) {
+    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nv + kTkExperts) * row_bytes);
+    __syncwarp();
+    for (int r = lane; r < nv + kTkExperts; r += 32) {
+      if (r < nv)
+        bulk_row(base + L.off_x + static_cast<uint32_t>(r * L.ld * 2), x + static_cast<int64_t>(r) * d,
+                 row_bytes, bar);
+      else
+        bulk_row(base + L.off_w + static_cast<uint32_t>((r - nv) * L.ld * 2),
+                 w + static_cast<int64_t>(e0 + r - nv) * d, row_bytes, bar);
+    }
+  }
+  const bool loaded = mbar_wait(bar, 0);
+
+  // ---- logits: warp q < 4 sums k in [q d/4, (q+1) d/4) for the CTA's 8 experts
+  if (loaded && warp < kTkMmaWarps) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int kq = d / kTkMmaWarps;
+    const int k0 = warp * kq;
+    const uint32_t a_base =
+        base + L.off_x + static_cast<uint32_t>((((lane & 7) + ((lane >> 3) & 1) * 8) * L.ld + (lane >> 4) * 8 + k0) * 2);
+    const uint32_t b_base =
+        base + L.off_w + static_cast<uint32_t>(((lane & 7) * L.ld + ((lane >> 3) & 1) * 8 + k0) * 2);
+    for (int kk = 0; kk < kq; kk += 16) {
+      uint32_t a0, a1, a2, a3, b0, b1;
+      ldsm_x4(a_base + 2u * kk, a0, a1, a2, a3);
+      ldsm_x2(b_base + 2u * kk, b0, b1);
+      mma16816(acc, a0, a1, a2, a3, b0, b1);
+    }
+    float* mine = zp + warp * kDecTok * kTkExperts;
+    const int rr = lane >> 2, cc = 2 * (lane & 3);
+    mine[rr * kTkExperts + cc] = acc[0];
+    mine[rr * kTkExperts + cc + 1] = acc[1];
+    mine[(rr + 8) * kTkExperts + cc] = acc[2];
+    mine[(rr + 8) * kTkExperts + cc + 1] = acc[3];
+  }
+  __syncthreads();
+  if (loaded) {
+    constexpr int n = kDecTok * kTkExperts;
+    for (int i = tid; i < nv * kTkExperts; i += kTkThreads) {
+      const float v = __fadd_rn(__fadd_rn(__fadd_rn(zp[i], zp[n + i]), zp[2 * n + i]), zp[3 * n + i]);
+      const int r = i / kTkExperts, c = i - r * kTkExperts;
+      z[static_cast<int64_t>(r) * E + e0 + c] = v;
+    }
+  }
+  __syncthreads();                       // this CTA's logits are stored
+  if (tid == 0) {
+    __threadfence();                     // ... and visible before its ticket
+    const uint32_t C = gridDim.x;
+    const uint32_t t = atomicAdd(ticket, 1u);
+    if (t >= C) raise_status(kStatusBadInput);   // the counter was not zero at the start
+    const int last = t == C - 1;
+    if (last) {
+      __threadfence();                   // every CTA's logits before this CTA's reads
+      atomicExch(ticket, 0u);            // all C tickets are taken: zero for the next call
+    }
+    *last_flag = last;
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+
+  // ---- the last CTA: selection of every token (warp per token), then the grouping
+  float* beta_s = reinterpret_cast<float*>(sm + L.off_beta);
+  uint32_t* pid = reinterpret_cast<uint32_t*>(sm + L.off_pids);
+  if constexpr (kBias) {
+    for (int e = tid; e < 128 * Q; e += kTkThreads) beta_s[e] = e < E ? bias[e] : 0.f;
+  }
+  __syncthreads();
+  RowScratch<Q>& sc = *reinterpret_cast<RowScratch<Q>*>(sm + L.off_sc + static_cast<uint32_t>(warp) * L.sc_bytes);
+  for (int r = warp; r < nv; r += kTkWarps) {
+    float zr[4 * Q];
+    const float* zrow = z + static_cast<int64_t>(r) * E;
+#pragma unroll
+    for (int q = 0; q < Q; ++q) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(zrow + 128 * q + 4 * lane));
+      zr[4 * q + 0] = v.x;
+      zr[4 * q + 1] = v.y;
+      zr[4 * q + 2] = v.z;
+      zr[4 * q + 3] = v.w;
+    }
+    int rk;
+    uint32_t key, id;
+    warp_select_row<Q, true, kBias>(zr, beta_s, 0xffffffffu, K, lane, sc, rk, key, id);
+    if (rk >= 0 && rk < K) {
+      const uint32_t e = id < static_cast<uint32_t>(E) ? id : 0u;
+      ids[r * K + rk] = static_cast<int32_t>(id);
+      gates[r * K + rk] = gate_sigmoid(sc.row[buffer_pos<Q>(e)]);
+      pid[r * K + rk] = e;
+    }
+    if (rk == K && alpha) alpha[r] = -key_to_float(key);
+    __syncwarp();
+  }
+  __syncthreads();
+  group_slots<kTkThreads>(pid, nv * K, E, reinterpret_cast<uint32_t*>(sm + L.off_pcnt),
+                          reinterpret_cast<uint32_t*>(sm + L.off_poff), pm);
+}
+
+template <int Q, bool kBias>
+cudaError_t launch_tk(const void* x, const void* w, const float* bias, float* z, int64_t N, int d, int E,
+                      int K, int32_t* ids, float* gates, float* alpha, const DecPerm& pm, uint32_t* ticket,
+                      cudaStream_t s) {
+  const TkLayout L = tk_layout<Q>(d);
+  auto kern = decode_ticket_kernel<Q, kBias>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(L.total));
+  if (err != cudaSuccess) return err;
+  return launch_pdl(kern, dim3(static_cast<unsigned>(E / kTkExperts)), dim3(kTkThreads), L.total, s,
+                    dim3(0, 0, 0), static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w),
+                    bias, z, static_cast<int>(N), d, E, K, ids, gates, alpha, pm, ticket);
 }
 
 }  // namespace
@@ -391,6 +602,35 @@ cudaError_t launch_router_decode_permute(const void* x, const void* w, const flo
   if (!router_decode_permutes(N, d, E, K)) return cudaErrorNotSupported;
   return decode_dispatch(x, w, bias, z, N, d, E, K, ids, gates, alpha,
                          DecPerm{counts, offsets, perm, inv}, s);
+}
+
+bool router_decode_ticket_supported(int64_t N, int32_t d, int32_t E, int32_t K) {
+  if (N < 1 || N > kDecTok || E % 128 != 0 || E > 512 || d % 64 != 0 || K < 1 || K > 16) return false;
+  const int Q = E / 128;
+  const size_t total = Q == 1 ? tk_layout<1>(d).total
+                     : Q == 2 ? tk_layout<2>(d).total
+                     : Q == 3 ? tk_layout<3>(d).total
+                              : tk_layout<4>(d).total;
+  return total <= 227u * 1024u;
+}
+
+cudaError_t launch_router_decode_ticket(const void* x, const void* w, const float* bias, float* z,
+                                        int64_t N, int32_t d, int32_t E, int32_t K, int32_t* ids,
+                                        float* gates, float* alpha, int32_t* counts, int64_t* offsets,
+                                        int32_t* perm, int32_t* inv, uint32_t* ticket, cudaStream_t s) {
+  if (!router_decode_ticket_supported(N, d, E, K) || ticket == nullptr) return cudaErrorNotSupported;
+  const DecPerm pm{counts, offsets, perm, inv};
+  const bool b = bias != nullptr;
+  switch (E / 128) {
+    case 1: return b ? launch_tk<1, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, ticket, s)
+                     : launch_tk<1, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, ticket, s);
+    case 2: return b ? launch_tk<2, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, ticket, s)
+                     : launch_tk<2, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, ticket, s);
+    case 3: return b ? launch_tk<3, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, ticket, s)
+                     : launch_tk<3, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, ticket, s);
+    default: return b ? launch_tk<4, true>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, ticket, s)
+                      : launch_tk<4, false>(x, w, bias, z, N, d, E, K, ids, gates, alpha, pm, ticket, s);
+  }
 }
 
 KOLIBRI_DEFINE_STATUS_TAKE(status_take_decode)

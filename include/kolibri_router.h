@@ -85,7 +85,11 @@ enum {
 KOLIBRI_API const char *kolibri_status_string(kolibri_status status);
 
 /* Bytes of caller-provided device workspace that `op` needs for these sizes
- * (0 if the sizes are invalid).  The workspace need not be initialised. */
+ * (0 if the sizes are invalid).  The workspace need not be initialised, with
+ * one exception: a KOLIBRI_OP_PERMUTE workspace given to
+ * kolibri_router_forward_permute holds a counter that must be zero when the
+ * workspace is first used (zero-fill it once after allocating it); every call
+ * leaves the counter zero. */
 KOLIBRI_API size_t kolibri_workspace_bytes(int op, int64_t N, int32_t E, int32_t K);
 
 /*
@@ -125,12 +129,21 @@ KOLIBRI_API kolibri_status kolibri_router_forward(const void *x, const void *w, 
  * kolibri_router_forward followed by kolibri_expert_permute on its ids, in
  * one call: the arguments and outputs of both ("Kolibri Pre-Training from
  * Scratch" 6.1 and 7.1; loads and grouping 6.1/6.2).  A decode batch of at
- * most 16 tokens with E a multiple of 128 (and the router rows fitting in
- * shared memory: E/16 rows of d per CTA) takes a single launch in which one
- * 16-CTA cluster forms the logits, the selection and the grouping; other
- * batches run the forward and then the permutation.  ws / ws_bytes as for
- * kolibri_expert_permute (ignored, and may be NULL, when N*K <= 4096).
- * inv may be NULL.
+ * most 16 tokens with E a multiple of 128 takes a single launch:
+ *   - with ws (not NULL, 16-byte aligned, ws_bytes at least
+ *     kolibri_workspace_bytes(KOLIBRI_OP_PERMUTE, N, E, K)): E/8 blocks, each
+ *     forming the logits of 8 experts; the last block to finish (by a counter
+ *     in ws, which must be zero on the workspace's first use and is left
+ *     zero) forms the selection and the grouping.  A counter found nonzero
+ *     sets KOLIBRI_ERR_DEVICE in the device status word and leaves the
+ *     outputs unspecified.  The same ws must not be used by two calls that
+ *     may run at the same time.
+ *   - without ws: one 16-CTA cluster (E/16 router rows of d per CTA, which
+ *     must fit in shared memory) forms the logits, the selection and the
+ *     grouping.
+ * Z equals kolibri_router_forward's bit for bit in both forms.  Other batches
+ * run the forward and then the permutation.  ws / ws_bytes otherwise as for
+ * kolibri_expert_permute (may be NULL when N*K <= 4096).  inv may be NULL.
  */
 KOLIBRI_API kolibri_status kolibri_router_forward_permute(const void *x, const void *w,
                                                           const float *bias, float *z, int64_t N,

@@ -117,6 +117,75 @@ def test_forward_permute_equals_the_two_calls(oracle_mod, N, d, E, K, with_bias)
     assert_bit_equal(host(got[4]), c_o, "counts vs oracle")
 
 
+def _forward_permute_no_ws(x, w, b, K):
+    """kolibri_router_forward_permute with ws = NULL: a decode batch then takes
+    the clustered form."""
+    N, d = x.shape
+    E = w.shape[0]
+    f32, i32 = torch.float32, torch.int32
+    z, gates = torch.empty((N, E), dtype=f32, device="cuda"), torch.empty((N, K), dtype=f32, device="cuda")
+    ids = torch.empty((N, K), dtype=i32, device="cuda")
+    alpha = torch.empty((N,), dtype=f32, device="cuda")
+    counts = torch.empty((E,), dtype=i32, device="cuda")
+    offsets = torch.empty((E + 1,), dtype=torch.int64, device="cuda")
+    perm, inv = torch.empty((N * K,), dtype=i32, device="cuda"), torch.empty((N * K,), dtype=i32, device="cuda")
+    st = B.load().kolibri_router_forward_permute(
+        B._ptr(x), B._ptr(w), B._ptr(b), B._ptr(z), N, d, E, K, B._ptr(ids), B._ptr(gates), B._ptr(alpha),
+        B._ptr(counts), B._ptr(offsets), B._ptr(perm), B._ptr(inv), None, 0, B._stream(None))
+    assert st == B.KOLIBRI_OK, B.status_string(st)
+    return z, ids, gates, alpha, counts, offsets, perm, inv
+
+
+@pytest.mark.parametrize("N,d,E,K", [(1, 2560, 384, 6), (8, 2560, 384, 6), (16, 2560, 384, 6),
+                                     (3, 2048, 128, 8), (11, 1024, 256, 16), (16, 1024, 512, 16)])
+def test_forward_permute_decode_forms(oracle_mod, N, d, E, K):
+    # up to 16 tokens: with a workspace, E/8 blocks and a counter (the last
+    # block selects and groups); without, one 16-CTA cluster.  Both equal the
+    # forward followed by the permutation bit for bit, over three calls on
+    # one workspace (the counter goes back to zero after each)
+    ws = B.workspace(B.KOLIBRI_OP_PERMUTE, N, E, K)
+    for seed in range(3):
+        wl = workloads.Workload("t", N, d, E, K, offsets="collapsed8", beta="normal0.1", seed=seed)
+        b = dev(workloads.make_beta(wl).numpy()) if seed != 1 else None
+        x, w = workloads.make_x(wl).cuda(), workloads.make_w(wl).cuda()
+        got = B.kolibri_router_forward_permute(x, w, b, K, ws=ws)
+        clustered = _forward_permute_no_ws(x, w, b, K)
+        z, ids, gates, alpha = B.kolibri_router_forward(x, w, b, K)
+        counts, offsets, perm, inv = B.kolibri_expert_permute(ids, E)
+        torch.cuda.synchronize()
+        check_status()
+        names = ("z", "ids", "gates", "alpha", "counts", "offsets", "perm", "inv")
+        for name, a, c, r in zip(names, got, clustered, (z, ids, gates, alpha, counts, offsets, perm, inv)):
+            assert_bit_equal(host(a), host(r), name)
+            assert_bit_equal(host(c), host(r), name + " (clustered)")
+        ids_o, gates_o, alpha_o = oracle_mod.select(host(z), None if b is None else host(b), K)
+        assert_bit_equal(host(got[1]), ids_o, "ids vs oracle")
+        assert_bit_equal(host(got[2]), gates_o, "gates vs oracle")
+        assert_bit_equal(host(got[3]), alpha_o, "alpha vs oracle")
+
+
+def test_forward_permute_decode_counter_not_zero_is_reported():
+    # a workspace whose counter was never zeroed: every block's ticket is out
+    # of range, none selects, and the device status says so; zeroed, the same
+    # workspace works
+    N, d, E, K = 4, 1024, 384, 6
+    wl = workloads.Workload("t", N, d, E, K, beta="normal0.1")
+    x, w = workloads.make_x(wl).cuda(), workloads.make_w(wl).cuda()
+    b = dev(workloads.make_beta(wl).numpy())
+    ws = B.workspace(B.KOLIBRI_OP_PERMUTE, N, E, K)
+    ws.fill_(0x7F)
+    B.kolibri_router_forward_permute(x, w, b, K, ws=ws)
+    torch.cuda.synchronize()
+    assert B.kolibri_device_status() == B.KOLIBRI_ERR_DEVICE
+    ws.zero_()
+    got = B.kolibri_router_forward_permute(x, w, b, K, ws=ws)
+    z, ids, gates, alpha = B.kolibri_router_forward(x, w, b, K)
+    torch.cuda.synchronize()
+    check_status()
+    for name, a, r in zip(("z", "ids", "gates", "alpha"), got, (z, ids, gates, alpha)):
+        assert_bit_equal(host(a), host(r), name)
+
+
 def test_forward_decode_heavy_ties(oracle_mod):
     # identical router rows in a decode batch: the selection's slow path
     N, d, E, K = 40, 256, 384, 6
