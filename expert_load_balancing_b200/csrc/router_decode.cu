@@ -9,9 +9,9 @@
 //
 // A cluster of 16 CTAs owns 16 tokens and all E experts: CTA c holds the
 // full-width router rows of experts [c E/16, (c+1) E/16) and the 16 token
-// rows in shared memory (bulk copies, one memory round trip), and its four
-// warps each form the 16 x E/16 logits over a quarter of d with mma.sync
-// m16n8k16 (bf16 in, fp32 accumulate); the quarters are added in a fixed
+// rows in shared memory (bulk copies, one memory round trip), and its eight
+// warps each form the 16 x E/16 logits over an eighth of d with mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate); the eighths are added in a fixed
 // order.  After a cluster barrier CTA r takes token r: its warp 0 reads the
 // token's E logits out of the 16 CTAs' shared memory (distributed shared
 // memory) into the lane layout of the row selection (route.cuh) and writes
@@ -30,8 +30,9 @@ namespace {
 
 constexpr int kDecTok = 16;              // tokens per cluster (one m16 tile)
 constexpr int kDecCtas = 16;             // CTAs per cluster (non-portable size)
-constexpr int kDecWarps = 4;
+constexpr int kDecWarps = 8;
 constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecParts = 8;             // d is summed in 8 parts, one per warp, added in order
 
 struct DecLayout {
   int ld;                                // padded row length of x and W rows, in bf16
@@ -71,8 +72,8 @@ __host__ __device__ inline DecLayout dec_layout(int d, int E) {
   o += 4 * kDecTok * 16;
   L.off_pcnt = o;                        // CTA 0: counts per expert
   o += 4 * 512;
-  L.off_poff = o;                        // CTA 0: starts per expert
-  o += 4 * 516;
+  L.off_poff = o;                        // CTA 0: starts per expert, then one word per warp
+  o += 4 * (512 + kDecWarps);
   L.off_bar = o;
   o += 16;
   L.total = o;
@@ -135,6 +136,22 @@ __device__ __forceinline__ void bulk_row(uint32_t dst, const void* src, uint32_t
 // with NaN scores) is counted under expert 0 and reported, never used as an
 // index; cnt: E words, start: 512 words followed by one word per warp
 // (shared).  Called by all kThreads threads of the block; E <= 512.
+// The 16-wide k-steps of part w of d: [w S / 8, (w + 1) S / 8) of S = d / 16.
+// Both decode kernels use this split and add the parts in order 0..7, so
+// they form the same Z bit for bit.
+__device__ __forceinline__ void part_steps(int d, int w, int& s0, int& s1) {
+  const int S = d / 16;
+  s0 = w * S / kDecParts;
+  s1 = (w + 1) * S / kDecParts;
+}
+// ((p_0 + p_1) + p_2) + ... + p_7 of element i, part w at p + w n.
+__device__ __forceinline__ float sum_parts(const float* p, int n, int i) {
+  float v = p[i];
+#pragma unroll
+  for (int w = 1; w < kDecParts; ++w) v = __fadd_rn(v, p[w * n + i]);
+  return v;
+}
+
 template <int kThreads>
 __device__ void group_slots(const uint32_t* pid, int nk, int E, uint32_t* cnt, uint32_t* start,
                             const DecPerm& pm) {
@@ -246,24 +263,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_forward_kernel(
   }
   const bool loaded = mbar_wait(bar, 0);
 
-  // ---- logits: warp w sums k in [w d/4, (w+1) d/4)
+  // ---- logits: warp w sums part w of d (part_steps)
   if (loaded) {
     float acc[Q][4];
 #pragma unroll
     for (int j = 0; j < Q; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    const int kq = d / kDecWarps;
-    const int k0 = warp * kq;
+    int s0, s1;
+    part_steps(d, warp, s0, s1);
     const uint32_t a_base =
-        base + L.off_x + static_cast<uint32_t>((((lane & 7) + ((lane >> 3) & 1) * 8) * L.ld + (lane >> 4) * 8 + k0) * 2);
-    const uint32_t b_base =
-        base + L.off_w + static_cast<uint32_t>(((lane & 7) * L.ld + ((lane >> 3) & 1) * 8 + k0) * 2);
-    for (int kk = 0; kk < kq; kk += 16) {
+        base + L.off_x + static_cast<uint32_t>((((lane & 7) + ((lane >> 3) & 1) * 8) * L.ld + (lane >> 4) * 8) * 2);
+    const uint32_t b_base = base + L.off_w + static_cast<uint32_t>(((lane & 7) * L.ld + ((lane >> 3) & 1) * 8) * 2);
+#pragma unroll 4
+    for (int st = s0; st < s1; ++st) {
+      const uint32_t kb = 32u * static_cast<uint32_t>(st);   // 16 bf16 per step
       uint32_t a0, a1, a2, a3;
-      ldsm_x4(a_base + 2u * kk, a0, a1, a2, a3);
+      ldsm_x4(a_base + kb, a0, a1, a2, a3);
 #pragma unroll
       for (int j = 0; j < Q; ++j) {
         uint32_t b0, b1;
-        ldsm_x2(b_base + static_cast<uint32_t>(8 * j * L.ld * 2) + 2u * kk, b0, b1);
+        ldsm_x2(b_base + static_cast<uint32_t>(8 * j * L.ld * 2) + kb, b0, b1);
         mma16816(acc[j], a0, a1, a2, a3, b0, b1);
       }
     }
@@ -280,10 +298,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_forward_kernel(
   }
   __syncthreads();
   if (loaded) {
-    // the four quarters in order; then Z out
+    // the eight parts in order; then Z out
     for (int i = tid; i < kDecTok * ec; i += kDecThreads) {
-      const int n = kDecTok * ec;
-      const float v = __fadd_rn(__fadd_rn(__fadd_rn(zp[i], zp[n + i]), zp[2 * n + i]), zp[3 * n + i]);
+      const float v = sum_parts(zp, kDecTok * ec, i);
       zc[i] = v;
       const int r = i / ec, c = i - r * ec;
       if (r < nv) z[(t0 + r) * E + e0 + c] = v;
@@ -369,7 +386,7 @@ cudaError_t launch_dec(const void* x, const void* w, const float* bias, float* z
 // ---- the ticketed form of a batch of at most 16 tokens (no cluster).  The
 // router rows are spread over E/8 CTAs, so each SM brings in 8 of them
 // instead of E/16: CTA b forms the logits of experts [8b, 8b + 8) with the
-// same four quarter sums as the clustered form (the same Z bit for bit) and
+// same eight partial sums as the clustered form (the same Z bit for bit) and
 // writes them to z.  Each CTA then takes a ticket (an atomic counter in the
 // caller's workspace, zero between calls); the last one to arrive reads the
 // batch's full rows of Z back from L2 and forms the selection and the
@@ -377,7 +394,7 @@ cudaError_t launch_dec(const void* x, const void* w, const float* bias, float* z
 constexpr int kTkExperts = 8;            // experts per CTA: one n8 tile
 constexpr int kTkWarps = 8;              // selection: one token per warp at a time
 constexpr int kTkThreads = 32 * kTkWarps;
-constexpr int kTkMmaWarps = 4;           // d in quarters, as the clustered form
+constexpr int kTkMmaWarps = kDecParts;   // d in eighths, as the clustered form
 
 struct TkLayout {
   int ld;
@@ -457,19 +474,20 @@ __global__ void __launch_bounds__(kTkThreads, 1) decode_ticket_kernel(
   }
   const bool loaded = mbar_wait(bar, 0);
 
-  // ---- logits: warp q < 4 sums k in [q d/4, (q+1) d/4) for the CTA's 8 experts
+  // ---- logits: warp w sums part w of d (part_steps) for the CTA's 8 experts
   if (loaded && warp < kTkMmaWarps) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const int kq = d / kTkMmaWarps;
-    const int k0 = warp * kq;
+    int s0, s1;
+    part_steps(d, warp, s0, s1);
     const uint32_t a_base =
-        base + L.off_x + static_cast<uint32_t>((((lane & 7) + ((lane >> 3) & 1) * 8) * L.ld + (lane >> 4) * 8 + k0) * 2);
-    const uint32_t b_base =
-        base + L.off_w + static_cast<uint32_t>(((lane & 7) * L.ld + ((lane >> 3) & 1) * 8 + k0) * 2);
-    for (int kk = 0; kk < kq; kk += 16) {
+        base + L.off_x + static_cast<uint32_t>((((lane & 7) + ((lane >> 3) & 1) * 8) * L.ld + (lane >> 4) * 8) * 2);
+    const uint32_t b_base = base + L.off_w + static_cast<uint32_t>(((lane & 7) * L.ld + ((lane >> 3) & 1) * 8) * 2);
+#pragma unroll 4
+    for (int st = s0; st < s1; ++st) {
+      const uint32_t kb = 32u * static_cast<uint32_t>(st);   // 16 bf16 per step
       uint32_t a0, a1, a2, a3, b0, b1;
-      ldsm_x4(a_base + 2u * kk, a0, a1, a2, a3);
-      ldsm_x2(b_base + 2u * kk, b0, b1);
+      ldsm_x4(a_base + kb, a0, a1, a2, a3);
+      ldsm_x2(b_base + kb, b0, b1);
       mma16816(acc, a0, a1, a2, a3, b0, b1);
     }
     float* mine = zp + warp * kDecTok * kTkExperts;
@@ -483,7 +501,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) decode_ticket_kernel(
   if (loaded) {
     constexpr int n = kDecTok * kTkExperts;
     for (int i = tid; i < nv * kTkExperts; i += kTkThreads) {
-      const float v = __fadd_rn(__fadd_rn(__fadd_rn(zp[i], zp[n + i]), zp[2 * n + i]), zp[3 * n + i]);
+      const float v = sum_parts(zp, n, i);
       const int r = i / kTkExperts, c = i - r * kTkExperts;
       z[static_cast<int64_t>(r) * E + e0 + c] = v;
     }
@@ -604,8 +622,11 @@ cudaError_t launch_router_decode_permute(const void* x, const void* w, const flo
                          DecPerm{counts, offsets, perm, inv}, s);
 }
 
+// Only where the forward itself takes the clustered kernel: the two forms
+// share their sums, so Z is the forward's bit for bit.
 bool router_decode_ticket_supported(int64_t N, int32_t d, int32_t E, int32_t K) {
   if (N < 1 || N > kDecTok || E % 128 != 0 || E > 512 || d % 64 != 0 || K < 1 || K > 16) return false;
+  if (!router_decode_supported(N, d, E, K)) return false;
   const int Q = E / 128;
   const size_t total = Q == 1 ? tk_layout<1>(d).total
                      : Q == 2 ? tk_layout<2>(d).total

@@ -129,7 +129,9 @@ KOLIBRI_API kolibri_status kolibri_router_forward(const void *x, const void *w, 
  * kolibri_router_forward followed by kolibri_expert_permute on its ids, in
  * one call: the arguments and outputs of both ("Kolibri Pre-Training from
  * Scratch" 6.1 and 7.1; loads and grouping 6.1/6.2).  A decode batch of at
- * most 16 tokens with E a multiple of 128 takes a single launch:
+ * most 16 tokens with E a multiple of 128, whose E/16 router rows of d and 16
+ * token rows fit in one CTA's shared memory (as for kolibri_router_forward's
+ * one-launch form), takes a single launch:
  *   - with ws (not NULL, 16-byte aligned, ws_bytes at least
  *     kolibri_workspace_bytes(KOLIBRI_OP_PERMUTE, N, E, K)): E/8 blocks, each
  *     forming the logits of 8 experts; the last block to finish (by a counter
@@ -138,9 +140,8 @@ KOLIBRI_API kolibri_status kolibri_router_forward(const void *x, const void *w, 
  *     sets KOLIBRI_ERR_DEVICE in the device status word and leaves the
  *     outputs unspecified.  The same ws must not be used by two calls that
  *     may run at the same time.
- *   - without ws: one 16-CTA cluster (E/16 router rows of d per CTA, which
- *     must fit in shared memory) forms the logits, the selection and the
- *     grouping.
+ *   - without ws: one 16-CTA cluster (E/16 router rows per CTA) forms the
+ *     logits, the selection and the grouping.
  * Z equals kolibri_router_forward's bit for bit in both forms.  Other batches
  * run the forward and then the permutation.  ws / ws_bytes otherwise as for
  * kolibri_expert_permute (may be NULL when N*K <= 4096).  inv may be NULL.

@@ -137,12 +137,15 @@ def _forward_permute_no_ws(x, w, b, K):
 
 
 @pytest.mark.parametrize("N,d,E,K", [(1, 2560, 384, 6), (8, 2560, 384, 6), (16, 2560, 384, 6),
-                                     (3, 2048, 128, 8), (11, 1024, 256, 16), (16, 1024, 512, 16)])
+                                     (3, 2048, 128, 8), (11, 1024, 256, 16), (16, 1024, 512, 16),
+                                     (2, 4096, 128, 6), (3, 2560, 512, 6), (5, 2624, 384, 6)])
 def test_forward_permute_decode_forms(oracle_mod, N, d, E, K):
     # up to 16 tokens: with a workspace, E/8 blocks and a counter (the last
     # block selects and groups); without, one 16-CTA cluster.  Both equal the
     # forward followed by the permutation bit for bit, over three calls on
-    # one workspace (the counter goes back to zero after each)
+    # one workspace (the counter goes back to zero after each).  The last two
+    # shapes do not fit the cluster's shared memory: the forward takes the
+    # small-batch kernels, and so does this call
     ws = B.workspace(B.KOLIBRI_OP_PERMUTE, N, E, K)
     for seed in range(3):
         wl = workloads.Workload("t", N, d, E, K, offsets="collapsed8", beta="normal0.1", seed=seed)
