@@ -52,6 +52,19 @@ def test_workspace_sizes(kolibri_lib):
     assert B.kolibri_workspace_bytes(B.KOLIBRI_OP_PERMUTE, 1 << 20, 384, 6) > 0
 
 
+def test_binding_workspace_is_zero_filled(kolibri_lib):
+    # the decode form of kolibri_router_forward_permute keeps a counter in the
+    # permutation workspace that must be zero on first use: the binding's
+    # buffers start zeroed, and a decode batch still gets a workspace
+    from expert_load_balancing_b200 import binding as B
+    for N in (1, 16, 4096):
+        need = B.kolibri_workspace_bytes(B.KOLIBRI_OP_PERMUTE, N, 384, 6)
+        assert need > 0
+        ws = B.workspace(B.KOLIBRI_OP_PERMUTE, N, 384, 6, device="cpu")
+        assert ws.numel() >= need and ws.dtype.itemsize == 1
+        assert int(ws.count_nonzero()) == 0
+
+
 def _call(lib, name, *args):
     return getattr(lib, name)(*args)
 
